@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Decode-step throughput of the SOCKET hot path on B200.
+
+One step = one socket_decode call for all B x Hq query heads of one layer:
+soft tables -> scoring -> top-k -> sparse attention (four kernels).  Inputs
+(the bucket-id index, value norms, K/V cache, queries) are resident in HBM
+before the timed region; steps rotate over several independently drawn
+layers, so consecutive steps share no data and every step's inputs exceed
+the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl socket|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU
+workload on its own data (weak scaling, no collective on the data path);
+timing is the max over ranks of the device time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the only reference this method has)
+on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as wl  # noqa: E402
+
+METRIC = "SOCKET decode steps/sec at 128K ctx; HBM GB/s vs roofline (1×B200)"
+UNIT = "steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6650 GB/s (earlier measurement on this pool)"
+
+
+def profiled_traffic(kernel: str, workload: str, src_files):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    is unchanged since the counters were taken; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for s in src_files:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    if rec.get("source_sha256") != h.hexdigest() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch_full")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml = pynvml
+            self.handle = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing or inaccessible
+            self.error = f"{type(e).__name__}: {e}"
+
+    def _sample(self):
+        nv = self.nvml
+        mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+        self.samples.append(mhz)
+        self.reasons |= int(r) & ~0x1
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.error is None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if self.error is not None and not self.samples:
+            return {"error": self.error}
+        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": float(self.max_mhz), "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_decode_timing(w, K, V, q, W, units_kvh, min_seconds=2.0, reps_max=50):
+    """Hash the sampled units with the oracle (untimed), then time the oracle
+    decode of those units (OpenMP across units).  K, V: [Hkv, Ncap, d] CPU
+    tensors of one batch row; q: [Hq, d].  Returns (seconds per rep, units, threads)."""
+    import oracle
+    S = len(units_kvh)
+    ids = np.zeros((S, w.L, w.ncap), dtype=np.uint8)
+    vn = np.zeros((S, w.ncap), dtype=np.float32)
+    for i, h in enumerate(units_kvh):
+        a, v, _ = oracle.hash_keys(K[h, : w.N], V[h, : w.N], W, w.L, w.P)
+        ids[i, :, : w.N] = a
+        vn[i, : w.N] = v.astype(np.float32)
+    qs = torch.stack([q[h * w.G:(h + 1) * w.G] for h in units_kvh])
+    Ks = torch.stack([K[h] for h in units_kvh])
+    Vs = torch.stack([V[h] for h in units_kvh])
+    threads = min(S, oracle.max_threads())
+    oracle.set_num_threads(threads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode(qs, W, w.L, w.P, w.tau, ids, vn, Ks, Vs, w.N, w.k, want_scores=False)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= reps_max:
+            break
+    return el / reps, S, threads
+
+
+def cpu_baseline(w, inp):
+    units = list(range(min(w.Hkv, 8)))
+    K = inp["K"][0].cpu()
+    V = inp["V"][0].cpu()
+    t, S, threads = oracle_decode_timing(w, K, V, inp["q"][0].cpu(), inp["W"].cpu(), units)
+    value = 1.0 / (t * w.U / S)
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{S} of {w.U} (batch, kv-head) units at full N={w.N}, oracle decode (soft tables, scores, "
+                      f"top-k, attention) in fp64, {t * 1e3:.1f} ms per sample; steps/s scaled by {w.U}/{S}"}
+
+
+def run_reference(args, world: int, rank: int):
+    if rank != 0:
+        return 0
+    import oracle
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w, "cpu", batches=[0])
+    S = min(w.Hkv, oracle.max_threads())
+    units = list(range(S))
+    K, V, q, W = inp["K"][0], inp["V"][0], inp["q"][0], inp["W"]
+    import oracle as orc
+    ids = np.zeros((S, w.L, w.ncap), dtype=np.uint8)
+    vn = np.zeros((S, w.ncap), dtype=np.float32)
+    for i, h in enumerate(units):
+        a, v, _ = orc.hash_keys(K[h, : w.N], V[h, : w.N], W, w.L, w.P)
+        ids[i, :, : w.N] = a
+        vn[i, : w.N] = v.astype(np.float32)
+    qs = torch.stack([q[h * w.G:(h + 1) * w.G] for h in units])
+    Ks, Vs = K[:S].contiguous(), V[:S].contiguous()
+    orc.set_num_threads(S)
+    step = lambda: orc.decode(qs, W, w.L, w.P, w.tau, ids, vn, Ks, Vs, w.N, w.k, want_scores=False)
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    per_sample = el / max(args.steps, 1)
+    value = 1.0 / (per_sample * w.U / S)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_sample * w.U / S * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "L": w.L,
+                   "P": w.P, "tau": w.tau, "k": w.k, "kv_dtype": w.dtype},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": S, "kind": "oracle",
+                         "sample": f"each step: oracle decode of {S} of {w.U} units at full N={w.N} "
+                                   f"(OpenMP over units), scaled by {w.U}/{S}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# the CUDA path
+# ----------------------------------------------------------------------------
+
+def run_socket(args, world: int, rank: int, local_rank: int):
+    import soft_lsh_top_b200 as sk
+    from soft_lsh_top_b200 import _build
+    _build.build()  # no-op when the in-tree library is current
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    w = wl.WORKLOADS[args.workload]
+    R = args.layers
+    layers = []
+    for li in range(R):
+        wi = w.scaled(seed=w.seed + 1000 * li + 7919 * rank)
+        inp = wl.make_inputs(wi, dev)
+        ids, vn = sk.alloc_cache_index(w.B, w.Hkv, w.ncap, w.L, dev)
+        sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vn, 0, w.N)
+        layers.append((inp, ids, vn))
+    torch.cuda.synchronize()
+    ws, idx, out = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, dev)
+
+    def step(s, q=None):
+        inp, ids, vn = layers[s % R]
+        sk.socket_decode(inp["q"] if q is None else q, inp["W"], ids, vn, inp["K"], inp["V"], w.N, w.tau, w.k,
+                         ws, idx, out)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-kernel events recorded by the library.
+    K = args.steps
+    nk = 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        start.record()
+        for s in range(K):
+            sk.socket_set_step_events(evs[s])
+            step(s)
+        end.record()
+        torch.cuda.synchronize()
+    sk.socket_set_step_events([])
+    barrier(world)
+    ms_total = max_over_ranks(start.elapsed_time(end), world)
+    names = ["soft_tables", "score", "topk", "attention"]
+    kern_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(K))
+               for i, n in enumerate(names)}
+    assert sk.read_device_error(ws) == 0
+
+    # ---- end to end through the public API with host buffers.
+    q_host = [torch.empty_like(l[0]["q"], device="cpu").pin_memory() for l in layers]
+    for l, qh in zip(layers, q_host):
+        qh.copy_(l[0]["q"])
+    q_dev = torch.empty_like(layers[0][0]["q"])
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    idx_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    for s in range(args.warmup):
+        q_dev.copy_(q_host[s % R], non_blocking=True)
+        step(s, q_dev)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(K):
+        q_dev.copy_(q_host[s % R], non_blocking=True)
+        step(s, q_dev)
+        out_host.copy_(out, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = q_dev.numel() * q_dev.element_size()
+    d2h = out.numel() * out.element_size() + idx.numel() * idx.element_size()
+
+    result = None
+    if rank == 0:
+        ms_step = ms_total / K
+        bytes_step = w.step_bytes()
+        peak, peak_src = hbm_peak()
+        score_bytes = w.U * w.N * (w.L + 4)
+        score_gbs = score_bytes / (kern_ms["score"] * 1e-3) / 1e9
+        attn_bytes = w.U * 2 * w.k * w.d * w.elem_bytes
+        traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
+                                                            "soft_lsh_top_b200/csrc/common.cuh"])
+        result = {
+            "metric": METRIC, "value": world * K / (ms_total * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "L": w.L,
+                       "P": w.P, "tau": w.tau, "k": w.k, "kv_dtype": w.dtype, "parallelism": f"replicas{world}",
+                       "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB per step, {R} rotating layers "
+                             "of independent data", "launch": "direct C-ABI calls, one stream"},
+            "bytes_per_step": bytes_step,
+            "step_hbm_gbs": bytes_step / (ms_step * 1e-3) / 1e9,
+            "step_roofline_frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak,
+            "kernels_ms": kern_ms,
+            "roofline": {"bound": "hbm", "kernel": "score_kernel", "achieved": score_gbs, "peak": peak,
+                         "unit": "GB/s", "frac": score_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": score_bytes, "peak_source": peak_src,
+                         "attention_gbs": attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9},
+            "gpu_launches": nk * K,
+            "clocks": clocks.summary(),
+            "e2e": {"value": world * K / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(w, layers[0][0])
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["socket", "reference"], default="socket")
+    ap.add_argument("--workload", default=wl.BATCH8_128K.name, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--layers", type=int, default=3, help="independently drawn layers rotated across steps")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_socket(args, world, rank, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

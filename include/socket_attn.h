@@ -1,0 +1,173 @@
+/*
+ * socket_attn.h -- C ABI of the SOCKET decode hot path on NVIDIA B200 (sm_100a).
+ *
+ * SOCKET (SOft Collision Kernel EsTimator) replaces dense decode attention by
+ * attention over the k keys with the largest "soft collision" score.  The
+ * method, as summarised on
+ *   [ES] "Resumen Técnico: SOCKET - Estimador de Núcleo de Colisión Suave para
+ *        Atención Escasa" (gist.science/es/paper/2602.06283),
+ *        "Metodología: SOCKET" > "Mecanismo Central: LSH Suave", steps 1-4;
+ *   [DE] "SOCKET: SOft Collision Kernel EsTimator for Sparse Attention"
+ *        (gist.science/de/paper/2602.06283), "Technische Zusammenfassung" >
+ *        "Methodik: SOCKET" > "Kernmechanismus: Soft LSH",
+ * has a prefill part (hash every key into L tables, cache value norms) and a
+ * decode part (soft-assign the query, score keys, select top-k, attend).
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named "device" are device memory (cudaMalloc'ed, e.g. by
+ *     PyTorch) owned by the caller.  The library never allocates or frees.
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  It never synchronises the
+ *     host.  A non-OK status means nothing was launched, except SOCKET_ECUDA
+ *     after a launch error; outputs are then undefined.
+ *   - No exceptions, device traps or device asserts.  Host-side checks reject
+ *     bad arguments before any launch; socket_last_error() explains why.
+ *   - Element types: SOCKET_F32 (IEEE binary32) or SOCKET_BF16 (bfloat16).
+ *   - Tensor layouts are dense, row-major, innermost dimension last.
+ *   - Head dimension d must be 128.  B, Hq, Hkv, N, Ncap are int64.
+ *   - Units: a (batch row, kv head) pair is a "unit"; U = B * Hkv.  The Hq/Hkv
+ *     query heads of a unit (grouped-query attention) share one selection.
+ */
+#ifndef SOCKET_ATTN_H
+#define SOCKET_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define SOCKET_OK            0  /* success (work queued on the stream)            */
+#define SOCKET_EINVAL        1  /* bad argument: null pointer, size, alignment    */
+#define SOCKET_EUNSUPPORTED  2  /* valid but not built: d != 128, P > 8, ...      */
+#define SOCKET_ECUDA         3  /* a CUDA launch failed; message has the reason   */
+#define SOCKET_EWORKSPACE    4  /* workspace too small or misaligned              */
+
+/* Element types. */
+#define SOCKET_F32  0
+#define SOCKET_BF16 1
+
+/* Limits. */
+#define SOCKET_HEAD_DIM   128
+#define SOCKET_MAX_P      8    /* bucket ids are one byte: 2^P <= 256 buckets */
+#define SOCKET_MAX_L      128
+#define SOCKET_MAX_GROUP  16   /* Hq / Hkv */
+
+/*
+ * Device error word.  The first 4 bytes of the decode workspace hold a word
+ * that socket_decode clears at its start and that a kernel sets (bitwise OR)
+ * when one of its bounded waits expires (it then skips its work and leaves
+ * its outputs undefined).  The host may read it after the stream has drained;
+ * 0 means every wait completed.
+ */
+#define SOCKET_WS_ERROR_OFFSET 0
+#define SOCKET_DEVERR_GATHER_TIMEOUT 0x1u
+
+/*
+ * socket_hash_keys -- prefill hashing ([ES] step 1 "Pre-cálculo (Prellenado)";
+ * [DE] "Vorverarbeitung (Prefill)").  Keys are hashed into L independent
+ * tables by random projection, one bucket id per table, and the value norms
+ * are cached:
+ *     id_l(k)  = sum_{p<P} [ <W_{l,p}, k> > 0 ] * 2^p      (bit p <-> plane p)
+ *     vnorm(k) = ||v||_2
+ * Only keys n_begin <= n < n_end of every unit are written, so the same call
+ * hashes a whole prefill (0, N) or appends one decode-step key (N, N + 1).
+ *
+ *   K, V      device, [B][Hkv][Ncap][d] of kv_dtype, 16-byte aligned.
+ *   W         device, [L][P][d] bfloat16 bits (one set of hyperplanes shared
+ *             by every batch row and head), 16-byte aligned.
+ *   ids       device out, [B][Hkv][L][Ncap] uint8 (table-major per unit),
+ *             16-byte aligned.
+ *   vnorm     device out, [B][Hkv][Ncap] float32, 16-byte aligned.
+ * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Ncap % 16 == 0;
+ * 0 <= n_begin <= n_end <= Ncap.  n_begin == n_end queues nothing.
+ * Bucket ids are exact except where some |<W_{l,p}, k>| is within float32
+ * accumulation error of 0 (below ~1e-6 * ||k|| for d = 128).
+ */
+int socket_hash_keys(const void* K, const void* V, int kv_dtype,
+                     int64_t B, int64_t Hkv, int64_t Ncap,
+                     int64_t n_begin, int64_t n_end, int64_t d,
+                     const uint16_t* W, int L, int P,
+                     uint8_t* ids, float* vnorm, void* stream);
+
+/*
+ * socket_decode_workspace_size -- bytes of device scratch socket_decode needs
+ * for these sizes (0 if the sizes are invalid).  The workspace needs no
+ * initialisation, must be 256-byte aligned, and may be reused by later calls
+ * on the same stream; calls that overlap in time need separate workspaces.
+ */
+size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
+                                    int64_t d, int L, int P, int k);
+
+/*
+ * socket_decode -- one decode step for all B*Hq query heads of one layer
+ * ([ES] steps 2-4 "Asignación Suave", "Puntuación", "Selección"; [DE] "Weiche
+ * Zuweisung (Decoding)", "Bewertung", "Auswahl"):
+ *   1. soft assignment: z_{h,l} = W_l q_h / ||q_h|| (z = 0 if q_h = 0), and
+ *      p_{h,l}(b) = softmax over the 2^P sign patterns s_b of <s_b, z_{h,l}>/tau,
+ *      which factorises to prod_p sigmoid(2 s_{b,p} z_{h,l,p} / tau);
+ *      evaluated in float64, rounded once to float32.
+ *   2. soft collision score of every live key n < N of a unit, summed over
+ *      the unit's query heads:
+ *         score(n) = vnorm(n) * sum_l sum_h p_{h,l}(id_l(n))      (float32)
+ *   3. deterministic top-k: the k keys of largest score, equal scores going
+ *      to the lower index; written in ascending index order.
+ *   4. exact softmax attention of every query head of the unit over its k
+ *      selected keys, with scale 1/sqrt(d); float32 output.
+ *
+ *   q          device, [B][Hq][d] of q_dtype, 16-byte aligned.
+ *   W          device, [L][P][d] bfloat16 bits (the same as for hashing).
+ *   ids, vnorm device, as written by socket_hash_keys.
+ *   K, V       device, [B][Hkv][Ncap][d] of kv_dtype, 16-byte aligned.
+ *   N          live keys per unit (the same for every unit), k <= N <= Ncap.
+ *   tau        temperature, finite and > 0.
+ *   workspace  device scratch of >= socket_decode_workspace_size() bytes,
+ *              256-byte aligned.
+ *   idx_out    device out, [B][Hkv][k] int32, ascending per unit.
+ *   out        device out, [B][Hq][d] float32, 16-byte aligned.
+ *   scores_out device out or NULL, [B][Hkv][Ncap] float32, 16-byte aligned:
+ *              if given, the scores of step 2 land here (entries n >= N are
+ *              unspecified).
+ * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Hq % Hkv == 0;
+ * 1 <= Hq / Hkv <= 16; Ncap % 16 == 0; 1 <= k <= N <= Ncap; N < 2^31.
+ * Inputs must be finite; non-finite values give an unspecified selection.
+ */
+int socket_decode(const void* q, int q_dtype, const uint16_t* W,
+                  const uint8_t* ids, const float* vnorm,
+                  const void* K, const void* V, int kv_dtype,
+                  int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d,
+                  int L, int P, double tau, int k,
+                  void* workspace, size_t workspace_bytes,
+                  int32_t* idx_out, float* out, float* scores_out, void* stream);
+
+/*
+ * socket_last_error -- message for the last non-OK status returned on the
+ * calling host thread ("" if none).  The pointer stays valid until the next
+ * call on that thread.
+ */
+const char* socket_last_error(void);
+
+/*
+ * socket_set_step_events -- timing diagnostics.  Until called again with
+ * n = 0, every socket_decode call made on the calling host thread records
+ * events[0] on its stream before its first kernel and events[i] after its
+ * i-th kernel, for i = 1 .. min(n - 1, SOCKET_DECODE_KERNELS).  The events
+ * are cudaEvent_t handles (passed as void*) that the caller created and
+ * reads with cudaEventElapsedTime; the library only records them.  Inside a
+ * stream capture they are recorded as external event nodes.  Returns
+ * SOCKET_EINVAL if n < 0, n > SOCKET_DECODE_KERNELS + 1, or a handle is NULL.
+ * The kernels, in order: soft tables, scoring, top-k, attention.
+ */
+#define SOCKET_DECODE_KERNELS 4
+int socket_set_step_events(void* const* events, int n);
+
+/* socket_version -- ABI version of this library (major * 100 + minor). */
+int socket_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SOCKET_ATTN_H */

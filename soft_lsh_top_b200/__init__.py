@@ -1,0 +1,227 @@
+"""SOCKET decode hot path on B200: Python binding of ``libsocket_attn.so``.
+
+The functions here only marshal arguments into the C ABI declared in
+``include/socket_attn.h`` (same names): they check that torch tensors have the
+shapes, dtypes, devices and layouts the C side assumes, pass raw pointers and
+sizes, and turn a non-zero status into ``SocketError``.  Every step of the
+method runs in the library's CUDA kernels; there is no Python or CPU
+implementation to fall back on, and importing a call fails loudly when the
+library has not been built (``python -m soft_lsh_top_b200._build``).
+
+PyTorch provides device memory and streams only.  Calls are asynchronous on
+the current torch stream unless ``stream`` (a ``torch.cuda.Stream``) is given.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_workspace_size",
+    "socket_last_error", "socket_version", "socket_set_step_events", "library_path", "load_library",
+    "alloc_cache_index", "alloc_decode_buffers",
+]
+
+SOCKET_OK, SOCKET_EINVAL, SOCKET_EUNSUPPORTED, SOCKET_ECUDA, SOCKET_EWORKSPACE = range(5)
+SOCKET_F32, SOCKET_BF16 = 0, 1
+HEAD_DIM = 128
+WS_ERROR_OFFSET = 0
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsocket_attn.so")
+_lib = None
+
+_i64, _int, _dbl, _vp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_size_t
+
+_STATUS = {1: "EINVAL", 2: "EUNSUPPORTED", 3: "ECUDA", 4: "EWORKSPACE"}
+
+
+class SocketError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"SOCKET_{_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library(path: str | None = None):
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or _LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"SOCKET CUDA library missing at {p}; build it with "
+                           "`python -m soft_lsh_top_b200._build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(p)
+    lib.socket_hash_keys.argtypes = [_vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp]
+    lib.socket_hash_keys.restype = _int
+    lib.socket_decode_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]
+    lib.socket_decode_workspace_size.restype = _sz
+    lib.socket_decode.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64,
+                                  _int, _int, _dbl, _int, _vp, _sz, _vp, _vp, _vp, _vp]
+    lib.socket_decode.restype = _int
+    lib.socket_last_error.argtypes = []
+    lib.socket_last_error.restype = ctypes.c_char_p
+    lib.socket_set_step_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _int]
+    lib.socket_set_step_events.restype = _int
+    lib.socket_version.argtypes = []
+    lib.socket_version.restype = _int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def socket_last_error() -> str:
+    return load_library().socket_last_error().decode()
+
+
+def socket_version() -> int:
+    return int(load_library().socket_version())
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+
+def _code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SOCKET_BF16
+    if t.dtype == torch.float32:
+        return SOCKET_F32
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _raise(status: int):
+    if status != SOCKET_OK:
+        raise SocketError(status, socket_last_error())
+
+
+# ----------------------------------------------------------------------------
+# the C ABI
+# ----------------------------------------------------------------------------
+
+def socket_hash_keys(K: torch.Tensor, V: torch.Tensor, W: torch.Tensor, ids: torch.Tensor,
+                     vnorm: torch.Tensor, n_begin: int = 0, n_end: int | None = None, stream=None) -> None:
+    """Hash keys [n_begin, n_end) of every unit into ``ids`` and ``vnorm``.
+
+    K, V: [B, Hkv, Ncap, 128] (float32 or bfloat16); W: [L, P, 128] bfloat16;
+    ids: [B, Hkv, L, Ncap] uint8; vnorm: [B, Hkv, Ncap] float32.
+    """
+    lib = load_library()
+    B, Hkv, Ncap, d = K.shape
+    L, P, _ = W.shape
+    dev = K.device
+    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
+    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
+    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
+    _check(ids, "ids", (B, Hkv, L, Ncap), dtype=torch.uint8, device=dev)
+    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    n_end = Ncap if n_end is None else int(n_end)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_hash_keys(K.data_ptr(), V.data_ptr(), _code(K), B, Hkv, Ncap, int(n_begin), n_end, d,
+                                    W.data_ptr(), L, P, ids.data_ptr(), vnorm.data_ptr(), _stream_handle(stream)))
+
+
+def socket_decode_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, d: int, L: int, P: int, k: int) -> int:
+    n = int(load_library().socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k))
+    if n == 0:
+        raise ValueError("invalid sizes for socket_decode")
+    return n
+
+
+def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
+                  K: torch.Tensor, V: torch.Tensor, N: int, tau: float, k: int,
+                  workspace: torch.Tensor, idx_out: torch.Tensor, out: torch.Tensor,
+                  scores_out: torch.Tensor | None = None, stream=None) -> None:
+    """One decode step (soft assignment, scoring, top-k, sparse attention).
+
+    q: [B, Hq, 128]; W: [L, P, 128] bfloat16; ids: [B, Hkv, L, Ncap] uint8;
+    vnorm: [B, Hkv, Ncap] float32; K, V: [B, Hkv, Ncap, 128];
+    workspace: uint8 tensor of >= socket_decode_workspace_size() bytes;
+    idx_out: [B, Hkv, k] int32; out: [B, Hq, 128] float32;
+    scores_out: optional [B, Hkv, Ncap] float32.
+    """
+    lib = load_library()
+    B, Hq, d = q.shape
+    _, Hkv, Ncap, _ = K.shape
+    L, P, _ = W.shape
+    dev = q.device
+    _check(q, "q", (B, Hq, d), device=dev)
+    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
+    _check(ids, "ids", (B, Hkv, L, Ncap), dtype=torch.uint8, device=dev)
+    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
+    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
+    _check(idx_out, "idx_out", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1 or not workspace.is_cuda or workspace.device != dev:
+        raise ValueError("workspace must be a 1-D uint8 CUDA tensor on the inputs' device")
+    if scores_out is not None:
+        _check(scores_out, "scores_out", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_decode(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(),
+                                 K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P,
+                                 float(tau), int(k), workspace.data_ptr(), workspace.numel(),
+                                 idx_out.data_ptr(), out.data_ptr(),
+                                 scores_out.data_ptr() if scores_out is not None else None,
+                                 _stream_handle(stream)))
+
+
+def socket_set_step_events(events) -> None:
+    """Register torch.cuda.Event objects (created with enable_timing=True) that
+    every later socket_decode on this thread records around its kernels;
+    an empty list turns the recording off."""
+    lib = load_library()
+    n = len(events)
+    arr = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(int(e.cuda_event)) for e in events])
+    _raise(lib.socket_set_step_events(arr, n))
+
+
+# ----------------------------------------------------------------------------
+# allocation helpers (torch owns the memory)
+# ----------------------------------------------------------------------------
+
+def alloc_cache_index(B: int, Hkv: int, Ncap: int, L: int, device) -> tuple[torch.Tensor, torch.Tensor]:
+    """Bucket-id and value-norm buffers for a cache of Ncap keys per unit."""
+    ids = torch.empty(B, Hkv, L, Ncap, dtype=torch.uint8, device=device)
+    vnorm = torch.empty(B, Hkv, Ncap, dtype=torch.float32, device=device)
+    return ids, vnorm
+
+
+def alloc_decode_buffers(B: int, Hq: int, Hkv: int, Ncap: int, L: int, P: int, k: int, device):
+    """(workspace, idx_out, out) for socket_decode at these sizes."""
+    ws = torch.empty(socket_decode_workspace_size(B, Hq, Hkv, Ncap, HEAD_DIM, L, P, k), dtype=torch.uint8,
+                     device=device)
+    idx = torch.empty(B, Hkv, k, dtype=torch.int32, device=device)
+    out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=device)
+    return ws, idx, out
+
+
+def read_device_error(workspace: torch.Tensor) -> int:
+    """The device error word of a decode workspace (synchronises the stream)."""
+    return int(workspace[WS_ERROR_OFFSET:WS_ERROR_OFFSET + 4].view(torch.int32).item())

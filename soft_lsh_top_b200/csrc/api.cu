@@ -1,0 +1,222 @@
+// C ABI of the SOCKET library: argument checks, workspace layout, launches.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "internal.h"
+#include "socket_attn.h"
+
+namespace socket_attn {
+namespace {
+
+thread_local std::string g_last_error;
+thread_local cudaEvent_t g_step_events[SOCKET_DECODE_KERNELS + 1];
+thread_local int g_num_step_events = 0;
+
+// Records diagnostic step event i (if registered) on the stream.
+cudaError_t mark_step(int i, cudaStream_t stream)
+{
+    if (i >= g_num_step_events) return cudaSuccess;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return e;
+    return cudaEventRecordWithFlags(g_step_events[i], stream,
+                                    cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : 0);
+}
+
+int fail(int status, const char* fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+int cuda_status(cudaError_t e, const char* what)
+{
+    if (e == cudaSuccess) return SOCKET_OK;
+    return fail(SOCKET_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Shape checks shared by both entry points; returns SOCKET_OK or a status.
+int check_common(int64_t B, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P)
+{
+    if (d != SOCKET_HEAD_DIM) return fail(SOCKET_EUNSUPPORTED, "head dim d=%lld unsupported (only 128)", (long long)d);
+    if (P < 1 || P > SOCKET_MAX_P) return fail(SOCKET_EUNSUPPORTED, "P=%d outside [1, 8]", P);
+    if (L < 1 || L > SOCKET_MAX_L) return fail(SOCKET_EUNSUPPORTED, "L=%d outside [1, 128]", L);
+    if (B < 1 || Hkv < 1) return fail(SOCKET_EINVAL, "B=%lld and Hkv=%lld must be >= 1", (long long)B, (long long)Hkv);
+    if (B * Hkv > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hkv=%lld above 65535", (long long)(B * Hkv));
+    if (Ncap < 16 || Ncap % 16 != 0) return fail(SOCKET_EINVAL, "Ncap=%lld must be a positive multiple of 16", (long long)Ncap);
+    if (Ncap >= (int64_t(1) << 31)) return fail(SOCKET_EUNSUPPORTED, "Ncap=%lld must be < 2^31", (long long)Ncap);
+    return SOCKET_OK;
+}
+
+bool valid_dtype(int t) { return t == SOCKET_F32 || t == SOCKET_BF16; }
+
+int fill_shape(DecodeShape& s, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d, int L, int P,
+               int k)
+{
+    int st = check_common(B, Hkv, Ncap, d, L, P);
+    if (st != SOCKET_OK) return st;
+    if (Hq < 1 || Hq % Hkv != 0) return fail(SOCKET_EINVAL, "Hq=%lld must be a positive multiple of Hkv=%lld", (long long)Hq, (long long)Hkv);
+    if (Hq / Hkv > SOCKET_MAX_GROUP) return fail(SOCKET_EUNSUPPORTED, "group size Hq/Hkv=%lld above 16", (long long)(Hq / Hkv));
+    if (k < 1) return fail(SOCKET_EINVAL, "k=%d must be >= 1", k);
+    if (N < k || N > Ncap) return fail(SOCKET_EINVAL, "need k <= N <= Ncap (k=%d N=%lld Ncap=%lld)", k, (long long)N, (long long)Ncap);
+    s.B = B;
+    s.Hq = Hq;
+    s.Hkv = Hkv;
+    s.Ncap = Ncap;
+    s.N = N;
+    s.d = d;
+    s.L = L;
+    s.P = P;
+    s.k = k;
+    s.G = (int)(Hq / Hkv);
+    s.U = B * Hkv;
+    s.NB = 1 << P;
+    s.nsplit = 0;
+    return SOCKET_OK;
+}
+
+}  // namespace
+
+DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
+{
+    DecodeWorkspace w;
+    size_t off = 0;
+    w.err = off;
+    off = align256(off + 4);
+    w.counters = off;
+    off = align256(off + 4 * (size_t)s.U);
+    w.tables = off;
+    off = align256(off + 4 * (size_t)s.U * s.L * s.NB);
+    w.scores = off;
+    off = align256(off + 4 * (size_t)s.U * s.Ncap);
+    w.topk = off;
+    off = align256(off + 4 * topk_scratch_words(s));
+    w.part_o = off;
+    off = align256(off + 4 * (size_t)s.U * s.G * s.nsplit * s.d);
+    w.part_ml = off;
+    off = align256(off + 8 * (size_t)s.U * s.G * s.nsplit);
+    w.total = off;
+    return w;
+}
+
+}  // namespace socket_attn
+
+using namespace socket_attn;
+
+extern "C" {
+
+int socket_version(void) { return 100; }
+
+int socket_set_step_events(void* const* events, int n)
+{
+    g_last_error.clear();
+    if (n < 0 || n > SOCKET_DECODE_KERNELS + 1) return fail(SOCKET_EINVAL, "n=%d outside [0, %d]", n, SOCKET_DECODE_KERNELS + 1);
+    if (n > 0 && !events) return fail(SOCKET_EINVAL, "null event array");
+    for (int i = 0; i < n; ++i)
+        if (!events[i]) return fail(SOCKET_EINVAL, "null event handle %d", i);
+    for (int i = 0; i < n; ++i) g_step_events[i] = static_cast<cudaEvent_t>(events[i]);
+    g_num_step_events = n;
+    return SOCKET_OK;
+}
+
+const char* socket_last_error(void) { return g_last_error.c_str(); }
+
+int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv, int64_t Ncap,
+                     int64_t n_begin, int64_t n_end, int64_t d, const uint16_t* W, int L, int P, uint8_t* ids,
+                     float* vnorm, void* stream)
+{
+    g_last_error.clear();
+    int st = check_common(B, Hkv, Ncap, d, L, P);
+    if (st != SOCKET_OK) return st;
+    if (!valid_dtype(kv_dtype)) return fail(SOCKET_EINVAL, "kv_dtype=%d unknown", kv_dtype);
+    if (n_begin < 0 || n_begin > n_end || n_end > Ncap)
+        return fail(SOCKET_EINVAL, "need 0 <= n_begin <= n_end <= Ncap (got %lld, %lld, %lld)", (long long)n_begin,
+                    (long long)n_end, (long long)Ncap);
+    if (!K || !V || !W || !ids || !vnorm) return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16))
+        return fail(SOCKET_EINVAL, "K, V, W, ids and vnorm must be 16-byte aligned");
+    if (n_begin == n_end) return SOCKET_OK;
+    return cuda_status(launch_hash_keys(K, V, kv_dtype, B, Hkv, Ncap, n_begin, n_end, W, L, P, ids, vnorm,
+                                        static_cast<cudaStream_t>(stream)),
+                       "hash kernel launch");
+}
+
+size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P,
+                                    int k)
+{
+    DecodeShape s;
+    const std::string saved = g_last_error;
+    // N = k is the smallest valid N; the layout does not depend on N.
+    if (fill_shape(s, B, Hq, Hkv, Ncap, k, d, L, P, k) != SOCKET_OK) {
+        g_last_error = saved;
+        return 0;
+    }
+    s.nsplit = (k + attention_chunk_rows(SOCKET_F32) - 1) / attention_chunk_rows(SOCKET_F32);
+    return decode_workspace_layout(s).total;
+}
+
+int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
+                  const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
+                  int64_t N, int64_t d, int L, int P, double tau, int k, void* workspace, size_t workspace_bytes,
+                  int32_t* idx_out, float* out, float* scores_out, void* stream)
+{
+    g_last_error.clear();
+    DecodeShape s;
+    int st = fill_shape(s, B, Hq, Hkv, Ncap, N, d, L, P, k);
+    if (st != SOCKET_OK) return st;
+    if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype))
+        return fail(SOCKET_EINVAL, "q_dtype=%d / kv_dtype=%d unknown", q_dtype, kv_dtype);
+    if (!(tau > 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and > 0", tau);
+    if (!q || !W || !ids || !vnorm || !K || !V || !idx_out || !out || !workspace)
+        return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(K, 16) ||
+        !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
+        return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
+    if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
+    // Splits follow the kv dtype's chunk; the advertised size covers the smallest chunk.
+    s.nsplit = (k + attention_chunk_rows(kv_dtype) - 1) / attention_chunk_rows(kv_dtype);
+    const size_t need = socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k);
+    if (workspace_bytes < need)
+        return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+
+    const DecodeWorkspace w = decode_workspace_layout(s);
+    char* base = static_cast<char*>(workspace);
+    uint32_t* err_word = reinterpret_cast<uint32_t*>(base + w.err);
+    uint32_t* counters = reinterpret_cast<uint32_t*>(base + w.counters);
+    float* tables = reinterpret_cast<float*>(base + w.tables);
+    float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
+    uint32_t* topk = reinterpret_cast<uint32_t*>(base + w.topk);
+    float* part_o = reinterpret_cast<float*>(base + w.part_o);
+    float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, cs), "soft-table kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, cs), "score kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_topk(scores, s, topk, idx_out, cs), "top-k kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,
+                                      out, cs),
+                     "attention kernel launch");
+    if (st != SOCKET_OK) return st;
+    return cuda_status(mark_step(4, cs), "step event record");
+}
+
+}  // extern "C"

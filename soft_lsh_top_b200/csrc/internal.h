@@ -1,0 +1,58 @@
+// Internal launchers and workspace layout of the SOCKET library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace socket_attn {
+
+// Sizes of one decode call, validated by the API layer.
+struct DecodeShape {
+    int64_t B, Hq, Hkv, Ncap, N, d;
+    int L, P, k;
+    int G;         // Hq / Hkv
+    int64_t U;     // B * Hkv
+    int NB;        // 2^P
+    int nsplit;    // attention splits per unit
+};
+
+// Workspace regions (byte offsets from the workspace base, 256-aligned).
+struct DecodeWorkspace {
+    size_t err;        // uint32 device error word (offset 0)
+    size_t counters;   // uint32 [U] merge counters
+    size_t tables;     // float [U][L][NB]
+    size_t scores;     // float [U][Ncap]
+    size_t topk;       // uint32 [U][topk_words] top-k scratch
+    size_t part_o;     // float [U][G][nsplit][d]
+    size_t part_ml;    // float2 [U][G][nsplit]
+    size_t total;
+};
+
+DecodeWorkspace decode_workspace_layout(const DecodeShape& s);
+
+// Rows of the key/value gather handled by one attention CTA.
+int attention_chunk_rows(int kv_dtype);
+
+// --- kernels (each returns cudaGetLastError() after its launch) -------------
+cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv,
+                             int64_t Ncap, int64_t n_begin, int64_t n_end, const uint16_t* W,
+                             int L, int P, uint8_t* ids, float* vnorm, cudaStream_t stream);
+
+cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
+                               double tau, float* tables, uint32_t* err_word, uint32_t* counters,
+                               cudaStream_t stream);
+
+cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm,
+                         const DecodeShape& s, float* scores, cudaStream_t stream);
+
+cudaError_t launch_topk(const float* scores, const DecodeShape& s, uint32_t* scratch,
+                        int32_t* idx_out, cudaStream_t stream);
+
+cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
+                             const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
+                             uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream);
+
+size_t topk_scratch_words(const DecodeShape& s);
+
+}  // namespace socket_attn

@@ -1,0 +1,143 @@
+"""The C ABI library loads, exports what include/*.h declares, and rejects bad
+arguments on the host before any launch (CPU only: no call here reaches a
+kernel launch)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from soft_lsh_top_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, EINVAL, EUNSUP, ECUDA, EWS = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = _build.build()
+    import soft_lsh_top_b200 as s
+    return s.load_library(path)
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(socket_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ("socket_hash_keys", "socket_decode", "socket_decode_workspace_size", "socket_last_error"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(_build.LIB)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_version(lib):
+    assert lib.socket_version() == 100
+
+
+# Fake, aligned, never-dereferenced device addresses: every call below fails
+# validation before it could touch them.
+P16 = 0x10000
+
+
+def decode(lib, **kw):
+    a = dict(q=P16, q_dtype=1, W=P16, ids=P16, vnorm=P16, K=P16, V=P16, kv_dtype=1, B=1, Hq=4, Hkv=1, Ncap=64,
+             N=64, d=128, L=4, P=8, tau=0.5, k=8, ws=P16, ws_bytes=1 << 30, idx=P16, out=P16, scores=None,
+             stream=None)
+    a.update(kw)
+    return lib.socket_decode(a["q"], a["q_dtype"], a["W"], a["ids"], a["vnorm"], a["K"], a["V"], a["kv_dtype"],
+                             a["B"], a["Hq"], a["Hkv"], a["Ncap"], a["N"], a["d"], a["L"], a["P"], a["tau"],
+                             a["k"], a["ws"], a["ws_bytes"], a["idx"], a["out"], a["scores"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=64), EUNSUP),
+    (dict(P=9), EUNSUP),
+    (dict(P=0), EUNSUP),
+    (dict(L=0), EUNSUP),
+    (dict(L=129), EUNSUP),
+    (dict(Hq=5, Hkv=2), EINVAL),
+    (dict(Hq=34, Hkv=2), EUNSUP),
+    (dict(k=0), EINVAL),
+    (dict(k=65), EINVAL),
+    (dict(N=80), EINVAL),
+    (dict(Ncap=70, N=64), EINVAL),
+    (dict(tau=0.0), EINVAL),
+    (dict(tau=-1.0), EINVAL),
+    (dict(tau=float("nan")), EINVAL),
+    (dict(tau=float("inf")), EINVAL),
+    (dict(q_dtype=7), EINVAL),
+    (dict(K=P16 + 8), EINVAL),
+    (dict(ids=P16 + 4), EINVAL),
+    (dict(out=P16 + 4), EINVAL),
+    (dict(scores=P16 + 4), EINVAL),
+    (dict(idx=P16 + 2), EINVAL),
+    (dict(K=None), EINVAL),
+    (dict(ws=P16 + 16), EWS),
+    (dict(ws_bytes=16), EWS),
+])
+def test_decode_rejects(lib, kw, status):
+    assert decode(lib, **kw) == status
+    assert lib.socket_last_error().decode() != ""
+
+
+def hash_call(lib, **kw):
+    a = dict(K=P16, V=P16, kv_dtype=1, B=2, Hkv=2, Ncap=64, n_begin=0, n_end=64, d=128, W=P16, L=4, P=8,
+             ids=P16, vnorm=P16, stream=None)
+    a.update(kw)
+    return lib.socket_hash_keys(a["K"], a["V"], a["kv_dtype"], a["B"], a["Hkv"], a["Ncap"], a["n_begin"],
+                                a["n_end"], a["d"], a["W"], a["L"], a["P"], a["ids"], a["vnorm"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d=96), EUNSUP),
+    (dict(P=9), EUNSUP),
+    (dict(n_begin=10, n_end=5), EINVAL),
+    (dict(n_end=65), EINVAL),
+    (dict(n_begin=-1), EINVAL),
+    (dict(Ncap=60, n_end=60), EINVAL),
+    (dict(kv_dtype=3), EINVAL),
+    (dict(vnorm=P16 + 4), EINVAL),
+    (dict(W=None), EINVAL),
+    (dict(B=0), EINVAL),
+])
+def test_hash_rejects(lib, kw, status):
+    assert hash_call(lib, **kw) == status
+
+
+def test_empty_hash_range_is_a_no_op(lib):
+    assert hash_call(lib, n_begin=16, n_end=16) == OK
+
+
+def test_workspace_size(lib):
+    f = lib.socket_decode_workspace_size
+    small = f(1, 4, 1, 64, 128, 4, 8, 8)
+    big = f(8, 32, 8, 131072, 128, 32, 8, 2048)
+    assert 0 < small < big
+    # scores (4 B per key) and the soft tables dominate; partials grow with k.
+    assert big >= 64 * 131072 * 4 + 64 * 32 * 256 * 4
+    assert f(8, 32, 8, 131072, 128, 32, 8, 4096) > big
+    assert f(1, 4, 1, 64, 64, 4, 8, 8) == 0          # d != 128
+    assert f(1, 4, 1, 64, 128, 4, 8, 100) == 0       # k > Ncap
+    assert f(1, 3, 2, 64, 128, 4, 8, 8) == 0         # Hq % Hkv != 0
+
+
+def test_python_binding_checks_shapes_before_the_library():
+    import torch
+    import soft_lsh_top_b200 as s
+    with pytest.raises((ValueError, TypeError)):
+        s.socket_hash_keys(torch.zeros(1, 1, 16, 128), torch.zeros(1, 1, 16, 128),
+                           torch.zeros(4, 8, 128, dtype=torch.bfloat16),
+                           torch.zeros(1, 1, 4, 16, dtype=torch.uint8), torch.zeros(1, 1, 16))

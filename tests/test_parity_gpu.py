@@ -1,0 +1,181 @@
+"""CUDA path vs oracle, element by element, through the C ABI (needs a GPU).
+
+Small and ragged cases are compared on every unit and key; the full-size
+workloads (batch-8 128K, one million tokens, batch-32 16K with appends) are
+compared on sampled units, in the same launch configuration the benchmark
+times.  Matching rules are in parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from parity import (check_decode, check_hash, gpu_decode, gpu_hash, oracle_hash_units, substitute_units)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+SMALL = {
+    "tiny_f32_4k": wl.TINY,
+    "llama_32k": wl.LLAMA_32K,
+    "ragged_multitile": wl.LLAMA_32K.scaled(name="ragged", B=2, Hq=8, Hkv=2, N=70001, L=12, k=700, tau=0.4,
+                                            seed=7001),
+    "odd_group3_p5": wl.Workload(name="odd", B=2, Hq=6, Hkv=2, N=3001, L=7, P=5, tau=0.7, k=77, seed=7002),
+    "f32_group2_p6": wl.Workload(name="f32g2", B=1, Hq=4, Hkv=2, N=2500, L=9, P=6, tau=0.25, k=100, dtype="f32",
+                                 seed=7003),
+}
+
+
+@pytest.fixture(scope="module", params=sorted(SMALL))
+def small(request):
+    w = SMALL[request.param]
+    inp = wl.make_inputs(w, DEV)
+    units = list(range(w.U))
+    orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units)
+    return w, inp, units, orc_ids, orc_vn, margin
+
+
+def test_hash_matches_oracle(small):
+    w, inp, units, orc_ids, orc_vn, margin = small
+    ids, vnorm = gpu_hash(inp, w)
+    torch.cuda.synchronize()
+    g_ids = ids.reshape(w.U, w.L, w.ncap).cpu().numpy()
+    g_vn = vnorm.reshape(w.U, w.ncap).cpu().numpy()
+    check_hash(g_ids, g_vn, orc_ids, orc_vn, margin, 0, w.N)
+
+
+def _decode_on_oracle_index(small, **kw):
+    w, inp, units, orc_ids, orc_vn, _ = small
+    orc_vn32 = orc_vn.astype(np.float32)
+    ids = torch.from_numpy(orc_ids).reshape(inp["K"].shape[0], w.Hkv, w.L, w.ncap).to(DEV)
+    vn = torch.from_numpy(orc_vn32).reshape(inp["K"].shape[0], w.Hkv, w.ncap).to(DEV)
+    idx, out, sc = gpu_decode(inp, w, ids, vn, **kw)
+    return check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, **kw)
+
+
+def test_decode_matches_oracle(small):
+    _decode_on_oracle_index(small)
+
+
+@pytest.mark.parametrize("variant", ["k1", "k_eq_n", "tau_0.01", "tau_5", "n_not_ncap"])
+def test_decode_edge_cases(small, variant):
+    w = small[0]
+    if variant == "k1":
+        _decode_on_oracle_index(small, k=1)
+    elif variant == "k_eq_n":
+        _decode_on_oracle_index(small, k=w.N)
+    elif variant == "tau_0.01":
+        _decode_on_oracle_index(small, tau=0.01)
+    elif variant == "tau_5":
+        _decode_on_oracle_index(small, tau=5.0)
+    else:
+        n = w.N - 13
+        _decode_on_oracle_index(small, N=n, k=min(w.k, n))
+
+
+def test_all_ties_select_lowest_indices():
+    """Zero queries give every bucket 2^-P and equal value norms give every key
+    the same score: the selection must be keys 0..k-1."""
+    w = wl.Workload(name="ties", B=1, Hq=4, Hkv=2, N=9000, L=5, P=8, tau=0.3, k=333, seed=7004)
+    inp = wl.make_inputs(w, DEV)
+    inp["q"].zero_()
+    inp["V"].fill_(1.0)
+    ids, vnorm = gpu_hash(inp, w)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    want = torch.arange(w.k, dtype=torch.int32, device=DEV)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            assert torch.equal(idx[b, h], want)
+    assert torch.all(sc[..., : w.N] == sc[0, 0, 0])
+    torch.testing.assert_close(out, torch.ones_like(out), atol=1e-6, rtol=0)
+
+
+def test_decode_is_deterministic():
+    w = SMALL["ragged_multitile"]
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)
+    a = gpu_decode(inp, w, ids, vnorm)
+    b = gpu_decode(inp, w, ids, vnorm)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int32) if x.dtype == torch.float32 else x,
+                           y.view(torch.int32) if y.dtype == torch.float32 else y)
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads, sampled units
+# ----------------------------------------------------------------------------
+
+def _full_size(w, sample_units):
+    torch.cuda.empty_cache()
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)
+    torch.cuda.synchronize()
+    orc_ids, orc_vn, margin = oracle_hash_units(inp, w, sample_units)
+    g_ids = torch.stack([ids[u // w.Hkv, u % w.Hkv] for u in sample_units]).cpu().numpy()
+    g_vn = torch.stack([vnorm[u // w.Hkv, u % w.Hkv] for u in sample_units]).cpu().numpy()
+    check_hash(g_ids, g_vn, orc_ids, orc_vn, margin, 0, w.N)
+    return inp, ids, vnorm, orc_ids, orc_vn.astype(np.float32)
+
+
+def test_batch8_128k_sampled_units_and_needles():
+    w = wl.BATCH8_128K
+    units = [0, 27, 63]
+    inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
+    # Needle recall on every unit with the kernels' own index.
+    idx, _, _ = gpu_decode(inp, w, ids, vnorm)
+    needles = inp["needles"]
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            got = torch.isin(needles[b, h].to(torch.int32), idx[b, h])
+            assert bool(got.all()), f"unit ({b},{h}) missed {int((~got).sum())} needles"
+    substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc)
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_million_token_sampled_units():
+    w = wl.MILLION
+    units = [2, 7]
+    inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
+    substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc)
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_append_mix_sampled_units():
+    """Prefill hash of 16384 keys, then 64 steps that each hash one appended
+    key at offset N+t and decode over N+t+1 keys; then the temperature sweep."""
+    w = wl.APPEND_MIX
+    units = [0, 131, 255]
+    torch.cuda.empty_cache()
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)                      # keys [0, N)
+    checked = {}
+    for t in range(w.appends):
+        import soft_lsh_top_b200 as sk
+        sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, w.N + t, w.N + t + 1)
+        if t in (0, 31, 63):
+            idx, out, sc = gpu_decode(inp, w, ids, vnorm, N=w.N + t + 1, q=inp["q_steps"][t])
+            checked[t] = (idx.cpu(), out.cpu(), sc.cpu())
+    torch.cuda.synchronize()
+    n_all = w.N + w.appends
+    orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units, 0, n_all)
+    g_ids = torch.stack([ids[u // w.Hkv, u % w.Hkv] for u in units]).cpu().numpy()
+    g_vn = torch.stack([vnorm[u // w.Hkv, u % w.Hkv] for u in units]).cpu().numpy()
+    check_hash(g_ids, g_vn, orc_ids, orc_vn, margin, 0, n_all)
+    orc_vn32 = orc_vn.astype(np.float32)
+    substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
+    for t in (0, 31, 63):
+        idx, out, sc = gpu_decode(inp, w, ids, vnorm, N=w.N + t + 1, q=inp["q_steps"][t])
+        check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, N=w.N + t + 1, q=inp["q_steps"][t])
+    for tau in w.tau_sweep:
+        idx, out, sc = gpu_decode(inp, w, ids, vnorm, N=n_all, tau=tau, q=inp["q_steps"][-1])
+        check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, N=n_all, tau=tau, q=inp["q_steps"][-1])
+    del inp
+    torch.cuda.empty_cache()

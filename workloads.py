@@ -140,7 +140,10 @@ def make_inputs(w: Workload, device="cpu", batches=None):
     V = torch.empty_like(K)
     needles = torch.empty(len(keep), w.Hkv, w.G * w.needles_per_head, dtype=torch.int64, device=device)
     pos = torch.arange(ncap, device=device, dtype=torch.float32)
+    last = max(keep)
     for b in range(w.B):
+        if b > last and not w.appends:
+            break  # later rows only consume the stream; nothing drawn after them is needed
         Kb = torch.randn(w.Hkv, ncap, d, generator=g, device=device)
         Vb = torch.randn(w.Hkv, ncap, d, generator=g, device=device)
         if w.outlier_channels:
