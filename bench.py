@@ -289,6 +289,9 @@ def run_socket(args, world: int, rank: int, local_rank: int):
     K = args.steps
     nk = 4
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for e in row:
+            e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()

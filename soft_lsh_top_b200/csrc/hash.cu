@@ -9,9 +9,9 @@
 // table, and the value-vector norms are cached.
 //
 // id_l(k) = sum_p [<W_{l,p}, k> > 0] 2^p, accumulated in float32 with one
-// fused multiply-add per element in channel order (bfloat16 x bfloat16 and
-// bfloat16 x float32 products are exact in float32, so the only error is the
-// float32 accumulation).  vnorm = sqrt(sum v^2), float32.
+// fused multiply-add per element in channel order (bfloat16 x bfloat16
+// products are exact in float32, so the only error is the float32
+// accumulation).  vnorm = sqrt(sum v^2) summed in float64, rounded to float32.
 #include "common.cuh"
 #include "internal.h"
 
@@ -57,12 +57,15 @@ __global__ __launch_bounds__(kThreads) void hash_kernel(const KT* __restrict__ K
     const int64_t n = n0 + key;
 
     if (tg == 0 && key < nk) {
-        float s = 0.0f;
+        // Squares of float32 / bfloat16 values are exact in float64 and the
+        // 128-term sum loses at most ~1e-14 relative, so the float32 norm is
+        // the correctly rounded norm except in rare rounding ties.
+        double s = 0.0;
         for (int j = 0; j < kHeadDim; ++j) {
-            const float v = elem(Vu, n * kHeadDim + j);
-            s = fmaf(v, v, s);
+            const double v = (double)elem(Vu, n * kHeadDim + j);
+            s = fma(v, v, s);
         }
-        vnorm[u * Ncap + n] = sqrtf(s);
+        vnorm[u * Ncap + n] = (float)sqrt(s);
     }
 
     const int wpr = P * kHeadDim / 2;  // 32-bit words of W per table

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import oracle
+import soft_lsh_top_b200 as sk
 import workloads as wl
 from parity import (check_decode, check_hash, gpu_decode, gpu_hash, oracle_hash_units, substitute_units)
 
@@ -120,19 +121,29 @@ def _full_size(w, sample_units):
 
 
 def test_batch8_128k_sampled_units_and_needles():
+    """Planted needles: on sampled units the kernels select exactly the needles
+    the oracle selects (some needles genuinely rank below k in fp64: a needle
+    planted for one query head competes with keys the group's other heads
+    favour); over all 64 units, recall stays at or above 99 %."""
     w = wl.BATCH8_128K
-    units = [0, 27, 63]
+    units = [0, 11, 27, 63]
     inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
-    # Needle recall on every unit with the kernels' own index.
     idx, _, _ = gpu_decode(inp, w, ids, vnorm)
     needles = inp["needles"]
-    for b in range(w.B):
-        for h in range(w.Hkv):
-            got = torch.isin(needles[b, h].to(torch.int32), idx[b, h])
-            assert bool(got.all()), f"unit ({b},{h}) missed {int((~got).sum())} needles"
+    found = sum(int(torch.isin(needles[b, h].to(torch.int32), idx[b, h]).sum())
+                for b in range(w.B) for h in range(w.Hkv))
+    recall = found / needles.numel()
+    assert recall >= 0.99, recall
     substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
     idx, out, sc = gpu_decode(inp, w, ids, vnorm)
     check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc)
+    for i, u in enumerate(units):
+        b, h = divmod(u, w.Hkv)
+        q_u = inp["q"][b, h * w.G:(h + 1) * w.G].cpu()
+        o_idx = oracle.decode_unit(q_u, inp["W"].cpu(), w.L, w.P, w.tau, orc_ids[i], orc_vn32[i],
+                                   inp["K"][b, h].cpu(), inp["V"][b, h].cpu(), w.N, w.k)[0]
+        nd = needles[b, h].cpu().numpy()
+        assert np.array_equal(np.isin(nd, idx[b, h].cpu().numpy()), np.isin(nd, o_idx)), u
     del inp
     torch.cuda.empty_cache()
 
@@ -156,13 +167,9 @@ def test_append_mix_sampled_units():
     torch.cuda.empty_cache()
     inp = wl.make_inputs(w, DEV)
     ids, vnorm = gpu_hash(inp, w)                      # keys [0, N)
-    checked = {}
     for t in range(w.appends):
-        import soft_lsh_top_b200 as sk
         sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, w.N + t, w.N + t + 1)
-        if t in (0, 31, 63):
-            idx, out, sc = gpu_decode(inp, w, ids, vnorm, N=w.N + t + 1, q=inp["q_steps"][t])
-            checked[t] = (idx.cpu(), out.cpu(), sc.cpu())
+        gpu_decode(inp, w, ids, vnorm, N=w.N + t + 1, q=inp["q_steps"][t])
     torch.cuda.synchronize()
     n_all = w.N + w.appends
     orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units, 0, n_all)
