@@ -143,6 +143,38 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W,
                   int32_t* idx_out, float* out, float* scores_out, void* stream);
 
 /*
+ * socket_decode_static -- socket_decode for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a packaging variant
+ * of socket_decode, same arguments minus the workspace, same results.
+ *
+ * Who needs it: code that runs where cudaMalloc is off limits and no one
+ * hands it scratch memory -- e.g. a kernel library embedded in a serving
+ * runtime that has already reserved (nearly) all device memory for its own
+ * pool and exposes no scratch allocator, or a caller that must not risk the
+ * device-wide synchronisation an allocation can cause in a latency-critical
+ * path.  Such callers still pass their inputs and outputs.
+ *
+ * Scratch: a file-scope device array of SOCKET_STATIC_WORKSPACE_BYTES (64 MiB)
+ * inside this library; every GPU that loads the library holds it until the
+ * process exits.  Calls whose socket_decode_workspace_size() exceeds it are
+ * rejected with SOCKET_EWORKSPACE before anything is launched.  The first
+ * call on a device looks up the array's device address (once per device,
+ * with that device current), so make that first call before any stream
+ * capture.  Nothing here calls cudaMalloc, cudaFree or an allocating library
+ * routine.  Every call on a device shares the same array, which keeps the
+ * previous call's contents; the decode clears what must start at zero (its
+ * counters and error word) itself.  Calls that overlap on the GPU (other
+ * streams, other host threads) race on the array: serialise them.
+ */
+#define SOCKET_STATIC_WORKSPACE_BYTES (64u << 20)
+int socket_decode_static(const void* q, int q_dtype, const uint16_t* W,
+                         const uint8_t* ids, const float* vnorm,
+                         const void* K, const void* V, int kv_dtype,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d,
+                         int L, int P, double tau, int k,
+                         int32_t* idx_out, float* out, float* scores_out, void* stream);
+
+/*
  * socket_last_error -- message for the last non-OK status returned on the
  * calling host thread ("" if none).  The pointer stays valid until the next
  * call on that thread.

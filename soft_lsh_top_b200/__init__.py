@@ -19,7 +19,7 @@ import os
 import torch
 
 __all__ = [
-    "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_workspace_size",
+    "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
     "socket_last_error", "socket_version", "socket_set_step_events", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -65,6 +65,9 @@ def load_library(path: str | None = None):
     lib.socket_decode.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64,
                                   _int, _int, _dbl, _int, _vp, _sz, _vp, _vp, _vp, _vp]
     lib.socket_decode.restype = _int
+    lib.socket_decode_static.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
+                                         _i64, _int, _int, _dbl, _int, _vp, _vp, _vp, _vp]
+    lib.socket_decode_static.restype = _int
     lib.socket_last_error.argtypes = []
     lib.socket_last_error.restype = ctypes.c_char_p
     lib.socket_set_step_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _int]
@@ -190,6 +193,37 @@ def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: to
                                  idx_out.data_ptr(), out.data_ptr(),
                                  scores_out.data_ptr() if scores_out is not None else None,
                                  _stream_handle(stream)))
+
+
+def socket_decode_static(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
+                         K: torch.Tensor, V: torch.Tensor, N: int, tau: float, k: int,
+                         idx_out: torch.Tensor, out: torch.Tensor, scores_out: torch.Tensor | None = None,
+                         stream=None) -> None:
+    """socket_decode without a caller workspace, for callers that cannot
+    allocate device memory: the library's own fixed 64 MiB device scratch is
+    used instead (see include/socket_attn.h).  Calls that overlap on the GPU
+    share that scratch and must be serialised by the caller."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    _, Hkv, Ncap, _ = K.shape
+    L, P, _ = W.shape
+    dev = q.device
+    _check(q, "q", (B, Hq, d), device=dev)
+    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
+    _check(ids, "ids", (B, Hkv, L, Ncap), dtype=torch.uint8, device=dev)
+    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
+    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
+    _check(idx_out, "idx_out", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
+    if scores_out is not None:
+        _check(scores_out, "scores_out", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_decode_static(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(),
+                                        K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P,
+                                        float(tau), int(k), idx_out.data_ptr(), out.data_ptr(),
+                                        scores_out.data_ptr() if scores_out is not None else None,
+                                        _stream_handle(stream)))
 
 
 def socket_set_step_events(events) -> None:

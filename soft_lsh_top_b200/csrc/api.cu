@@ -89,6 +89,12 @@ int fill_shape(DecodeShape& s, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
 
 }  // namespace
 
+int record_error(int status, const char* message)
+{
+    g_last_error = message;
+    return status;
+}
+
 DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
 {
     DecodeWorkspace w;

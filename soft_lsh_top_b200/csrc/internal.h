@@ -55,4 +55,7 @@ cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const vo
 
 size_t topk_scratch_words(const DecodeShape& s);
 
+// Sets the calling thread's socket_last_error() message; returns `status`.
+int record_error(int status, const char* message);
+
 }  // namespace socket_attn
