@@ -2,6 +2,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 
 #include <string>
 
@@ -89,6 +90,12 @@ int fill_shape(DecodeShape& s, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
 
 }  // namespace
 
+bool pdl_enabled()
+{
+    static const bool on = getenv("SOCKET_NO_PDL") == nullptr;
+    return on;
+}
+
 int record_error(int status, const char* message)
 {
     g_last_error = message;
@@ -103,12 +110,12 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 4);
     w.counters = off;
     off = align256(off + 4 * (size_t)s.U);
+    w.unit_max = off;
+    off = align256(off + 4 * (size_t)s.U);
     w.tables = off;
     off = align256(off + 4 * (size_t)s.U * s.L * s.NB);
     w.scores = off;
     off = align256(off + 4 * (size_t)s.U * s.Ncap);
-    w.topk = off;
-    off = align256(off + 4 * topk_scratch_words(s));
     w.part_o = off;
     off = align256(off + 4 * (size_t)s.U * s.G * s.nsplit * s.d);
     w.part_ml = off;
@@ -203,19 +210,19 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
     uint32_t* counters = reinterpret_cast<uint32_t*>(base + w.counters);
     float* tables = reinterpret_cast<float*>(base + w.tables);
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
-    uint32_t* topk = reinterpret_cast<uint32_t*>(base + w.topk);
+    uint32_t* unit_max = reinterpret_cast<uint32_t*>(base + w.unit_max);
     float* part_o = reinterpret_cast<float*>(base + w.part_o);
     float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
     if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, cs), "soft-table kernel launch");
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, cs), "soft-table kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, cs), "score kernel launch");
+    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, cs), "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_topk(scores, s, topk, idx_out, cs), "top-k kernel launch");
+    st = cuda_status(launch_topk(scores, unit_max, s, idx_out, cs), "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
     st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,

@@ -7,9 +7,9 @@
 // pages run this step with a "Flash Decode" backend ("Contribuciones Clave"
 // 2 / "Hauptbeiträge"); here it is a hand-written split-K kernel.
 //
-// Each CTA takes one chunk of a unit's selected rows: it gathers the chunk's
-// key and value rows into shared memory with bulk asynchronous copies (one
-// 256-byte row per copy, completion counted on an mbarrier), computes the
+// Each CTA takes one chunk (64 rows) of a unit's selected rows: it gathers the
+// chunk's key and value rows into shared memory with bulk asynchronous copies
+// (one 256-byte row per copy, completion counted on an mbarrier), computes the
 // logits of all query heads of the unit (scale 1/sqrt(d)), the chunk's
 // running max and exp-sum, and the unnormalised weighted value sum.  The
 // last CTA of a unit to finish (an atomic ticket, no waiting) merges the
@@ -30,12 +30,12 @@ template <typename KT>
 struct Rows;
 template <>
 struct Rows<uint16_t> {  // bfloat16
-    static constexpr int kChunk = 128;
+    static constexpr int kChunk = 64;
     static constexpr int kRowBytes = kHeadDim * 2;
 };
 template <>
 struct Rows<float> {
-    static constexpr int kChunk = 64;
+    static constexpr int kChunk = 32;
     static constexpr int kRowBytes = kHeadDim * 4;
 };
 
@@ -73,6 +73,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     __shared__ int32_t rows[kChunk];
     __shared__ __align__(8) uint64_t bar;
     __shared__ uint32_t s_last;
+    __shared__ float wsm[kThreads];  // merge weights
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t u = blockIdx.x / nsplit;
@@ -81,12 +82,6 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     const int r0 = split * kChunk;
     const int nrows = min(kChunk, k - r0);
 
-    if (tid < nrows) {
-        // Indices come from the top-k kernel and are < N; clamp anyway so a
-        // gather can never leave the unit's cache rows.
-        const int32_t r = idx[u * k + r0 + tid];
-        rows[tid] = (r >= 0 && r < Ncap) ? r : 0;
-    }
     const int64_t qrow0 = b * Hq + kvh * G;
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
         const int64_t off = qrow0 * kHeadDim + e;
@@ -96,6 +91,13 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     if (tid == 0) {
         mbar_init(&bar, 1);
         fence_mbarrier_init();
+    }
+    pdl_wait();  // the selected indices come from the previous kernel on the stream
+    if (tid < nrows) {
+        // Indices come from the top-k kernel and are < N; clamp anyway so a
+        // gather can never leave the unit's cache rows.
+        const int32_t r = __ldcg(idx + u * k + r0 + tid);
+        rows[tid] = (r >= 0 && r < Ncap) ? r : 0;
     }
     __syncthreads();
     if (tid == 0) mbar_arrive_expect_tx(&bar, (uint32_t)nrows * 2u * kRowBytes);
@@ -211,19 +213,52 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-#pragma unroll
+    // Per head: M = max_s m_s; w_s = exp(m_s - M); out = sum_s w_s o_s / sum_s w_s l_s,
+    // accumulated in split order.  Weights are staged in shared memory, kThreads
+    // splits at a time, and the partial rows are read with many loads in flight.
     for (int h = 0; h < G; ++h) {
         const int64_t base = pbase + h * nsplit;
-        float M = -INFINITY;
-        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(&part_ml[base + sp]).x);
-        float Lsum = 0.0f, acc = 0.0f;
-        for (int sp = 0; sp < nsplit; ++sp) {
-            const float2 t = __ldcg(&part_ml[base + sp]);
-            const float w = expf(t.x - M);
-            Lsum += t.y * w;
-            acc += __ldcg(&part_o[(base + sp) * kHeadDim + tid]) * w;
+        float m = -INFINITY;
+        for (int sp = tid; sp < nsplit; sp += kThreads) m = fmaxf(m, __ldcg(&part_ml[base + sp]).x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
+        __syncthreads();
+        if (lane == 0) red[warp][0] = m;
+        __syncthreads();
+        float M = red[0][0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) M = fmaxf(M, red[w][0]);
+        float lsum = 0.0f, acc = 0.0f;
+        for (int s0 = 0; s0 < nsplit; s0 += kThreads) {
+            const int cnt = min(kThreads, nsplit - s0);
+            __syncthreads();
+            if (tid < cnt) {
+                const float2 t = __ldcg(&part_ml[base + s0 + tid]);
+                const float w = expf(t.x - M);
+                wsm[tid] = w;
+                lsum += t.y * w;
+            }
+            __syncthreads();
+            const float* po = part_o + (base + s0) * kHeadDim + tid;
+            int i = 0;
+            for (; i + 16 <= cnt; i += 16) {
+                float v[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) v[r] = __ldcg(po + (int64_t)(i + r) * kHeadDim);
+#pragma unroll
+                for (int r = 0; r < 16; ++r) acc += v[r] * wsm[i + r];
+            }
+            for (; i < cnt; ++i) acc += __ldcg(po + (int64_t)i * kHeadDim) * wsm[i];
         }
-        out[(qrow0 + h) * kHeadDim + tid] = acc / Lsum;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, o);
+        __syncthreads();
+        if (lane == 0) red[warp][0] = lsum;
+        __syncthreads();
+        float L = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) L += red[w][0];
+        out[(qrow0 + h) * kHeadDim + tid] = acc / L;
     }
     if (tid == 0) counters[u] = 0u;
 }
@@ -237,9 +272,10 @@ cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, c
     auto kern = attention_kernel<KT, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(s.U * s.nsplit), kThreads, smem, stream>>>(
-        q, q_dtype, static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.Hq, s.Hkv, s.Ncap, s.k, s.nsplit,
-        part_o, part_ml, counters, err_word, out);
+    e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream, q, q_dtype,
+                   static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.Hq, s.Hkv, s.Ncap, s.k, s.nsplit,
+                   part_o, part_ml, counters, err_word, out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

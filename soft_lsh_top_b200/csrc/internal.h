@@ -21,9 +21,9 @@ struct DecodeShape {
 struct DecodeWorkspace {
     size_t err;        // uint32 device error word (offset 0)
     size_t counters;   // uint32 [U] merge counters
+    size_t unit_max;   // uint32 [U] bit pattern of each unit's largest score
     size_t tables;     // float [U][L][NB]
     size_t scores;     // float [U][Ncap]
-    size_t topk;       // uint32 [U][topk_words] top-k scratch
     size_t part_o;     // float [U][G][nsplit][d]
     size_t part_ml;    // float2 [U][G][nsplit]
     size_t total;
@@ -39,21 +39,20 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
                              int64_t Ncap, int64_t n_begin, int64_t n_end, const uint16_t* W,
                              int L, int P, uint8_t* ids, float* vnorm, cudaStream_t stream);
 
+// Also zeroes the error word, the merge counters and the per-unit max scores.
 cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
                                double tau, float* tables, uint32_t* err_word, uint32_t* counters,
-                               cudaStream_t stream);
+                               uint32_t* unit_max, cudaStream_t stream);
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm,
-                         const DecodeShape& s, float* scores, cudaStream_t stream);
+                         const DecodeShape& s, float* scores, uint32_t* unit_max, cudaStream_t stream);
 
-cudaError_t launch_topk(const float* scores, const DecodeShape& s, uint32_t* scratch,
+cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const DecodeShape& s,
                         int32_t* idx_out, cudaStream_t stream);
 
 cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
                              const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
                              uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream);
-
-size_t topk_scratch_words(const DecodeShape& s);
 
 // Sets the calling thread's socket_last_error() message; returns `status`.
 int record_error(int status, const char* message);
