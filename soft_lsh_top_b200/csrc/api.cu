@@ -112,6 +112,12 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 4 * (size_t)s.U);
     w.unit_max = off;
     off = align256(off + 4 * (size_t)s.U);
+    w.unit_hist = off;
+    off = align256(off + 4 * (size_t)s.U * kScoreHistBins);
+    w.cand_cnt = off;
+    off = align256(off + 4 * (size_t)s.U);
+    w.cand = off;
+    off = align256(off + 8 * (size_t)s.U * kTopkCandidates);
     w.tables = off;
     off = align256(off + 4 * (size_t)s.U * s.L * s.NB);
     w.scores = off;
@@ -211,18 +217,21 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
     float* tables = reinterpret_cast<float*>(base + w.tables);
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
     uint32_t* unit_max = reinterpret_cast<uint32_t*>(base + w.unit_max);
+    uint32_t* unit_hist = reinterpret_cast<uint32_t*>(base + w.unit_hist);
+    uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
+    uint2* cand = reinterpret_cast<uint2*>(base + w.cand);
     float* part_o = reinterpret_cast<float*>(base + w.part_o);
     float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
     if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, cs), "soft-table kernel launch");
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt, cs), "soft-table kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, cs), "score kernel launch");
+    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, cs), "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_topk(scores, unit_max, s, idx_out, cs), "top-k kernel launch");
+    st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
     st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,

@@ -17,11 +17,23 @@ struct DecodeShape {
     int nsplit;    // attention splits per unit
 };
 
+// Per-unit histogram of live scores, taken by the scoring kernel over the
+// score bit pattern >> kScoreHistShift (1/16 octave per bin; finite
+// non-negative scores land below bin 4081).
+constexpr int kScoreHistBins = 4096;
+constexpr int kScoreHistShift = 19;
+// Top-k candidate capacity per unit (keys in the threshold bin of the
+// histogram); above it the top-k kernel takes its multi-pass path.
+constexpr int kTopkCandidates = 4096;
+
 // Workspace regions (byte offsets from the workspace base, 256-aligned).
 struct DecodeWorkspace {
     size_t err;        // uint32 device error word (offset 0)
     size_t counters;   // uint32 [U] merge counters
     size_t unit_max;   // uint32 [U] bit pattern of each unit's largest score
+    size_t unit_hist;  // uint32 [U][kScoreHistBins] score histogram
+    size_t cand_cnt;   // uint32 [U] top-k candidate counters
+    size_t cand;       // uint2 [U][kTopkCandidates] top-k candidates (index, bit pattern)
     size_t tables;     // float [U][L][NB]
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
@@ -39,16 +51,18 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
                              int64_t Ncap, int64_t n_begin, int64_t n_end, const uint16_t* W,
                              int L, int P, uint8_t* ids, float* vnorm, cudaStream_t stream);
 
-// Also zeroes the error word, the merge counters and the per-unit max scores.
+// Also zeroes the error word, the merge counters, the per-unit max scores,
+// the score histograms and the candidate counters.
 cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
                                double tau, float* tables, uint32_t* err_word, uint32_t* counters,
-                               uint32_t* unit_max, cudaStream_t stream);
+                               uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream);
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm,
-                         const DecodeShape& s, float* scores, uint32_t* unit_max, cudaStream_t stream);
+                         const DecodeShape& s, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
+                         cudaStream_t stream);
 
-cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const DecodeShape& s,
-                        int32_t* idx_out, cudaStream_t stream);
+cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const uint32_t* unit_hist,
+                        uint32_t* cand_cnt, uint2* cand, const DecodeShape& s, int32_t* idx_out, cudaStream_t stream);
 
 cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
                              const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,

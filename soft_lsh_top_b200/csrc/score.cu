@@ -13,8 +13,10 @@
 // B200 design.  The step streams L + 4 bytes per key from HBM (one uint8 id
 // per table, table-major, plus the fp32 norm) and performs L random lookups
 // into 2^P-entry tables.  Lookups go to shared memory in a lane-private
-// layout: a buffer holds two tables as float[256 buckets][2 tables][32 lanes],
-// so lane j only ever touches bank j and a warp's 32 lookups are one
+// layout: a 64 KB buffer holds four tables as float[256 buckets][4 tables]
+// [16 replicas]; lane j uses replica j % 16, and the two half-warps look up
+// different tables of the buffer in the same instruction (round t: slot
+// t ^ half), so a warp's 32 random lookups land in 32 distinct banks -- one
 // conflict-free wavefront whatever the ids are.  The buffers sit at 64 KB-
 // aligned shared addresses, so one byte-permute of the packed id word yields
 // the full shared address of a lookup.  Each
@@ -33,24 +35,18 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kGroupsPerThread = 4;                      // 16-key groups per thread per pass
 constexpr int kPassGroups = kThreads * kGroupsPerThread;  // 2048 groups = 32768 keys
-constexpr uint32_t kBufBytes = 1u << 16;                 // [bucket 256][table pair 2][lane 32] floats
+constexpr uint32_t kBufBytes = 1u << 16;                 // [bucket 256][table 4][replica 16] floats
+constexpr int kTablesPerBuf = 4;
 constexpr int kStageSlots = kBufBytes / 16 / kThreads;   // float4 stores per thread per buffer (8)
-constexpr int kPrefetchAhead = 4;                        // tables prefetched into L2 ahead
+constexpr int kPrefetchAhead = 8;                        // tables prefetched into L2 ahead
+constexpr int kHistBins = kScoreHistBins;                // unit histogram of score bit patterns >> kHistShift
+constexpr int kHistShift = kScoreHistShift;
 // The two staging buffers sit at 64 KB-aligned shared addresses A and
-// A + 64 KB.  A lookup address is then A_buf | (id << 8) | (tt << 7) | (lane << 2):
-// one byte-permute of the packed id word with a per-thread base that already
-// holds A_buf, the table-in-pair and the lane.  The dynamic allocation spans
+// A + 64 KB.  A lookup address is then A_buf | (id << 8) | (slot << 6) | (replica << 2):
+// one byte-permute of the packed id word with a per-lane base that already
+// holds A_buf, the table slot and the replica.  The dynamic allocation spans
 // three 64 KB windows so an aligned pair fits wherever the window starts.
 constexpr int kSmemBytes = 3 * (int)kBufBytes;
-
-__device__ __forceinline__ void load_ids(uint4 (&v)[kGroupsPerThread], const uint8_t* row, int npg, int tid)
-{
-#pragma unroll
-    for (int j = 0; j < kGroupsPerThread; ++j) {
-        const int g = j * kThreads + tid;
-        v[j] = g < npg ? ldg_stream_u4(row + (int64_t)g * 16) : make_uint4(0, 0, 0, 0);
-    }
-}
 
 __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
@@ -59,39 +55,34 @@ __device__ __forceinline__ float lds_f32(uint32_t addr)
     return v;
 }
 
-// Accumulate one table's contribution for this thread's live groups.
-// `base` = shared address of the buffer | (table-in-pair << 7) | (lane << 2),
-// whose byte 1 is zero.
-__device__ __forceinline__ void lookup(float (&acc)[kGroupsPerThread][16], const uint4 (&v)[kGroupsPerThread],
-                                       uint32_t base, int npg, int tid)
+// Ids of round rr for this lane's 4 groups: table (rr & ~3) + ((rr & 3) ^ half).
+// Groups past the pass read the pass's last group instead (their sums are
+// never stored), so the lookup loop needs no per-group condition.
+__device__ __forceinline__ void load_round(uint4 (&v)[kGroupsPerThread], const uint8_t* idu, int64_t Ncap, int L,
+                                           int npg, int tid, int half, int rr)
 {
+    const int tab = (rr & ~(kTablesPerBuf - 1)) + ((rr & (kTablesPerBuf - 1)) ^ half);
+    const uint8_t* row = idu + (int64_t)min(tab, L - 1) * Ncap;
 #pragma unroll
     for (int j = 0; j < kGroupsPerThread; ++j) {
-        if (j * kThreads + tid < npg) {
-            const uint32_t words[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-#pragma unroll
-                for (int byte = 0; byte < 4; ++byte) {
-                    // bytes 0, 2, 3 from base; byte 1 = the id
-                    const uint32_t addr = __byte_perm(base, words[w], 0x3240u + (byte << 4));
-                    acc[j][w * 4 + byte] += lds_f32(addr);
-                }
-            }
-        }
+        const int g = min(j * kThreads + tid, npg - 1);
+        v[j] = ldg_stream_u4(row + (int64_t)g * 16);
     }
 }
 
 // One pass: groups [first_group, first_group + npg) of one unit, npg <= kPassGroups.
 __device__ __forceinline__ void score_pass(const float* __restrict__ tables, const uint8_t* __restrict__ ids,
                                            const float* __restrict__ vnorm, float* __restrict__ scores,
-                                           uint32_t* __restrict__ unit_max, char* smem, uint32_t buf0, int L,
+                                           uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
+                                           uint32_t* shist, char* smem, uint32_t buf0, int L,
                                            int NB, int64_t Ncap, int64_t N, int64_t unit, int64_t first_group,
                                            int npg, bool first_pass, uint32_t* red)
 {
-    const int tid = threadIdx.x;
-    const uint32_t lane4 = (uint32_t)(tid & 31) << 2;
-    const int nbuf = (L + 1) >> 1;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int half = lane >> 4;
+    // byte 0 of a lookup address for slot s: (s << 6) | (replica << 2); slot = t ^ half.
+    const uint32_t rep4 = (uint32_t)(lane & 15) << 2;
+    const int nbuf = (L + kTablesPerBuf - 1) / kTablesPerBuf;
     const float* tu = tables + unit * L * (int64_t)NB;
     const uint8_t* idu = ids + unit * L * Ncap + first_group * 16;
     const float* vu = vnorm + unit * Ncap + first_group * 16;
@@ -104,18 +95,18 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
         for (int l = 0; l < min(L, kPrefetchAhead); ++l) prefetch_l2_bulk(idu + l * Ncap, pass_bytes);
     }
     uint4 cur[kGroupsPerThread];
-    load_ids(cur, idu, npg, tid);
+    load_round(cur, idu, Ncap, L, npg, tid, half, 0);
     // The soft tables come from the previous kernel on the stream.
     if (first_pass) pdl_wait();
 
     // Stage values for buffer bi: float4 slot e = i*kThreads + tid holds
-    // bucket e >> 4, table-in-pair (e >> 3) & 1, four lanes' copies.
+    // bucket e >> 4, table slot (e >> 2) & 3, replicas 4*(e & 3) .. +3.
     float stage[kStageSlots];
     auto load_stage = [&](int bi) {
 #pragma unroll
         for (int i = 0; i < kStageSlots; ++i) {
             const int e = i * kThreads + tid;
-            const int bucket = e >> 4, l = 2 * bi + ((e >> 3) & 1);
+            const int bucket = e >> 4, l = kTablesPerBuf * bi + ((e >> 2) & 3);
             stage[i] = (bucket < NB && l < L) ? __ldcg(tu + (int64_t)l * NB + bucket) : 0.0f;
         }
     };
@@ -140,22 +131,35 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[j][e] = 0.0f;
 
+    const int nrounds = nbuf * kTablesPerBuf;
     for (int bi = 0; bi < nbuf; ++bi) {
-        const uint32_t bbase = buf0 + (uint32_t)(bi & 1) * kBufBytes + lane4;
+        if (tid == 0) {
+            const int l0 = kTablesPerBuf * bi + kPrefetchAhead;
+            for (int l = l0; l < min(L, l0 + kTablesPerBuf); ++l) prefetch_l2_bulk(idu + l * Ncap, pass_bytes);
+        }
+        const uint32_t bbase = buf0 + (uint32_t)(bi & 1) * kBufBytes + rep4;
 #pragma unroll
-        for (int tt = 0; tt < 2; ++tt) {
-            const int l = 2 * bi + tt;
-            if (l < L) {
-                if (tid == 0 && l + kPrefetchAhead < L)
-                    prefetch_l2_bulk(idu + (l + kPrefetchAhead) * Ncap, pass_bytes);
-                uint4 nxt[kGroupsPerThread];
-                if (l + 1 < L) load_ids(nxt, idu + (l + 1) * Ncap, npg, tid);
-                lookup(acc, cur, bbase + (uint32_t)tt * 128u, npg, tid);
-                if (l + 1 < L) {
+        for (int t = 0; t < kTablesPerBuf; ++t) {
+            const int rr = kTablesPerBuf * bi + t;
+            uint4 nxt[kGroupsPerThread];
+            if (rr + 1 < nrounds) load_round(nxt, idu, Ncap, L, npg, tid, half, rr + 1);
+            // Rounds past table L-1 look up the zero-filled slots of the last buffer.
+            const uint32_t base = bbase + ((uint32_t)(t ^ half) << 6);
 #pragma unroll
-                    for (int j = 0; j < kGroupsPerThread; ++j) cur[j] = nxt[j];
+            for (int j = 0; j < kGroupsPerThread; ++j) {
+                const uint32_t words[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+#pragma unroll
+                    for (int byte = 0; byte < 4; ++byte) {
+                        // bytes 0, 2, 3 from base; byte 1 = the id
+                        const uint32_t addr = __byte_perm(base, words[w], 0x3240u + (byte << 4));
+                        acc[j][w * 4 + byte] += lds_f32(addr);
+                    }
                 }
             }
+#pragma unroll
+            for (int j = 0; j < kGroupsPerThread; ++j) cur[j] = nxt[j];
         }
         if (bi + 1 < nbuf) {
             store_stage((bi + 1) & 1);
@@ -164,7 +168,8 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
         __syncthreads();
     }
 
-    // Scores, and the largest score of a live key (n < N) of the pass.
+    // Scores, the largest score of a live key (n < N) of the pass, and the
+    // histogram of the live scores' top bits (bit pattern >> kHistShift).
     uint32_t mx = 0;
     const int64_t key0 = first_group * 16;
 #pragma unroll
@@ -181,10 +186,15 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
                 sc.w = acc[j][w * 4 + 3] * vn.w;
                 *reinterpret_cast<float4*>(su + (int64_t)g * 16 + w * 4) = sc;
                 const int64_t n = key0 + (int64_t)g * 16 + w * 4;
-                if (n + 0 < N) mx = max(mx, __float_as_uint(sc.x));
-                if (n + 1 < N) mx = max(mx, __float_as_uint(sc.y));
-                if (n + 2 < N) mx = max(mx, __float_as_uint(sc.z));
-                if (n + 3 < N) mx = max(mx, __float_as_uint(sc.w));
+                const uint32_t bits[4] = {__float_as_uint(sc.x), __float_as_uint(sc.y), __float_as_uint(sc.z),
+                                          __float_as_uint(sc.w)};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (n + e < N) {
+                        mx = max(mx, bits[e]);
+                        atomicAdd(shist + min(bits[e] >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
+                    }
+                }
             }
         }
     }
@@ -196,6 +206,15 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
         for (int w = 0; w < kThreads / 32; ++w) m = max(m, red[w]);
         atomicMax(unit_max + unit, m);
     }
+    // Flush the pass histogram into the unit's histogram and clear it.
+    uint32_t* gh = unit_hist + unit * kHistBins;
+    for (int b = tid; b < kHistBins; b += kThreads) {
+        const uint32_t c = shist[b];
+        if (c) {
+            atomicAdd(gh + b, c);
+            shist[b] = 0;
+        }
+    }
 }
 
 // Persistent grid: CTA c owns groups [c * per_cta, (c+1) * per_cta) of the
@@ -203,11 +222,13 @@ __device__ __forceinline__ void score_pass(const float* __restrict__ tables, con
 // and each piece into equal passes of at most kPassGroups groups.
 __global__ __launch_bounds__(kThreads, 1) void score_kernel(
     const float* __restrict__ tables, const uint8_t* __restrict__ ids, const float* __restrict__ vnorm,
-    float* __restrict__ scores, uint32_t* __restrict__ unit_max, int L, int NB, int64_t Ncap, int64_t N,
-    int64_t groups_per_unit, int64_t total_groups, int64_t groups_per_cta)
+    float* __restrict__ scores, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist, int L, int NB,
+    int64_t Ncap, int64_t N, int64_t groups_per_unit, int64_t total_groups, int64_t groups_per_cta)
 {
     extern __shared__ __align__(1024) char smem[];
     __shared__ uint32_t red[kThreads / 32];
+    __shared__ uint32_t shist[kHistBins];
+    for (int b = threadIdx.x; b < kHistBins; b += kThreads) shist[b] = 0;
     const uint32_t buf0 = (smem_addr(smem) + kBufBytes - 1) & ~(kBufBytes - 1);
     int64_t g = (int64_t)blockIdx.x * groups_per_cta;
     const int64_t g1 = min(total_groups, g + groups_per_cta);
@@ -220,7 +241,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(
         const int64_t npass = (seg + kPassGroups - 1) / kPassGroups;
         for (int64_t ip = 0; ip < npass; ++ip) {
             const int64_t a = g + seg * ip / npass, e = g + seg * (ip + 1) / npass;
-            score_pass(tables, ids, vnorm, scores, unit_max, smem, buf0, L, NB, Ncap, N, unit,
+            score_pass(tables, ids, vnorm, scores, unit_max, unit_hist, shist, smem, buf0, L, NB, Ncap, N, unit,
                        a - unit * groups_per_unit, (int)(e - a), first, red);
             first = false;
         }
@@ -239,7 +260,7 @@ int num_sms()
 }  // namespace
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         float* scores, uint32_t* unit_max, cudaStream_t stream)
+                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, cudaStream_t stream)
 {
     const int64_t gpu = (s.N + 15) / 16;
     const int64_t total = s.U * gpu;
@@ -250,7 +271,7 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(score_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, tables, ids, vnorm, scores,
-                   unit_max, s.L, s.NB, s.Ncap, s.N, gpu, total, per_cta);
+                   unit_max, unit_hist, s.L, s.NB, s.Ncap, s.N, gpu, total, per_cta);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -35,7 +35,8 @@ template <typename QT>
 __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int64_t Hq, int64_t Hkv, int G, int L,
     int P, double tau, float* __restrict__ tables, uint32_t* __restrict__ err_word,
-    uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max)
+    uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
+    uint32_t* __restrict__ cand_cnt)
 {
     // Dynamic shared memory, sized for the unit's G heads (see soft_tables_smem).
     extern __shared__ __align__(16) double dsm[];
@@ -52,10 +53,15 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const int NB = 1 << P;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    if (blockIdx.y == 0 && tid == 0) {
-        counters[u] = 0u;
-        unit_max[u] = 0u;
-        if (u == 0) *err_word = 0u;
+    if (blockIdx.y == 0) {
+        if (tid == 0) {
+            counters[u] = 0u;
+            unit_max[u] = 0u;
+            cand_cnt[u] = 0u;
+            if (u == 0) *err_word = 0u;
+        }
+        uint4* h = reinterpret_cast<uint4*>(unit_hist + u * kScoreHistBins);
+        for (int i = tid; i < kScoreHistBins / 4; i += kThreads) h[i] = make_uint4(0, 0, 0, 0);
     }
     // Let the scoring kernel start its table-independent prologue.
     pdl_launch_dependents();
@@ -126,7 +132,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
 
 cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
                                double tau, float* tables, uint32_t* err_word, uint32_t* counters,
-                               uint32_t* unit_max, cudaStream_t stream)
+                               uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream)
 {
     dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
     const size_t smem = sizeof(double) * ((size_t)s.G * kHeadDim + kMaxGroup + (size_t)s.G * kTablesPerBlock * kMaxP * 2 +
@@ -138,11 +144,11 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
     if (q_dtype == 1)
         soft_tables_kernel<uint16_t><<<grid, kThreads, smem, stream>>>(
             static_cast<const uint16_t*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
-            unit_max);
+            unit_max, unit_hist, cand_cnt);
     else
         soft_tables_kernel<float><<<grid, kThreads, smem, stream>>>(
             static_cast<const float*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
-            unit_max);
+            unit_max, unit_hist, cand_cnt);
     return cudaGetLastError();
 }
 

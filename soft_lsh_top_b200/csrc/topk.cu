@@ -9,12 +9,11 @@
 // index, and the chosen indices are written in ascending order.
 //
 // Scores are non-negative float32, so their bit patterns order like the
-// values.  A three-digit radix select (11 + 11 + 9 bits of the 31 magnitude
-// bits) finds the k-th largest pattern t and how many keys equal to t are
-// needed; one ordered compaction pass then keeps every key above t plus the
-// lowest-index keys equal to t.  A unit is handled by a thread-block cluster
-// of up to 16 CTAs that exchange histograms and counts through distributed
-// shared memory, so no global scratch and no second kernel are needed.
+// values.  The selection finds the bit pattern t of the k-th largest score
+// and the number of keys equal to t to keep (the lowest-index ones), then
+// writes every key above t and those ties in index order.  A unit is handled
+// by a thread-block cluster of up to 16 CTAs that exchange counts through
+// distributed shared memory; the paths are described at the kernel.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -25,15 +24,16 @@ namespace cg = cooperative_groups;
 namespace socket_attn {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kBins = 2048;
-constexpr int kBinsPerThread = kBins / kThreads;      // 4
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;                           // radix bins of the multi-pass path
 constexpr int kKeysPerThread = 16;                    // compaction: 16 consecutive keys per thread
-constexpr int kTileKeys = kThreads * kKeysPerThread;  // 8192
-constexpr int kSliceKeys = 16384;                     // target keys per CTA of a cluster
-constexpr int kCacheKeys = 16384;                     // keys of the CTA's slice kept in shared memory
+constexpr int kTileKeys = kThreads * kKeysPerThread;  // 4096
+constexpr int kSliceKeys = 32768;                     // target keys per CTA of a cluster
+constexpr int kBatch = 8;                             // 16-byte loads in flight per thread
 constexpr int kMaxCluster = 16;
-constexpr int kWindowShift = 15;                      // first-digit bin = 2^15 ulps (1/256 octave)
+constexpr int kWindowShift = 15;                      // multi-pass first digit: 2^15 ulps (1/256 octave)
+constexpr int kCand = kTopkCandidates;
 
 // Block-wide exclusive prefix sum of one uint32 per thread; also returns the total.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t& total)
@@ -48,190 +48,86 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
     if (lane == 31) warp_sums[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        uint32_t w = lane < kThreads / 32 ? warp_sums[lane] : 0u;
+        uint32_t w = lane < kWarps ? warp_sums[lane] : 0u;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(kFullMask, w, o);
             if (lane >= o) w += y;
         }
-        if (lane < kThreads / 32) warp_sums[lane] = w;  // inclusive over warps
+        if (lane < kWarps) warp_sums[lane] = w;  // inclusive over warps
     }
     __syncthreads();
-    total = warp_sums[kThreads / 32 - 1];
+    total = warp_sums[kWarps - 1];
     const uint32_t before = warp == 0 ? 0u : warp_sums[warp - 1];
     const uint32_t excl = before + x - v;
     __syncthreads();  // warp_sums reusable after return
     return excl;
 }
 
-// Position of 16-byte chunk c in the shared cache: XOR swizzle that keeps both
-// the coalesced pattern (chunk = base + lane) and the compaction pattern
-// (chunk = 4 * lane + q) free of bank conflicts.
-__device__ __forceinline__ int cache_pos(int c) { return c ^ ((c >> 3) & 3); }
-
-// Grid: U * C CTAs in clusters of C (one cluster per unit).  CTA r of a
-// cluster owns keys [r*R, min(N, (r+1)*R)) of its unit and keeps up to
-// kCacheKeys of them in shared memory.  Three radix digits of the score bit
-// pattern select the k-th largest: the first digit covers the 8 octaves
-// below the unit's largest score in 2048 bins of 1/256 octave (spread scores
-// over many bins, so the shared-memory atomics rarely collide); if fewer
-// than k keys fall in that window, the first digit is redone over the full
-// range (bits 30-20).  Every CTA sums the cluster's histograms through
-// distributed shared memory and picks the same digit.  Then each CTA counts
-// its keys above the threshold and equal to it; the counts of lower-ranked
-// CTAs give its output offset and tie budget, and it writes its selected
-// indices in index order.
-__global__ __launch_bounds__(kThreads) void topk_kernel(const float* __restrict__ scores,
-                                                        const uint32_t* __restrict__ unit_max, int64_t Ncap,
-                                                        int N, int k, int R, int32_t* __restrict__ idx_out)
-{
-    extern __shared__ uint4 cache[];
-    __shared__ uint32_t hist[kBins];
-    __shared__ uint32_t warp_sums[32];
-    __shared__ uint32_t s_digit, s_krem, s_total;
-    __shared__ uint32_t s_counts[2];
-
-    cg::cluster_group cluster = cg::this_cluster();
-    const unsigned rank = cluster.block_rank(), C = cluster.num_blocks();
-    const int tid = threadIdx.x;
-    const int64_t u = blockIdx.x / C;
-    const uint32_t* su = reinterpret_cast<const uint32_t*>(scores + u * Ncap);
-    int32_t* out = idx_out + u * (int64_t)k;
-    const int lo = (int)min64((int64_t)rank * R, N), hi = (int)min64((int64_t)lo + R, N);
-    const int n = hi - lo, ncache = min(n, kCacheKeys);
-
-    pdl_wait();  // scores and the unit maxima come from the previous kernel on the stream
-
-    const uint32_t maxbits = __ldcg(unit_max + u);
-    for (int i = tid * 4; i < ncache; i += kThreads * 4)
-        cache[cache_pos(i >> 2)] = __ldcg(reinterpret_cast<const uint4*>(su + lo + i));
-    // Four keys starting at offset i (a multiple of 4) of the CTA's range.
-    auto get4 = [&](int i) -> uint4 {
-        return i < ncache ? cache[cache_pos(i >> 2)] : __ldcg(reinterpret_cast<const uint4*>(su + lo + i));
+struct Shared {
+    uint32_t warp_sums[32];
+    uint32_t digit, krem, sure, total, pick, pick_above, grand;
+    uint32_t counts[2];
+    __align__(16) uint32_t hist[kBins];
+    union {  // the multi-pass path uses `slice`, the candidate path `cand`
+        __align__(16) uint32_t slice[kBins];
+        uint2 cand[kCand];  // (global index, bit pattern) of the unit's candidates
     };
+};
 
-    const uint32_t dmax = maxbits >> kWindowShift;
-    const uint32_t dlow = dmax >= (uint32_t)(kBins - 1) ? dmax - (kBins - 1) : 0u;
-    bool windowed = true;
-    uint32_t prefix = 0, mask = 0, krem = (uint32_t)k;
-    if (tid == 0) {
-        s_digit = 0;
-        s_krem = krem;
+// Finds, over bins given in descending order as per-thread runs of `nb`
+// counts c[0..nb) (thread t's run precedes thread t+1's), the bin holding the
+// krem-th key from the top: writes (bin id via `bin_of(t, q)`, keys still
+// needed inside it) to sh.digit / sh.krem.  `above` is the count above all bins.
+template <int NB, typename BinOf>
+__device__ __forceinline__ void find_bin(const uint32_t (&c)[NB], uint32_t above, uint32_t krem, Shared& sh,
+                                         BinOf bin_of)
+{
+    uint32_t sum = 0;
+#pragma unroll
+    for (int q = 0; q < NB; ++q) sum += c[q];
+    uint32_t total;
+    uint32_t run = above + block_exclusive_scan(sum, sh.warp_sums, total);
+#pragma unroll
+    for (int q = 0; q < NB; ++q) {
+        if (run < krem && krem <= run + c[q]) {
+            sh.digit = bin_of(q);
+            sh.krem = krem - run;
+        }
+        run += c[q];
     }
-    for (int pass = 0; pass < 3; ++pass) {
-        // Digit of this pass: bits [shift, shift + width) of the pattern
-        // (the first windowed digit is taken relative to dlow).
-        int shift, width;
-        if (windowed) {
-            shift = pass == 0 ? kWindowShift : pass == 1 ? 4 : 0;
-            width = pass == 0 ? 17 : pass == 1 ? 11 : 4;
-        } else {
-            shift = pass == 0 ? 20 : pass == 1 ? 9 : 0;
-            width = pass == 0 ? 11 : pass == 1 ? 11 : 9;
-        }
-        const uint32_t dmask = width >= 32 ? 0xffffffffu : (1u << width) - 1u;
-        for (int b = tid; b < kBins; b += kThreads) hist[b] = 0;
-        __syncthreads();
-        for (int i = tid * 4; i < n; i += kThreads * 4) {
-            const uint4 v = get4(i);
-            const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                if (i + e < n) {
-                    const uint32_t x = vals[e];
-                    if (pass == 0 && windowed) {
-                        const uint32_t dgt = x >> kWindowShift;
-                        if (dgt >= dlow) atomicAdd(&hist[min(dgt - dlow, (uint32_t)(kBins - 1))], 1u);
-                    } else if ((x & mask) == prefix) {
-                        atomicAdd(&hist[(x >> shift) & dmask], 1u);
-                    }
-                }
-            }
-        }
-        cluster.sync();  // every CTA's histogram is complete
-        // Thread t owns bins b0, b0-1, b0-2, b0-3 with b0 = 2047 - 4t (descending order).
-        const int b0 = kBins - 1 - kBinsPerThread * tid;
-        uint32_t c[kBinsPerThread] = {0, 0, 0, 0};
-        for (unsigned r = 0; r < C; ++r) {
-            const uint32_t* rh = cluster.map_shared_rank(hist, r);
-#pragma unroll
-            for (int q = 0; q < kBinsPerThread; ++q) c[q] += rh[b0 - q];
-        }
-        uint32_t total;
-        uint32_t run = block_exclusive_scan(c[0] + c[1] + c[2] + c[3], warp_sums, total);
-#pragma unroll
-        for (int q = 0; q < kBinsPerThread; ++q) {
-            if (run < krem && krem <= run + c[q]) {
-                s_digit = (uint32_t)(b0 - q);
-                s_krem = krem - run;
-            }
-            run += c[q];
-        }
-        if (tid == 0) s_total = total;
-        cluster.sync();  // remote histograms read; s_digit, s_total visible
-        if (pass == 0 && windowed && s_total < krem) {
-            // The k-th largest score lies below the window: redo the first
-            // digit over the full range.
-            windowed = false;
-            pass = -1;
-            continue;
-        }
-        if (pass == 0 && windowed) {
-            prefix = (s_digit + dlow) << kWindowShift;
-            mask = 0xffffffffu << kWindowShift;
-        } else {
-            prefix |= s_digit << shift;
-            mask |= dmask << shift;
-        }
-        krem = s_krem;
-    }
+}
 
-    // prefix = bit pattern of the unit's k-th largest score; krem = keys equal
-    // to it that are kept (the lowest-index ones).
-    const uint32_t t = prefix, need_ties = krem;
-    uint32_t gt = 0, eq = 0;
-    for (int i = tid * 4; i < n; i += kThreads * 4) {
-        const uint4 v = get4(i);
-        const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
+// Writes this CTA's selected indices (keys of [lo, hi) above t, plus the first
+// `budget` keys equal to t) in index order from position out_base.
+__device__ __forceinline__ void load_tile(uint32_t (&vals)[kKeysPerThread], const uint32_t* su, int lo, int n, int i0)
+{
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (i + e < n) {
-                gt += vals[e] > t;
-                eq += vals[e] == t;
-            }
-        }
+    for (int q = 0; q < kKeysPerThread / 4; ++q) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i0 + 4 * q < n) v = __ldcg(reinterpret_cast<const uint4*>(su + lo + i0 + 4 * q));
+        vals[4 * q + 0] = v.x;
+        vals[4 * q + 1] = v.y;
+        vals[4 * q + 2] = v.z;
+        vals[4 * q + 3] = v.w;
     }
-    uint32_t tot_gt, tot_eq;
-    block_exclusive_scan(gt, warp_sums, tot_gt);
-    block_exclusive_scan(eq, warp_sums, tot_eq);
-    if (tid == 0) {
-        s_counts[0] = tot_gt;
-        s_counts[1] = tot_eq;
-    }
-    cluster.sync();
-    uint32_t out_base = 0, ties_before = 0;
-    for (unsigned r = 0; r < rank; ++r) {
-        const uint32_t* rc = cluster.map_shared_rank(s_counts, r);
-        const uint32_t rgt = rc[0], req = rc[1];
-        const uint32_t budget = need_ties > ties_before ? need_ties - ties_before : 0u;
-        out_base += rgt + min(req, budget);
-        ties_before += req;
-    }
-    cluster.sync();  // no remote shared-memory access after this point
+}
 
-    uint32_t ties_seen = ties_before;
+// Writes this CTA's selected indices (keys of [lo, hi) above t, plus the first
+// `budget` keys equal to t) in index order from position out_base.  Each
+// tile's loads are issued before the previous tile's scan.
+__device__ __forceinline__ void compact(const uint32_t* su, int lo, int hi, uint32_t t, uint32_t budget,
+                                        uint32_t out_base, int k, int32_t* out, Shared& sh)
+{
+    const int tid = threadIdx.x;
+    const int n = hi - lo;
+    uint32_t ties_seen = 0;
+    uint32_t vals[kKeysPerThread];
+    load_tile(vals, su, lo, n, tid * kKeysPerThread);
     for (int tile = 0; tile < n; tile += kTileKeys) {
         const int i0 = tile + tid * kKeysPerThread;
-        uint32_t vals[kKeysPerThread];
-#pragma unroll
-        for (int q = 0; q < kKeysPerThread / 4; ++q) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (i0 + 4 * q < n) v = get4(i0 + 4 * q);
-            vals[4 * q + 0] = v.x;
-            vals[4 * q + 1] = v.y;
-            vals[4 * q + 2] = v.z;
-            vals[4 * q + 3] = v.w;
-        }
+        uint32_t next[kKeysPerThread];
+        if (tile + kTileKeys < n) load_tile(next, su, lo, n, i0 + kTileKeys);
         uint32_t tgt = 0, teq = 0;
 #pragma unroll
         for (int e = 0; e < kKeysPerThread; ++e) {
@@ -241,10 +137,10 @@ __global__ __launch_bounds__(kThreads) void topk_kernel(const float* __restrict_
             }
         }
         uint32_t total;
-        const uint32_t excl = block_exclusive_scan((tgt << 16) | teq, warp_sums, total);
+        const uint32_t excl = block_exclusive_scan((tgt << 16) | teq, sh.warp_sums, total);
         const uint32_t gt_before = excl >> 16, eq_before = excl & 0xffffu;
-        const uint32_t budget = need_ties > ties_seen ? need_ties - ties_seen : 0u;
-        uint32_t pos = out_base + gt_before + min(eq_before, budget);
+        const uint32_t left = budget > ties_seen ? budget - ties_seen : 0u;
+        uint32_t pos = out_base + gt_before + min(eq_before, left);
         uint32_t my_eq = eq_before;
 #pragma unroll
         for (int e = 0; e < kKeysPerThread; ++e) {
@@ -255,7 +151,7 @@ __global__ __launch_bounds__(kThreads) void topk_kernel(const float* __restrict_
                     if (pos < (uint32_t)k) out[pos] = lo + i0 + e;
                     ++pos;
                 } else if (vals[e] == t) {
-                    if (my_eq < budget) {
+                    if (my_eq < left) {
                         if (pos < (uint32_t)k) out[pos] = lo + i0 + e;
                         ++pos;
                     }
@@ -263,28 +159,323 @@ __global__ __launch_bounds__(kThreads) void topk_kernel(const float* __restrict_
                 }
             }
         }
-        out_base += (total >> 16) + min(total & 0xffffu, budget);
+        out_base += (total >> 16) + min(total & 0xffffu, left);
         ties_seen += total & 0xffffu;
+#pragma unroll
+        for (int e = 0; e < kKeysPerThread; ++e) vals[e] = next[e];
     }
+}
+
+// Multi-pass radix select over the cluster (any score distribution): three
+// digits of the bit pattern; the first covers the 8 octaves below the unit's
+// largest score in 2048 bins of 1/256 octave, redone over the full range
+// (bits 30-20) if fewer than k keys fall in that window.  Histograms are
+// combined through distributed shared memory: CTA r sums the r-th 1/C of the
+// bins over the cluster, the slice totals locate the slice holding the k-th
+// key, and every CTA scans that slice, so all pick the same digit.
+// Returns the threshold pattern t and the ties at t to keep in *need.
+__device__ uint32_t select_multipass(cg::cluster_group& cluster, const uint32_t* su, int lo, int hi,
+                                     uint32_t maxbits, int k, Shared& sh, uint32_t* need)
+{
+    const unsigned rank = cluster.block_rank(), C = cluster.num_blocks();
+    const int tid = threadIdx.x;
+    const int n = hi - lo;
+    const uint32_t dmax = maxbits >> kWindowShift;
+    const uint32_t dlow = dmax >= (uint32_t)(kBins - 1) ? dmax - (kBins - 1) : 0u;
+    bool windowed = true;
+    uint32_t prefix = 0, mask = 0, krem = (uint32_t)k;
+    for (int pass = 0; pass < 3; ++pass) {
+        int shift, width;
+        if (windowed) {
+            shift = pass == 0 ? kWindowShift : pass == 1 ? 4 : 0;
+            width = pass == 0 ? 17 : pass == 1 ? 11 : 4;
+        } else {
+            shift = pass == 0 ? 20 : pass == 1 ? 9 : 0;
+            width = pass == 0 ? 11 : pass == 1 ? 11 : 9;
+        }
+        const uint32_t dmask = (1u << width) - 1u;
+        for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+        __syncthreads();
+        for (int i = tid * 4; i < n; i += kThreads * 4) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(su + lo + i));
+            const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (i + e < n) {
+                    const uint32_t x = vals[e];
+                    if (pass == 0 && windowed) {
+                        const uint32_t dgt = x >> kWindowShift;
+                        if (dgt >= dlow) atomicAdd(&sh.hist[min(dgt - dlow, (uint32_t)(kBins - 1))], 1u);
+                    } else if ((x & mask) == prefix) {
+                        atomicAdd(&sh.hist[(x >> shift) & dmask], 1u);
+                    }
+                }
+            }
+        }
+        cluster.sync();  // every CTA's histogram is complete
+        const int S = kBins / (int)C;
+        const int s0 = (int)rank * S;
+        uint32_t part = 0;
+        for (int i = tid; i < S / 4; i += kThreads) {
+            uint4 acc4 = make_uint4(0, 0, 0, 0);
+            for (unsigned r = 0; r < C; ++r) {
+                const uint4 v = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(sh.hist, r) + s0 + 4 * i);
+                acc4.x += v.x;
+                acc4.y += v.y;
+                acc4.z += v.z;
+                acc4.w += v.w;
+            }
+            *reinterpret_cast<uint4*>(sh.slice + 4 * i) = acc4;
+            part += acc4.x + acc4.y + acc4.z + acc4.w;
+        }
+        uint32_t slice_total;
+        block_exclusive_scan(part, sh.warp_sums, slice_total);
+        if (tid == 0) sh.total = slice_total;
+        cluster.sync();  // slices and slice totals complete
+        if (tid == 0) {
+            uint32_t above = 0, pick_above = 0;
+            int pick = -1;
+            for (int r = (int)C - 1; r >= 0; --r) {
+                const uint32_t t = *cluster.map_shared_rank(&sh.total, (unsigned)r);
+                if (pick < 0 && above + t >= krem) {
+                    pick = r;
+                    pick_above = above;
+                }
+                above += t;
+            }
+            sh.pick = pick < 0 ? 0u : (uint32_t)pick;
+            sh.pick_above = pick_above;
+            sh.grand = above;
+        }
+        __syncthreads();
+        {
+            // Thread t owns bins b0, b0-1, ..., b0-7 (b0 = S-1-8t) of the picked slice.
+            const uint32_t* ps = cluster.map_shared_rank(sh.slice, sh.pick);
+            const int b0 = S - 1 - 8 * tid;
+            uint32_t c[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (b0 >= 7) {
+                const uint4 v0 = *reinterpret_cast<const uint4*>(ps + b0 - 7);
+                const uint4 v1 = *reinterpret_cast<const uint4*>(ps + b0 - 3);
+                c[0] = v1.w; c[1] = v1.z; c[2] = v1.y; c[3] = v1.x;
+                c[4] = v0.w; c[5] = v0.z; c[6] = v0.y; c[7] = v0.x;
+            }
+            const uint32_t pick = sh.pick;
+            find_bin<8>(c, sh.pick_above, krem, sh, [&](int q) { return pick * (uint32_t)S + (uint32_t)(b0 - q); });
+        }
+        cluster.sync();  // remote slices read; digit, krem, grand visible
+        if (pass == 0 && windowed && sh.grand < krem) {
+            windowed = false;  // the k-th score lies below the window
+            pass = -1;
+            continue;
+        }
+        if (pass == 0 && windowed) {
+            prefix = (sh.digit + dlow) << kWindowShift;
+            mask = 0xffffffffu << kWindowShift;
+        } else {
+            prefix |= sh.digit << shift;
+            mask |= dmask << shift;
+        }
+        krem = sh.krem;
+    }
+    *need = krem;
+    return prefix;
+}
+
+// Grid: U * C CTAs in clusters of C (a power of two; one cluster per unit).
+// CTA r of a cluster owns keys [r*R, min(N, (r+1)*R)) of its unit.
+//
+// Fast path.  The scoring kernel left a histogram of the unit's score bit
+// patterns >> 19 (1/16 octave per bin).  Every CTA reads it and finds the bin
+// d0 holding the k-th largest score; the keys above that bin are selected for
+// sure, and the keys inside it (a few hundred on typical data) are the
+// candidates.  Each CTA appends its candidates (index, pattern) to the unit's
+// candidate list, every CTA then loads the whole list and selects among it
+// with two more radix digits (11 + 8 bits) in its own shared memory -- the
+// same exact threshold t and tie count everywhere.  The CTA's output offset
+// follows from the "sure" counts of lower-ranked CTAs (distributed shared
+// memory) and the candidate list, and it writes its selected indices in
+// index order.  If the threshold bin holds more than kTopkCandidates keys,
+// the cluster takes the multi-pass path instead.
+__global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restrict__ scores,
+                                                        const uint32_t* __restrict__ unit_max,
+                                                        const uint32_t* __restrict__ unit_hist,
+                                                        uint32_t* __restrict__ cand_cnt, uint2* __restrict__ cand,
+                                                        int64_t Ncap, int N, int k, int R,
+                                                        int32_t* __restrict__ idx_out)
+{
+    __shared__ Shared sh;
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned rank = cluster.block_rank(), C = cluster.num_blocks();
+    const int tid = threadIdx.x;
+    const int64_t u = blockIdx.x / C;
+    const uint32_t* su = reinterpret_cast<const uint32_t*>(scores + u * Ncap);
+    int32_t* out = idx_out + u * (int64_t)k;
+    const int lo = (int)min64((int64_t)rank * R, N), hi = (int)min64((int64_t)lo + R, N);
+    const int n = hi - lo;
+
+    pdl_wait();  // scores, maxima and histograms come from the previous kernel on the stream
+
+    // ---- the unit histogram: bin d0 of the k-th largest score.
+    {
+        constexpr int kPer = kScoreHistBins / kThreads;  // 16 bins per thread, descending
+        const int b0 = kScoreHistBins - 1 - kPer * tid;
+        const uint4* hp = reinterpret_cast<const uint4*>(unit_hist + u * kScoreHistBins + (b0 - (kPer - 1)));
+        uint32_t c[kPer];
+#pragma unroll
+        for (int v = 0; v < kPer / 4; ++v) {
+            const uint4 w = __ldcg(hp + (kPer / 4 - 1 - v));
+            c[4 * v + 0] = w.w;
+            c[4 * v + 1] = w.z;
+            c[4 * v + 2] = w.y;
+            c[4 * v + 3] = w.x;
+        }
+        if (tid == 0) {
+            sh.digit = 0;
+            sh.krem = (uint32_t)k;
+        }
+        __syncthreads();
+        find_bin<kPer>(c, 0u, (uint32_t)k, sh, [&](int q) { return (uint32_t)(b0 - q); });
+        __syncthreads();
+    }
+    const uint32_t d0 = sh.digit, krem0 = sh.krem;
+    const uint32_t ncand = __ldcg(unit_hist + u * kScoreHistBins + d0);
+
+    uint32_t t, need, out_base, budget;
+    if (ncand > (uint32_t)kCand) {
+        t = select_multipass(cluster, su, lo, hi, __ldcg(unit_max + u), k, sh, &need);
+        uint32_t gt = 0, eq = 0;
+        for (int i = tid * 4; i < n; i += kThreads * 4) {
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(su + lo + i));
+            const uint32_t vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (i + e < n) {
+                    gt += vals[e] > t;
+                    eq += vals[e] == t;
+                }
+            }
+        }
+        uint32_t tot_gt, tot_eq;
+        block_exclusive_scan(gt, sh.warp_sums, tot_gt);
+        block_exclusive_scan(eq, sh.warp_sums, tot_eq);
+        if (tid == 0) {
+            sh.counts[0] = tot_gt;
+            sh.counts[1] = tot_eq;
+        }
+        cluster.sync();
+        out_base = 0;
+        uint32_t ties_before = 0;
+        for (unsigned r = 0; r < rank; ++r) {
+            const uint32_t* rc = cluster.map_shared_rank(sh.counts, r);
+            const uint32_t b = need > ties_before ? need - ties_before : 0u;
+            out_base += rc[0] + min(rc[1], b);
+            ties_before += rc[1];
+        }
+        budget = need > ties_before ? need - ties_before : 0u;
+        cluster.sync();  // no remote shared-memory access after this point
+    } else {
+        // ---- candidates of this slice -> the unit list; count keys above bin d0.
+        uint32_t sure = 0;
+        for (int base = tid * 4; base < n; base += kThreads * 4 * kBatch) {
+            uint4 v[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int i = base + b * kThreads * 4;
+                v[b] = i < n ? __ldcg(reinterpret_cast<const uint4*>(su + lo + i)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int i = base + b * kThreads * 4;
+                const uint32_t vals[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (i + e < n) {
+                        const uint32_t top = vals[e] >> kScoreHistShift;
+                        sure += top > d0;
+                        if (top == d0) {
+                            const uint32_t slot = atomicAdd(cand_cnt + u, 1u);
+                            if (slot < (uint32_t)kCand)
+                                cand[u * kCand + slot] = make_uint2((uint32_t)(lo + i + e), vals[e]);
+                        }
+                    }
+                }
+            }
+        }
+        uint32_t sure_total;
+        block_exclusive_scan(sure, sh.warp_sums, sure_total);
+        if (tid == 0) sh.sure = sure_total;
+        __threadfence();
+        cluster.sync();  // candidate list complete; sure counts visible
+        if (tid == 0) {
+            uint32_t before = 0;
+            for (unsigned r = 0; r < rank; ++r) before += *cluster.map_shared_rank(&sh.sure, r);
+            sh.pick_above = before;
+        }
+        const int nc = (int)min(ncand, (uint32_t)kCand);
+        for (int i = tid; i < nc; i += kThreads) sh.cand[i] = __ldcg(cand + u * kCand + i);
+        cluster.sync();  // no remote shared-memory access after this point
+        const uint32_t sure_before = sh.pick_above;
+
+        // ---- the krem0-th largest among the candidates: digits 18-8 and 7-0.
+        uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, krem = krem0;
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 8 : 0;
+            const uint32_t dmask = pass == 0 ? 0x7ffu : 0xffu;
+            for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+            __syncthreads();
+            for (int i = tid; i < nc; i += kThreads) {
+                const uint32_t x = sh.cand[i].y;
+                if ((x & mask) == prefix) atomicAdd(&sh.hist[(x >> shift) & dmask], 1u);
+            }
+            __syncthreads();
+            constexpr int kPer = kBins / kThreads;  // 8 bins per thread, descending
+            const int b0 = kBins - 1 - kPer * tid;
+            uint32_t c[kPer];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) c[q] = sh.hist[b0 - q];
+            find_bin<kPer>(c, 0u, krem, sh, [&](int q) { return (uint32_t)(b0 - q); });
+            __syncthreads();
+            prefix |= sh.digit << shift;
+            mask |= dmask << shift;
+            krem = sh.krem;
+            __syncthreads();
+        }
+        t = prefix;
+        need = krem;
+        // Keys before this slice that are selected: sure keys of lower CTAs,
+        // candidates above t before lo, and ties at t before lo (up to need).
+        uint32_t gt_before = 0, eq_before = 0;
+        for (int i = tid; i < nc; i += kThreads) {
+            const uint2 e = sh.cand[i];
+            if ((int)e.x < lo) {
+                gt_before += e.y > t;
+                eq_before += e.y == t;
+            }
+        }
+        uint32_t tg, te;
+        block_exclusive_scan(gt_before, sh.warp_sums, tg);
+        block_exclusive_scan(eq_before, sh.warp_sums, te);
+        out_base = sure_before + tg + min(te, need);
+        budget = need > te ? need - te : 0u;
+    }
+    compact(su, lo, hi, t, budget, out_base, k, out, sh);
 }
 
 }  // namespace
 
-cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const DecodeShape& s, int32_t* idx_out,
-                        cudaStream_t stream)
+cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const uint32_t* unit_hist,
+                        uint32_t* cand_cnt, uint2* cand, const DecodeShape& s, int32_t* idx_out, cudaStream_t stream)
 {
     const int64_t want = (s.N + kSliceKeys - 1) / kSliceKeys;
-    const int C = (int)max64(1, min64(kMaxCluster, want));
+    int C = 1;  // a power of two, so the multi-pass bins split evenly over the cluster
+    while (C < kMaxCluster && C < want) C *= 2;
     const int R = (int)(((s.N + C - 1) / C + 31) / 32 * 32);
-    const int smem = (int)min64(R, kCacheKeys) * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCacheKeys * 4);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(s.U * C));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -295,7 +486,8 @@ cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const Dec
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl_enabled() ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, topk_kernel, scores, unit_max, s.Ncap, (int)s.N, s.k, R, idx_out);
+    e = cudaLaunchKernelEx(&cfg, topk_kernel, scores, unit_max, unit_hist, cand_cnt, cand, s.Ncap, (int)s.N, s.k, R,
+                           idx_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
