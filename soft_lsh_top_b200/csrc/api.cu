@@ -204,8 +204,8 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
         !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
         return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
     if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
-    // Splits follow the kv dtype's chunk; the advertised size covers the smallest chunk.
-    s.nsplit = (k + attention_chunk_rows(kv_dtype) - 1) / attention_chunk_rows(kv_dtype);
+    // Splits are at most ceil(k / chunk rows); the advertised size covers the smallest chunk.
+    s.nsplit = attention_splits(kv_dtype, s.U, k, device_num_sms());
     const size_t need = socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k);
     if (workspace_bytes < need)
         return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);

@@ -43,8 +43,12 @@ struct DecodeWorkspace {
 
 DecodeWorkspace decode_workspace_layout(const DecodeShape& s);
 
-// Rows of the key/value gather handled by one attention CTA.
+// Rows of one attention chunk (the gather unit of the attention kernel).
 int attention_chunk_rows(int kv_dtype);
+// Attention CTAs per unit for these sizes (<= ceil(k / chunk rows)).
+int attention_splits(int kv_dtype, int64_t U, int k, int num_sms);
+int attention_rows_per_cta(int k, int nsplit, int chunk);
+int device_num_sms();
 
 // --- kernels (each returns cudaGetLastError() after its launch) -------------
 cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv,

@@ -249,15 +249,15 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(
     }
 }
 
-int num_sms()
+}  // namespace
+
+int device_num_sms()
 {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n > 0 ? n : 1;
 }
-
-}  // namespace
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
                          float* scores, uint32_t* unit_max, uint32_t* unit_hist, cudaStream_t stream)
@@ -266,7 +266,7 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     const int64_t total = s.U * gpu;
     // At least ~8192 keys per CTA so the table staging stays amortised.
     const int64_t want = (total + 511) / 512;
-    const int grid = (int)max64(1, min64(num_sms(), want));
+    const int grid = (int)max64(1, min64(device_num_sms(), want));
     const int64_t per_cta = (total + grid - 1) / grid;
     cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;

@@ -26,6 +26,11 @@ SMALL = {
     "odd_group3_p5": wl.Workload(name="odd", B=2, Hq=6, Hkv=2, N=3001, L=7, P=5, tau=0.7, k=77, seed=7002),
     "f32_group2_p6": wl.Workload(name="f32g2", B=1, Hq=4, Hkv=2, N=2500, L=9, P=6, tau=0.25, k=100, dtype="f32",
                                  seed=7003),
+    # bfloat16 at the group sizes that bound the attention kernels: one head,
+    # eight heads (the widest tensor-core tile) and sixteen (the CUDA-core path).
+    "bf16_single_head": wl.Workload(name="g1", B=2, Hq=2, Hkv=2, N=4099, L=8, P=8, tau=0.3, k=200, seed=7005),
+    "bf16_group8_p7": wl.Workload(name="g8", B=1, Hq=16, Hkv=2, N=5000, L=10, P=7, tau=0.5, k=300, seed=7006),
+    "bf16_group16": wl.Workload(name="g16", B=1, Hq=16, Hkv=1, N=3000, L=6, P=8, tau=0.4, k=129, seed=7007),
 }
 
 
