@@ -265,6 +265,10 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     w = wl.WORKLOADS[args.workload]
+    if args.batch and args.batch != w.B:
+        # A smaller batch of the same workload (profiling captures); renamed so
+        # nothing measured on it passes for the full workload.
+        w = w.scaled(B=args.batch, name=f"{w.name}_batch{args.batch}")
     R = args.layers
     layers = []
     for li in range(R):
@@ -385,6 +389,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=wl.BATCH8_128K.name, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--layers", type=int, default=3, help="independently drawn layers rotated across steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -63,7 +63,8 @@ extern "C" {
  * 0 means every wait completed.
  */
 #define SOCKET_WS_ERROR_OFFSET 0
-#define SOCKET_DEVERR_GATHER_TIMEOUT 0x1u
+#define SOCKET_DEVERR_GATHER_TIMEOUT 0x1u  /* attention: a key/value row gather */
+#define SOCKET_DEVERR_TABLE_TIMEOUT  0x2u  /* scoring: a soft-table copy into shared memory */
 
 /*
  * socket_hash_keys -- prefill hashing ([ES] step 1 "Pre-cálculo (Prellenado)";
@@ -78,8 +79,12 @@ extern "C" {
  *   K, V      device, [B][Hkv][Ncap][d] of kv_dtype, 16-byte aligned.
  *   W         device, [L][P][d] bfloat16 bits (one set of hyperplanes shared
  *             by every batch row and head), 16-byte aligned.
- *   ids       device out, [B][Hkv][L][Ncap] uint8 (table-major per unit),
- *             16-byte aligned.
+ *   ids       device out, [B][Hkv][Ncap][Lr] uint8, Lr = socket_ids_row_bytes(L)
+ *             = 32 * ceil(L / 32), 16-byte aligned: one row of Lr bytes per
+ *             key, in blocks of 32 slots.  Slot s of block c of key n holds the
+ *             id of table 32c + (s + n) mod 32 when that table is < L, else 0.
+ *             (The rotation by n lets the 32 lanes of a warp, scoring keys
+ *             32m .. 32m + 31, read 32 different tables in every lookup.)
  *   vnorm     device out, [B][Hkv][Ncap] float32, 16-byte aligned.
  * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Ncap % 16 == 0;
  * 0 <= n_begin <= n_end <= Ncap.  n_begin == n_end queues nothing.
@@ -91,6 +96,12 @@ int socket_hash_keys(const void* K, const void* V, int kv_dtype,
                      int64_t n_begin, int64_t n_end, int64_t d,
                      const uint16_t* W, int L, int P,
                      uint8_t* ids, float* vnorm, void* stream);
+
+/*
+ * socket_ids_row_bytes -- bytes of one key's id row for L tables
+ * (32 * ceil(L / 32)), or 0 if L is outside 1..SOCKET_MAX_L.
+ */
+int socket_ids_row_bytes(int L);
 
 /*
  * socket_decode_workspace_size -- bytes of device scratch socket_decode needs

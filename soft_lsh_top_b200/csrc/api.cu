@@ -119,7 +119,7 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     w.cand = off;
     off = align256(off + 8 * (size_t)s.U * kTopkCandidates);
     w.tables = off;
-    off = align256(off + 4 * (size_t)s.U * s.L * s.NB);
+    off = align256(off + 4 * (size_t)s.U * ((s.L + 31) / 32) * s.NB * 64);
     w.scores = off;
     off = align256(off + 4 * (size_t)s.U * s.Ncap);
     w.part_o = off;
@@ -136,7 +136,7 @@ using namespace socket_attn;
 
 extern "C" {
 
-int socket_version(void) { return 100; }
+int socket_version(void) { return 200; }
 
 int socket_set_step_events(void* const* events, int n)
 {
@@ -171,6 +171,8 @@ int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int6
                                         static_cast<cudaStream_t>(stream)),
                        "hash kernel launch");
 }
+
+int socket_ids_row_bytes(int L) { return (L >= 1 && L <= SOCKET_MAX_L) ? ids_row_bytes(L) : 0; }
 
 size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P,
                                     int k)
@@ -228,7 +230,7 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
     st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt, cs), "soft-table kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, cs), "score kernel launch");
+    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, err_word, cs), "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
     st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");

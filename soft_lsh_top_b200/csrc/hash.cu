@@ -40,6 +40,8 @@ __global__ __launch_bounds__(kThreads) void hash_kernel(const KT* __restrict__ K
 {
     __shared__ float ks[kKeys][kKPad];
     __shared__ uint32_t ws[kTablesPerStage * 8 * kHeadDim / 2];  // bf16 pairs, [table][plane][d/2]
+    extern __shared__ __align__(16) uint8_t idrow[];              // [kKeys][Lr] rotated id rows
+    const int Lr = 32 * ((L + 31) / 32);
 
     const int tid = threadIdx.x;
     const int64_t u = blockIdx.y;
@@ -52,6 +54,7 @@ __global__ __launch_bounds__(kThreads) void hash_kernel(const KT* __restrict__ K
         const int r = e / kHeadDim, j = e % kHeadDim;
         ks[r][j] = r < nk ? elem(Ku, (n0 + r) * kHeadDim + j) : 0.0f;
     }
+    for (int e = tid; e < kKeys * Lr / 16; e += kThreads) reinterpret_cast<uint4*>(idrow)[e] = make_uint4(0, 0, 0, 0);
 
     const int key = tid % kKeys, tg = tid / kKeys;
     const int64_t n = n0 + key;
@@ -95,9 +98,15 @@ __global__ __launch_bounds__(kThreads) void hash_kernel(const KT* __restrict__ K
 #pragma unroll
             for (int p = 0; p < 8; ++p)
                 if (p < P && y[p] > 0.0f) id |= 1u << p;
-            if (key < nk) ids[(u * L + l0 + lt) * Ncap + n] = (uint8_t)id;
+            // Slot of table l in key n's row: 32 (l / 32) + (l - n) mod 32.
+            const int l = l0 + lt;
+            idrow[key * Lr + (l & ~31) + (((l & 31) - (int)(n & 31)) & 31)] = (uint8_t)id;
         }
     }
+    __syncthreads();
+    // Keys n0 .. n0 + nk - 1 are consecutive rows of the unit's id array.
+    uint4* dst = reinterpret_cast<uint4*>(ids + (u * Ncap + n0) * Lr);
+    for (int e = tid; e < nk * Lr / 16; e += kThreads) dst[e] = reinterpret_cast<const uint4*>(idrow)[e];
 }
 
 }  // namespace
@@ -108,12 +117,16 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
 {
     const int64_t nkeys = n_end - n_begin;
     dim3 grid((unsigned)((nkeys + kKeys - 1) / kKeys), (unsigned)(B * Hkv));
+    const int smem = kKeys * 32 * ((L + 31) / 32);
+    cudaError_t e = cudaFuncSetAttribute(kv_dtype == 1 ? (const void*)hash_kernel<uint16_t> : (const void*)hash_kernel<float>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
     if (kv_dtype == 1)
-        hash_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(K),
+        hash_kernel<uint16_t><<<grid, kThreads, smem, stream>>>(static_cast<const uint16_t*>(K),
                                                             static_cast<const uint16_t*>(V), Ncap, n_begin, n_end,
                                                             W, L, P, ids, vnorm);
     else
-        hash_kernel<float><<<grid, kThreads, 0, stream>>>(static_cast<const float*>(K), static_cast<const float*>(V),
+        hash_kernel<float><<<grid, kThreads, smem, stream>>>(static_cast<const float*>(K), static_cast<const float*>(V),
                                                          Ncap, n_begin, n_end, W, L, P, ids, vnorm);
     return cudaGetLastError();
 }

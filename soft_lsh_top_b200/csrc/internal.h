@@ -34,7 +34,7 @@ struct DecodeWorkspace {
     size_t unit_hist;  // uint32 [U][kScoreHistBins] score histogram
     size_t cand_cnt;   // uint32 [U] top-k candidate counters
     size_t cand;       // uint2 [U][kTopkCandidates] top-k candidates (index, bit pattern)
-    size_t tables;     // float [U][L][NB]
+    size_t tables;     // float [U][ceil(L/32)][NB][64], column j = table 32c + j mod 32
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
     size_t part_ml;    // float2 [U][G][nsplit]
@@ -61,9 +61,11 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                double tau, float* tables, uint32_t* err_word, uint32_t* counters,
                                uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream);
 
-cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm,
-                         const DecodeShape& s, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
+cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
+                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* err_word,
                          cudaStream_t stream);
+// Bytes of one key's rotated id row (32 per started block of 32 tables).
+int ids_row_bytes(int L);
 
 cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const uint32_t* unit_hist,
                         uint32_t* cand_cnt, uint2* cand, const DecodeShape& s, int32_t* idx_out, cudaStream_t stream);

@@ -10,43 +10,44 @@
 // pages implement this step as "a custom CUDA scoring kernel"
 // ("Contribuciones Clave" 2 / "Hauptbeiträge").
 //
-// B200 design.  The step streams L + 4 bytes per key from HBM (one uint8 id
-// per table, table-major, plus the fp32 norm) and performs L random lookups
-// into 2^P-entry tables.  Lookups go to shared memory in a lane-private
-// layout: a 64 KB buffer holds four tables as float[256 buckets][4 tables]
-// [16 replicas]; lane j uses replica j % 16, and the two half-warps look up
-// different tables of the buffer in the same instruction (round t: slot
-// t ^ half), so a warp's 32 random lookups land in 32 distinct banks -- one
-// conflict-free wavefront whatever the ids are.  The buffers sit at 64 KB-
-// aligned shared addresses, so one byte-permute of the packed id word yields
-// the full shared address of a lookup.  Each
-// thread keeps 64 keys' accumulators in registers across all L tables, so a
-// pass covers 32768 keys per CTA and the 64 KB table staging per table pair
-// is amortised over them.  Ids are read with 16-byte streaming loads one table
-// ahead in registers and several tables ahead through bulk L2 prefetches.
-// The grid is persistent (at most one CTA per SM) and splits the flattened
-// (unit, key-group) range evenly, so every SM streams the same byte count.
+// B200 design.  The step streams the key's id row (one byte per table) and
+// its fp32 norm from HBM and performs L random lookups into 2^P-entry tables.
+// The lookups go to shared memory, conflict-free for any ids, without
+// replicating the tables:
+//   * ids are stored key-major and rotated: slot s of block c (32 tables) of
+//     key n holds the id of table 32c + (s + n) mod 32;
+//   * a block's tables sit in a 64 KB region as float[bucket][64 columns],
+//     column j holding table 32c + j mod 32 (written in that form by the
+//     soft-table kernel and copied in with one bulk copy);
+//   * lane j of a warp scores key 32m + j and, in round r, reads column
+//     j + r of the row of its id for slot r -- table 32c + (j + r) mod 32, the
+//     table slot r holds for that key -- so the 32 lanes of every lookup hit
+//     32 distinct banks.
+// A region starts at a 64 KB-aligned shared address, so one byte-permute of
+// the packed id word (id into byte 1, lane column in byte 0) gives the row
+// address and the round's column is the load's immediate offset: a lookup is
+// one PRMT, one LDS and one FADD.  Each thread keeps KEYS keys in flight with
+// the next batch's id rows loading behind them and the batch after that
+// prefetched into L2.  The grid is persistent (one CTA per SM) and splits the
+// flattened (unit, 32-key chunk) range evenly; a CTA stages the tables of
+// each unit it touches (two units at once when a unit needs one region).
 #include "common.cuh"
 #include "internal.h"
+#include "socket_attn.h"
 
 namespace socket_attn {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kGroupsPerThread = 4;                      // 16-key groups per thread per pass
-constexpr int kPassGroups = kThreads * kGroupsPerThread;  // 2048 groups = 32768 keys
-constexpr uint32_t kBufBytes = 1u << 16;                 // [bucket 256][table 4][replica 16] floats
-constexpr int kTablesPerBuf = 4;
-constexpr int kStageSlots = kBufBytes / 16 / kThreads;   // float4 stores per thread per buffer (8)
-constexpr int kPrefetchAhead = 8;                        // tables prefetched into L2 ahead
-constexpr int kHistBins = kScoreHistBins;                // unit histogram of score bit patterns >> kHistShift
+constexpr int kWarps = kThreads / 32;
+constexpr uint32_t kRegionBytes = 1u << 16;  // [256 buckets][64 columns] floats
+constexpr int kRegions = 2;
+constexpr int kHistBins = kScoreHistBins;  // unit histogram of score bit patterns >> kHistShift
 constexpr int kHistShift = kScoreHistShift;
-// The two staging buffers sit at 64 KB-aligned shared addresses A and
-// A + 64 KB.  A lookup address is then A_buf | (id << 8) | (slot << 6) | (replica << 2):
-// one byte-permute of the packed id word with a per-lane base that already
-// holds A_buf, the table slot and the replica.  The dynamic allocation spans
-// three 64 KB windows so an aligned pair fits wherever the window starts.
-constexpr int kSmemBytes = 3 * (int)kBufBytes;
+// The regions sit at 64 KB-aligned shared addresses; the dynamic allocation
+// spans three 64 KB windows so two aligned regions fit wherever it starts.
+constexpr int kSmemBytes = 3 * (int)kRegionBytes;
+constexpr uint32_t kMaxPolls = 1u << 22;
 
 __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
@@ -55,198 +56,219 @@ __device__ __forceinline__ float lds_f32(uint32_t addr)
     return v;
 }
 
-// Ids of round rr for this lane's 4 groups: table (rr & ~3) + ((rr & 3) ^ half).
-// Groups past the pass read the pass's last group instead (their sums are
-// never stored), so the lookup loop needs no per-group condition.
-__device__ __forceinline__ void load_round(uint4 (&v)[kGroupsPerThread], const uint8_t* idu, int64_t Ncap, int L,
-                                           int npg, int tid, int half, int rr)
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i)
 {
-    const int tab = (rr & ~(kTablesPerBuf - 1)) + ((rr & (kTablesPerBuf - 1)) ^ half);
-    const uint8_t* row = idu + (int64_t)min(tab, L - 1) * Ncap;
-#pragma unroll
-    for (int j = 0; j < kGroupsPerThread; ++j) {
-        const int g = min(j * kThreads + tid, npg - 1);
-        v[j] = ldg_stream_u4(row + (int64_t)g * 16);
-    }
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-// One pass: groups [first_group, first_group + npg) of one unit, npg <= kPassGroups.
-__device__ __forceinline__ void score_pass(const float* __restrict__ tables, const uint8_t* __restrict__ ids,
-                                           const float* __restrict__ vnorm, float* __restrict__ scores,
-                                           uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
-                                           uint32_t* shist, char* smem, uint32_t buf0, int L,
-                                           int NB, int64_t Ncap, int64_t N, int64_t unit, int64_t first_group,
-                                           int npg, bool first_pass, uint32_t* red)
+__device__ __forceinline__ float ldg_stream_f32(const float* p)
 {
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int half = lane >> 4;
-    // byte 0 of a lookup address for slot s: (s << 6) | (replica << 2); slot = t ^ half.
-    const uint32_t rep4 = (uint32_t)(lane & 15) << 2;
-    const int nbuf = (L + kTablesPerBuf - 1) / kTablesPerBuf;
-    const float* tu = tables + unit * L * (int64_t)NB;
-    const uint8_t* idu = ids + unit * L * Ncap + first_group * 16;
-    const float* vu = vnorm + unit * Ncap + first_group * 16;
-    float* su = scores + unit * Ncap + first_group * 16;
-    const uint32_t pass_bytes = (uint32_t)npg * 16u;
-    char* bufp0 = smem + (buf0 - smem_addr(smem));
-
-    if (tid == 0) {
-        prefetch_l2_bulk(vu, pass_bytes * 4u);
-        for (int l = 0; l < min(L, kPrefetchAhead); ++l) prefetch_l2_bulk(idu + l * Ncap, pass_bytes);
-    }
-    uint4 cur[kGroupsPerThread];
-    load_round(cur, idu, Ncap, L, npg, tid, half, 0);
-    // The soft tables come from the previous kernel on the stream.
-    if (first_pass) pdl_wait();
-
-    // Stage values for buffer bi: float4 slot e = i*kThreads + tid holds
-    // bucket e >> 4, table slot (e >> 2) & 3, replicas 4*(e & 3) .. +3.
-    float stage[kStageSlots];
-    auto load_stage = [&](int bi) {
-#pragma unroll
-        for (int i = 0; i < kStageSlots; ++i) {
-            const int e = i * kThreads + tid;
-            const int bucket = e >> 4, l = kTablesPerBuf * bi + ((e >> 2) & 3);
-            stage[i] = (bucket < NB && l < L) ? __ldcg(tu + (int64_t)l * NB + bucket) : 0.0f;
-        }
-    };
-    auto store_stage = [&](int buf) {
-        float4* dst = reinterpret_cast<float4*>(bufp0 + buf * kBufBytes);
-#pragma unroll
-        for (int i = 0; i < kStageSlots; ++i) {
-            const int e = i * kThreads + tid;
-            if ((e >> 4) < NB) dst[e] = make_float4(stage[i], stage[i], stage[i], stage[i]);
-        }
-    };
-
-    __syncthreads();  // the previous pass finished reading both buffers
-    load_stage(0);
-    store_stage(0);
-    if (nbuf > 1) load_stage(1);
-    __syncthreads();
-
-    float acc[kGroupsPerThread][16];
-#pragma unroll
-    for (int j = 0; j < kGroupsPerThread; ++j)
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[j][e] = 0.0f;
-
-    const int nrounds = nbuf * kTablesPerBuf;
-    for (int bi = 0; bi < nbuf; ++bi) {
-        if (tid == 0) {
-            const int l0 = kTablesPerBuf * bi + kPrefetchAhead;
-            for (int l = l0; l < min(L, l0 + kTablesPerBuf); ++l) prefetch_l2_bulk(idu + l * Ncap, pass_bytes);
-        }
-        const uint32_t bbase = buf0 + (uint32_t)(bi & 1) * kBufBytes + rep4;
-#pragma unroll
-        for (int t = 0; t < kTablesPerBuf; ++t) {
-            const int rr = kTablesPerBuf * bi + t;
-            uint4 nxt[kGroupsPerThread];
-            if (rr + 1 < nrounds) load_round(nxt, idu, Ncap, L, npg, tid, half, rr + 1);
-            // Rounds past table L-1 look up the zero-filled slots of the last buffer.
-            const uint32_t base = bbase + ((uint32_t)(t ^ half) << 6);
-#pragma unroll
-            for (int j = 0; j < kGroupsPerThread; ++j) {
-                const uint32_t words[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-#pragma unroll
-                    for (int byte = 0; byte < 4; ++byte) {
-                        // bytes 0, 2, 3 from base; byte 1 = the id
-                        const uint32_t addr = __byte_perm(base, words[w], 0x3240u + (byte << 4));
-                        acc[j][w * 4 + byte] += lds_f32(addr);
-                    }
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kGroupsPerThread; ++j) cur[j] = nxt[j];
-        }
-        if (bi + 1 < nbuf) {
-            store_stage((bi + 1) & 1);
-            if (bi + 2 < nbuf) load_stage(bi + 2);
-        }
-        __syncthreads();
-    }
-
-    // Scores, the largest score of a live key (n < N) of the pass, and the
-    // histogram of the live scores' top bits (bit pattern >> kHistShift).
-    uint32_t mx = 0;
-    const int64_t key0 = first_group * 16;
-#pragma unroll
-    for (int j = 0; j < kGroupsPerThread; ++j) {
-        const int g = j * kThreads + tid;
-        if (g < npg) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float4 vn = ldg_stream_f4(vu + (int64_t)g * 16 + w * 4);
-                float4 sc;
-                sc.x = acc[j][w * 4 + 0] * vn.x;
-                sc.y = acc[j][w * 4 + 1] * vn.y;
-                sc.z = acc[j][w * 4 + 2] * vn.z;
-                sc.w = acc[j][w * 4 + 3] * vn.w;
-                *reinterpret_cast<float4*>(su + (int64_t)g * 16 + w * 4) = sc;
-                const int64_t n = key0 + (int64_t)g * 16 + w * 4;
-                const uint32_t bits[4] = {__float_as_uint(sc.x), __float_as_uint(sc.y), __float_as_uint(sc.z),
-                                          __float_as_uint(sc.w)};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if (n + e < N) {
-                        mx = max(mx, bits[e]);
-                        atomicAdd(shist + min(bits[e] >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
-                    }
-                }
-            }
-        }
-    }
-    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFullMask, mx, o));
-    if ((tid & 31) == 0) red[tid >> 5] = mx;
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t m = 0;
-        for (int w = 0; w < kThreads / 32; ++w) m = max(m, red[w]);
-        atomicMax(unit_max + unit, m);
-    }
-    // Flush the pass histogram into the unit's histogram and clear it.
-    uint32_t* gh = unit_hist + unit * kHistBins;
-    for (int b = tid; b < kHistBins; b += kThreads) {
-        const uint32_t c = shist[b];
-        if (c) {
-            atomicAdd(gh + b, c);
-            shist[b] = 0;
-        }
-    }
+    float v;
+    asm("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
 }
 
-// Persistent grid: CTA c owns groups [c * per_cta, (c+1) * per_cta) of the
-// flattened (unit, 16-key group) range.  The range is cut at unit boundaries
-// and each piece into equal passes of at most kPassGroups groups.
-__global__ __launch_bounds__(kThreads, 1) void score_kernel(
-    const float* __restrict__ tables, const uint8_t* __restrict__ ids, const float* __restrict__ vnorm,
-    float* __restrict__ scores, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist, int L, int NB,
-    int64_t Ncap, int64_t N, int64_t groups_per_unit, int64_t total_groups, int64_t groups_per_cta)
+struct ScoreArgs {
+    const float* tables;  // [U][nblk][NB][64] expanded soft tables
+    const uint8_t* ids;   // [U][Ncap][32 nblk] rotated id rows
+    const float* vnorm;   // [U][Ncap]
+    float* scores;        // [U][Ncap]
+    uint32_t* unit_max;
+    uint32_t* unit_hist;
+    uint32_t* err_word;
+    int nblk;             // 32-table blocks of L
+    int blk0;             // first block of this launch
+    int NB;
+    int first, last;      // first / last launch of the step (partial sums between)
+    int64_t Ncap, N;
+    int64_t chunks_per_unit, total_chunks, chunks_per_cta;
+};
+
+// NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: keys per thread
+// per batch; FIRST / LAST: whether this launch starts / finishes the sum
+// (launches in between pass partial sums through the score buffer).
+template <int NBLK, int KEYS, bool FIRST, bool LAST>
+__global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 {
+    constexpr int V = 2 * NBLK;              // 16-byte id words per key
+    constexpr int kSlots = kRegions / NBLK;  // units staged at once
     extern __shared__ __align__(1024) char smem[];
-    __shared__ uint32_t red[kThreads / 32];
     __shared__ uint32_t shist[kHistBins];
-    for (int b = threadIdx.x; b < kHistBins; b += kThreads) shist[b] = 0;
-    const uint32_t buf0 = (smem_addr(smem) + kBufBytes - 1) & ~(kBufBytes - 1);
-    int64_t g = (int64_t)blockIdx.x * groups_per_cta;
-    const int64_t g1 = min(total_groups, g + groups_per_cta);
-    bool first = true;
-    if (g >= g1) pdl_wait();
-    while (g < g1) {
-        const int64_t unit = g / groups_per_unit;
-        const int64_t seg_end = min(g1, (unit + 1) * groups_per_unit);
-        const int64_t seg = seg_end - g;
-        const int64_t npass = (seg + kPassGroups - 1) / kPassGroups;
-        for (int64_t ip = 0; ip < npass; ++ip) {
-            const int64_t a = g + seg * ip / npass, e = g + seg * (ip + 1) / npass;
-            score_pass(tables, ids, vnorm, scores, unit_max, unit_hist, shist, smem, buf0, L, NB, Ncap, N, unit,
-                       a - unit * groups_per_unit, (int)(e - a), first, red);
-            first = false;
-        }
-        g = seg_end;
+    __shared__ uint32_t red[kWarps];
+    __shared__ __align__(8) uint64_t bar[kSlots];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t region0 = (smem_addr(smem) + kRegionBytes - 1) & ~(kRegionBytes - 1);
+    char* region0_ptr = smem + (region0 - smem_addr(smem));
+
+    const int64_t c0 = (int64_t)blockIdx.x * a.chunks_per_cta;
+    const int64_t c1 = min64(a.total_chunks, c0 + a.chunks_per_cta);
+    if (c0 >= c1) return;
+    const int cpu = (int)a.chunks_per_unit;
+    const int64_t u_first = c0 / cpu;
+    const int nseg = (int)((c1 - 1) / cpu - u_first + 1);
+    const int Lr = 32 * a.nblk;  // id row bytes
+    const int N = (int)a.N;
+    const uint32_t region_bytes = (uint32_t)a.NB * 256u;
+
+    // Let the next kernel on the stream get its CTAs queued behind this grid.
+    pdl_launch_dependents();
+    if (LAST)
+        for (int b = tid; b < kHistBins; b += kThreads) shist[b] = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
+        fence_mbarrier_init();
     }
+    __syncthreads();
+
+    // Bulk copy of segment k's table blocks into its slot's regions.
+    auto issue_tables = [&](int k) {
+        const int s = k % kSlots;
+        const int64_t u = u_first + k;
+        mbar_arrive_expect_tx(&bar[s], NBLK * region_bytes);
+        for (int bl = 0; bl < NBLK; ++bl) {
+            const char* src = reinterpret_cast<const char*>(a.tables) +
+                              ((u * a.nblk + a.blk0 + bl) * (int64_t)region_bytes);
+            char* dst = region0_ptr + (s * NBLK + bl) * kRegionBytes;
+            for (uint32_t off = 0; off < region_bytes; off += 16384u)
+                bulk_copy_g2s(dst + off, src + off, min(16384u, region_bytes - off), &bar[s]);
+        }
+    };
+
+    uint32_t mx = 0;
+    for (int k = 0; k < nseg; ++k) {
+        const int64_t u = u_first + k;
+        const int cbeg = (int)(max64(c0, u * cpu) - u * cpu);
+        const int nch = (int)(min64(c1, (u + 1) * cpu) - u * cpu) - cbeg;
+        const int slot = k % kSlots;
+        // This warp's chunks: cbeg + warp + kWarps * m for m < cnt; batch b
+        // holds m = KEYS b .. KEYS b + KEYS - 1.
+        const int cnt = nch > warp ? (nch - warp + kWarps - 1) / kWarps : 0;
+        const int nbatch = (cnt + KEYS - 1) / KEYS;
+        const uint8_t* idu = a.ids + u * a.Ncap * Lr;
+        const float* vu = a.vnorm + u * a.Ncap;
+        float* su = a.scores + u * a.Ncap;
+        const int key0 = (cbeg + warp) * 32 + lane;  // this lane's key of m = 0
+        constexpr int kKeyStride = kWarps * 32;       // keys between m and m + 1
+
+        // Key of batch b, slot j; clamped to the warp's last chunk and to a
+        // live key so that loads stay inside the unit's rows.
+        auto key_at = [&](int b, int j) { return min(key0 + kKeyStride * min(b * KEYS + j, cnt - 1), N - 1); };
+        auto load = [&](uint4 (&v)[KEYS][V], float (&vn)[KEYS], int b) {
+#pragma unroll
+            for (int j = 0; j < KEYS; ++j) {
+                const int n = key_at(b, j);
+                const uint4* p = reinterpret_cast<const uint4*>(idu + (int64_t)n * Lr + 32 * a.blk0);
+#pragma unroll
+                for (int i = 0; i < V; ++i) v[j][i] = ldg_stream_u4(p + i);
+                vn[j] = LAST ? ldg_stream_f32(vu + n) : 0.0f;
+            }
+        };
+        // Score batch b from its id words, store, and count it.
+        auto score = [&](const uint4 (&v)[KEYS][V], const float (&vn)[KEYS], int b) {
+            if (lane < KEYS && (b + 2) * KEYS + lane < cnt) {
+                // L2 prefetch of the id rows two batches ahead.
+                const int c = cbeg + warp + kWarps * ((b + 2) * KEYS + lane);
+                const int rows = min(32, N - c * 32);
+                prefetch_l2_bulk(idu + (int64_t)c * 32 * Lr, (uint32_t)(rows * Lr));
+            }
+            float acc[KEYS];
+#pragma unroll
+            for (int j = 0; j < KEYS; ++j) acc[j] = FIRST ? 0.0f : __ldcg(su + key_at(b, j));
+#pragma unroll
+            for (int bl = 0; bl < NBLK; ++bl) {
+                const uint32_t base = region0 + (uint32_t)(slot * NBLK + bl) * kRegionBytes + ((uint32_t)lane << 2);
+#pragma unroll
+                for (int r = 0; r < 32; ++r) {
+                    const int q = bl * 32 + r;  // id byte within this launch's part of the row
+#pragma unroll
+                    for (int j = 0; j < KEYS; ++j) {
+                        // byte 1 <- the id (row), bytes 0, 2, 3 <- region and lane column
+                        const uint32_t row =
+                            __byte_perm(base, word_of(v[j][q >> 4], (q >> 2) & 3), 0x3240u | ((q & 3) << 4));
+                        acc[j] += lds_f32(row + 4u * r);
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < KEYS; ++j) {
+                const int m = b * KEYS + j;
+                const int n = key0 + kKeyStride * m;
+                if (m < cnt && n < N) {
+                    const float sc = LAST ? acc[j] * vn[j] : acc[j];
+                    su[n] = sc;
+                    if (LAST) {
+                        const uint32_t bits = __float_as_uint(sc);
+                        mx = max(mx, bits);
+                        atomicAdd(shist + min(bits >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
+                    }
+                }
+            }
+        };
+
+        uint4 ia[KEYS][V], ib[KEYS][V];
+        float va[KEYS], vb[KEYS];
+        if (nbatch > 0) load(ia, va, 0);
+        if (k == 0) {
+            // The soft tables (and, after the first launch, the partial sums)
+            // come from the previous kernel on the stream.
+            pdl_wait();
+            if (tid == 0)
+                for (int kk = 0; kk < min(kSlots, nseg); ++kk) issue_tables(kk);
+        }
+        if (!mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls)) {
+            if (tid == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
+            // Let the copies in flight land before the CTA exits.
+            mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
+            return;
+        }
+        // Two id buffers in turn: batch b + 1 loads while batch b is scored.
+        for (int b = 0; b < nbatch; b += 2) {
+            if (b + 1 < nbatch) load(ib, vb, b + 1);
+            score(ia, va, b);
+            if (b + 1 >= nbatch) break;
+            if (b + 2 < nbatch) load(ia, va, b + 2);
+            score(ib, vb, b + 1);
+        }
+
+        if (LAST) {
+            // The unit's largest live score and its score histogram.
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFullMask, mx, o));
+            if (lane == 0) red[warp] = mx;
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t m = 0;
+                for (int w = 0; w < kWarps; ++w) m = max(m, red[w]);
+                atomicMax(a.unit_max + u, m);
+            }
+            uint32_t* gh = a.unit_hist + u * kHistBins;
+            for (int bn = tid; bn < kHistBins; bn += kThreads) {
+                const uint32_t c = shist[bn];
+                if (c) {
+                    atomicAdd(gh + bn, c);
+                    shist[bn] = 0;
+                }
+            }
+            mx = 0;
+        }
+        if (k + kSlots < nseg) {
+            __syncthreads();  // every warp is done with this slot's regions
+            if (tid == 0) issue_tables(k + kSlots);
+        } else if (LAST) {
+            __syncthreads();  // histogram cleared before the next segment counts
+        }
+    }
+}
+
+template <int NBLK, int KEYS, bool FIRST, bool LAST>
+cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
+{
+    auto kern = score_kernel<NBLK, KEYS, FIRST, LAST>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, args);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -259,21 +281,47 @@ int device_num_sms()
     return n > 0 ? n : 1;
 }
 
+int ids_row_bytes(int L) { return 32 * ((L + 31) / 32); }
+
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, cudaStream_t stream)
+                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* err_word,
+                         cudaStream_t stream)
 {
-    const int64_t gpu = (s.N + 15) / 16;
-    const int64_t total = s.U * gpu;
-    // At least ~8192 keys per CTA so the table staging stays amortised.
-    const int64_t want = (total + 511) / 512;
+    ScoreArgs a;
+    a.tables = tables;
+    a.ids = ids;
+    a.vnorm = vnorm;
+    a.scores = scores;
+    a.unit_max = unit_max;
+    a.unit_hist = unit_hist;
+    a.err_word = err_word;
+    a.nblk = (s.L + 31) / 32;
+    a.NB = s.NB;
+    a.Ncap = s.Ncap;
+    a.N = s.N;
+    a.chunks_per_unit = (s.N + 31) / 32;
+    a.total_chunks = s.U * a.chunks_per_unit;
+    // At least one chunk per warp per CTA; at most one CTA per SM.
+    const int64_t want = (a.total_chunks + kWarps - 1) / kWarps;
     const int grid = (int)max64(1, min64(device_num_sms(), want));
-    const int64_t per_cta = (total + grid - 1) / grid;
-    cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(score_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, tables, ids, vnorm, scores,
-                   unit_max, unit_hist, s.L, s.NB, s.Ncap, s.N, gpu, total, per_cta);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    a.chunks_per_cta = (a.total_chunks + grid - 1) / grid;
+    // Blocks two at a time (two 64 KB regions); partial sums pass through
+    // the score buffer between launches when L > 64.
+    for (int b0 = 0; b0 < a.nblk; b0 += kRegions) {
+        const int nb = min(kRegions, a.nblk - b0);
+        a.blk0 = b0;
+        a.first = b0 == 0;
+        a.last = b0 + nb == a.nblk;
+        cudaError_t e;
+        if (nb == 1)
+            e = a.first ? launch_one<1, 4, true, true>(a, grid, stream) : launch_one<1, 4, false, true>(a, grid, stream);
+        else if (a.first)
+            e = a.last ? launch_one<2, 2, true, true>(a, grid, stream) : launch_one<2, 2, true, false>(a, grid, stream);
+        else
+            e = a.last ? launch_one<2, 2, false, true>(a, grid, stream) : launch_one<2, 2, false, false>(a, grid, stream);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace socket_attn

@@ -17,20 +17,25 @@
 namespace socket_attn {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTablesPerBlock = 8;
+constexpr int kThreads = 128;
+constexpr int kTablesPerBlock = 2;
 constexpr int kMaxGroup = 16;
 constexpr int kMaxP = 8;
+constexpr int kHalf = kHeadDim / 2;  // channels per thread of a dot product
 
 // Grid: (U, ceil(L / kTablesPerBlock)).  Block: kThreads.
-//   1. the unit's G query rows are widened to float64 and their norms taken;
-//   2. one thread per (head, table, plane) row forms z = <W_{l,p}, q_h>/||q_h||
-//      (all 16 loads of its hyperplane row in flight at once) and the two
-//      per-plane factors sigmoid(+-2z/tau);
+//   1. two threads per (head, table, plane) row load the two halves of the
+//      hyperplane row W_{l,p} (issued first, so they are in flight while the
+//      query is staged); the unit's G query rows are widened to float64 and
+//      their norms taken;
+//   2. each pair forms z = <W_{l,p}, q_h>/||q_h|| (its halves added with one
+//      shuffle) and the two per-plane factors sigmoid(+-2z/tau);
 //   3. the per-plane factors of planes 0-3 and 4-7 are multiplied into two
 //      16-entry nibble tables per (head, table);
-//   4. each entry T_l(b) = sum_h lo_h(b & 15) * hi_h(b >> 4), rounded once to
-//      float32.
+//   4. each entry T_l(b) = sum_h lo_h(b & 15) * hi_h(b >> 4) is rounded once
+//      to float32 and written in the expanded layout the scoring kernel
+//      copies into shared memory: per 32-table block c a [bucket][64] row
+//      whose column j holds table 32c + j mod 32 (tables past L are zero).
 template <typename QT>
 __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int64_t Hq, int64_t Hkv, int G, int L,
@@ -38,13 +43,10 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
     uint32_t* __restrict__ cand_cnt)
 {
-    // Dynamic shared memory, sized for the unit's G heads (see soft_tables_smem).
-    extern __shared__ __align__(16) double dsm[];
-    double (*qd)[kHeadDim] = reinterpret_cast<double (*)[kHeadDim]>(dsm);
-    double* qnorm = dsm + G * kHeadDim;
-    double (*sig)[kTablesPerBlock][kMaxP][2] =
-        reinterpret_cast<double (*)[kTablesPerBlock][kMaxP][2]>(qnorm + kMaxGroup);
-    double (*nib)[kTablesPerBlock][2][16] = reinterpret_cast<double (*)[kTablesPerBlock][2][16]>(sig + G);
+    __shared__ double qd[kMaxGroup][kHeadDim];
+    __shared__ double qnorm[kMaxGroup];
+    __shared__ double sig[kMaxGroup][kTablesPerBlock][kMaxP][2];
+    __shared__ double nib[kMaxGroup][kTablesPerBlock][2][16];
 
     const int64_t u = blockIdx.x;
     const int64_t b = u / Hkv, kvh = u % Hkv;
@@ -52,6 +54,19 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const int nt = min(kTablesPerBlock, L - l0);
     const int NB = 1 << P;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // Rows ordered (head, table, plane); thread pair (2r, 2r + 1) takes row r.
+    const int rows = G * nt * P;
+    const int half = tid & 1;
+    int r = tid >> 1;
+    uint4 wv[kHalf / 8];
+    auto load_w = [&](int row) {
+        const int lt = (row / P) % nt, p = row % P;
+        const uint4* w = reinterpret_cast<const uint4*>(W + ((int64_t)(l0 + lt) * P + p) * kHeadDim + half * kHalf);
+#pragma unroll
+        for (int c = 0; c < kHalf / 8; ++c) wv[c] = __ldg(w + c);
+    };
+    if (r < rows) load_w(r);
 
     if (blockIdx.y == 0) {
         if (tid == 0) {
@@ -80,51 +95,68 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     }
     __syncthreads();
 
-    // Rows ordered (head, table, plane) so neighbouring threads share q_h.
-    const int rows = G * nt * P;
-    for (int r = tid; r < rows; r += kThreads) {
-        const int h = r / (nt * P), lt = (r / P) % nt, p = r % P;
-        const uint4* w = reinterpret_cast<const uint4*>(W + ((int64_t)(l0 + lt) * P + p) * kHeadDim);
-        uint4 wv[kHeadDim / 8];
-#pragma unroll
-        for (int c = 0; c < kHeadDim / 8; ++c) wv[c] = __ldg(w + c);
+    // Every pair runs the same number of rounds so the shuffle sees both halves.
+    for (; r < (rows + kThreads / 2 - 1) / (kThreads / 2) * (kThreads / 2); r += kThreads / 2) {
+        const bool live = r < rows;
+        const int h = live ? r / (nt * P) : 0;
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        if (live) {
+            const double* qh = qd[h] + half * kHalf;
 #pragma unroll
-        for (int c = 0; c < kHeadDim / 8; ++c) {
-            const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+            for (int c = 0; c < kHalf / 8; ++c) {
+                const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = bf16x2_to_f32x2(words[i]);
-                acc[i] = fma((double)f.x, qd[h][c * 8 + 2 * i], acc[i]);
-                acc[i] = fma((double)f.y, qd[h][c * 8 + 2 * i + 1], acc[i]);
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = bf16x2_to_f32x2(words[i]);
+                    acc[i] = fma((double)f.x, qh[c * 8 + 2 * i], acc[i]);
+                    acc[i] = fma((double)f.y, qh[c * 8 + 2 * i + 1], acc[i]);
+                }
             }
         }
-        const double y = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        const double z = qnorm[h] > 0.0 ? y / qnorm[h] : 0.0;
-        const double x = 2.0 * z / tau;
-        sig[h][lt][p][1] = 1.0 / (1.0 + exp(-x));  // sign +1: bit set
-        sig[h][lt][p][0] = 1.0 / (1.0 + exp(x));   // sign -1: bit clear
+        double y = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        y += __shfl_xor_sync(kFullMask, y, 1);
+        if (live && half == 0) {
+            const int lt = (r / P) % nt, p = r % P;
+            const double z = qnorm[h] > 0.0 ? y / qnorm[h] : 0.0;
+            const double x = 2.0 * z / tau;
+            sig[h][lt][p][1] = 1.0 / (1.0 + exp(-x));  // sign +1: bit set
+            sig[h][lt][p][0] = 1.0 / (1.0 + exp(x));   // sign -1: bit clear
+        }
+        if (r + kThreads / 2 < rows) load_w(r + kThreads / 2);
     }
     __syncthreads();
 
     // Nibble tables: lo over planes 0..min(P,4)-1, hi over planes 4..P-1.
     const int plo = min(P, 4);
     for (int e = tid; e < G * nt * 32; e += kThreads) {
-        const int h = e / (nt * 32), lt = (e / 32) % nt, half = (e / 16) & 1, v = e & 15;
+        const int h = e / (nt * 32), lt = (e / 32) % nt, hi = (e / 16) & 1, v = e & 15;
         double prod = 1.0;
-        const int p0 = half ? 4 : 0, p1 = half ? P : plo;
+        const int p0 = hi ? 4 : 0, p1 = hi ? P : plo;
         for (int p = p0; p < p1; ++p) prod *= sig[h][lt][p][(v >> (p - p0)) & 1];
-        nib[h][lt][half][v] = prod;
+        nib[h][lt][hi][v] = prod;
     }
     __syncthreads();
 
-    float* tu = tables + (u * L + l0) * (int64_t)NB;
+    const int nblk = (L + 31) / 32;
+    float* tu = tables + u * nblk * (int64_t)NB * 64;
     for (int e = tid; e < nt * NB; e += kThreads) {
-        const int lt = e / NB, bucket = e % NB;
+        const int lt = e % nt, bucket = e / nt;
         double acc = 0.0;
         for (int h = 0; h < G; ++h)
             acc += nib[h][lt][0][bucket & 15] * nib[h][lt][1][bucket >> 4];
-        tu[e] = (float)acc;
+        const int l = l0 + lt;
+        float* row = tu + ((int64_t)(l >> 5) * NB + bucket) * 64;
+        row[l & 31] = (float)acc;
+        row[(l & 31) + 32] = (float)acc;
+    }
+    if (blockIdx.y == 0) {
+        const int npad = 32 * nblk - L;
+        for (int e = tid; e < npad * NB; e += kThreads) {
+            const int l = L + e % npad, bucket = e / npad;
+            float* row = tu + ((int64_t)(l >> 5) * NB + bucket) * 64;
+            row[l & 31] = 0.0f;
+            row[(l & 31) + 32] = 0.0f;
+        }
     }
 }
 
@@ -135,18 +167,12 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream)
 {
     dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
-    const size_t smem = sizeof(double) * ((size_t)s.G * kHeadDim + kMaxGroup + (size_t)s.G * kTablesPerBlock * kMaxP * 2 +
-                                          (size_t)s.G * kTablesPerBlock * 32);
-    cudaError_t e = cudaFuncSetAttribute(q_dtype == 1 ? (const void*)soft_tables_kernel<uint16_t>
-                                                      : (const void*)soft_tables_kernel<float>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     if (q_dtype == 1)
-        soft_tables_kernel<uint16_t><<<grid, kThreads, smem, stream>>>(
+        soft_tables_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(
             static_cast<const uint16_t*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
             unit_max, unit_hist, cand_cnt);
     else
-        soft_tables_kernel<float><<<grid, kThreads, smem, stream>>>(
+        soft_tables_kernel<float><<<grid, kThreads, 0, stream>>>(
             static_cast<const float*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
             unit_max, unit_hist, cand_cnt);
     return cudaGetLastError();

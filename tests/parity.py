@@ -30,6 +30,31 @@ SET_BAND = 1e-6
 OUT_ATOL = 2e-3
 
 
+def row_slots(L, ncap):
+    """Slot of table l in key n's id row, [L, ncap]: 32 (l // 32) + (l - n) mod 32
+    (the rotated key-major layout documented for socket_hash_keys)."""
+    l = np.arange(L)[:, None]
+    n = np.arange(ncap)[None, :]
+    return 32 * (l // 32) + (l % 32 - n) % 32
+
+
+def ids_to_rows(tab_ids, L):
+    """Table-major ids [..., L, ncap] -> rotated rows [..., ncap, Lr] (padding 0)."""
+    ncap = tab_ids.shape[-1]
+    Lr = 32 * ((L + 31) // 32)
+    rows = np.zeros(tab_ids.shape[:-2] + (ncap, Lr), dtype=np.uint8)
+    n = np.broadcast_to(np.arange(ncap)[None, :], (L, ncap))
+    rows[..., n, row_slots(L, ncap)] = tab_ids
+    return rows
+
+
+def rows_to_ids(rows, L):
+    """Rotated rows [..., ncap, Lr] -> table-major ids [..., L, ncap]."""
+    ncap = rows.shape[-2]
+    n = np.broadcast_to(np.arange(ncap)[None, :], (L, ncap))
+    return rows[..., n, row_slots(L, ncap)]
+
+
 def gpu_hash(inp, w, n_begin=0, n_end=None):
     dev = inp["K"].device
     ids, vnorm = sk.alloc_cache_index(inp["K"].shape[0], w.Hkv, w.ncap, w.L, dev)
@@ -71,8 +96,15 @@ def oracle_hash_units(inp, w, units, n_begin=0, n_end=None):
     return ids, vn, mg
 
 
-def check_hash(gpu_ids, gpu_vn, orc_ids, orc_vn, margin, n_begin, n_end):
-    """gpu_*: numpy for the same units as the oracle arrays."""
+def check_hash(gpu_rows, gpu_vn, orc_ids, orc_vn, margin, n_begin, n_end):
+    """gpu_rows [U, ncap, Lr], gpu_vn [U, ncap]: numpy for the same units as the
+    oracle arrays.  Slots of tables >= L must hold 0."""
+    L = orc_ids.shape[1]
+    ncap = gpu_rows.shape[1]
+    used = np.zeros(gpu_rows.shape[1:], dtype=bool)
+    used[np.broadcast_to(np.arange(ncap)[None, :], (L, ncap)), row_slots(L, ncap)] = True
+    assert not np.any(gpu_rows[:, n_begin:n_end][:, ~used[n_begin:n_end]]), "padding slots not zero"
+    gpu_ids = rows_to_ids(gpu_rows, L)
     g = gpu_ids[..., n_begin:n_end]
     o = orc_ids[..., n_begin:n_end]
     exempt = margin[:, n_begin:n_end] < ID_MARGIN                    # [U, n]
@@ -127,5 +159,5 @@ def substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32):
     """Copy the oracle's ids / norms of `units` into the device index tensors."""
     for i, u in enumerate(units):
         b, h = divmod(u, w.Hkv)
-        ids[b, h].copy_(torch.from_numpy(orc_ids[i]))
+        ids[b, h].copy_(torch.from_numpy(ids_to_rows(orc_ids[i], w.L)))
         vnorm[b, h].copy_(torch.from_numpy(orc_vn32[i]))

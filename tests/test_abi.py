@@ -6,6 +6,8 @@ import glob
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from soft_lsh_top_b200 import _build
@@ -44,7 +46,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version(lib):
-    assert lib.socket_version() == 100
+    assert lib.socket_version() == 200
 
 
 # Fake, aligned, never-dereferenced device addresses: every call below fails
@@ -141,3 +143,39 @@ def test_python_binding_checks_shapes_before_the_library():
         s.socket_hash_keys(torch.zeros(1, 1, 16, 128), torch.zeros(1, 1, 16, 128),
                            torch.zeros(4, 8, 128, dtype=torch.bfloat16),
                            torch.zeros(1, 1, 4, 16, dtype=torch.uint8), torch.zeros(1, 1, 16))
+
+
+def test_ids_row_bytes(lib):
+    f = lib.socket_ids_row_bytes
+    assert [f(L) for L in (1, 12, 32, 33, 60, 64, 65, 128)] == [32, 32, 32, 64, 64, 64, 96, 128]
+    assert f(0) == 0 and f(129) == 0 and f(-3) == 0
+
+
+@pytest.mark.parametrize("L", [1, 7, 32, 33, 60, 128])
+def test_rotated_id_rows(L):
+    """The documented id-row layout: a bijection between tables and used slots,
+    and, in every slot, the 32 keys 32m .. 32m + 31 name 32 different tables,
+    the one periodic column lane + r of the expanded soft table holds."""
+    from parity import ids_to_rows, row_slots, rows_to_ids
+    ncap = 96
+    slot = row_slots(L, ncap)                                       # [L, ncap]
+    for n in range(ncap):
+        assert len(set(slot[:, n])) == L
+    Lr = 32 * ((L + 31) // 32)
+    table_of = np.full((ncap, Lr), -1)
+    for l in range(L):
+        table_of[np.arange(ncap), slot[l]] = l
+    for s in range(Lr):
+        c, r = divmod(s, 32)
+        for m in range(ncap // 32):
+            keys = np.arange(32 * m, 32 * m + 32)
+            t = table_of[keys, s]
+            lane = keys % 32
+            want = 32 * c + (lane + r) % 32                         # column lane + r of block c
+            live = want < L
+            assert np.array_equal(t[live], want[live]) and np.all(t[~live] == -1)
+    rng = np.random.default_rng(5)
+    ids = rng.integers(0, 256, size=(3, L, ncap), dtype=np.uint8)
+    rows = ids_to_rows(ids, L)
+    assert rows.shape == (3, ncap, Lr)
+    assert np.array_equal(rows_to_ids(rows, L), ids)
