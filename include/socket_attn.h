@@ -79,14 +79,18 @@ extern "C" {
  *   K, V      device, [B][Hkv][Ncap][d] of kv_dtype, 16-byte aligned.
  *   W         device, [L][P][d] bfloat16 bits (one set of hyperplanes shared
  *             by every batch row and head), 16-byte aligned.
- *   ids       device out, [B][Hkv][Ncap][Lr] uint8, Lr = socket_ids_row_bytes(L)
- *             = 32 * ceil(L / 32), 16-byte aligned: one row of Lr bytes per
- *             key, in blocks of 32 slots.  Slot s of block c of key n holds the
- *             id of table 32c + (s + n) mod 32 when that table is < L, else 0.
- *             (The rotation by n lets the 32 lanes of a warp, scoring keys
- *             32m .. 32m + 31, read 32 different tables in every lookup.)
+ *   ids       device out, [B][Hkv][Ncap/32][Lr/16][32][16] uint8,
+ *             Lr = socket_ids_row_bytes(L) = 32 * ceil(L / 32), 16-byte aligned.
+ *             Every key has an id row of Lr bytes, in blocks of 32 slots: slot
+ *             s of block c of key n holds the id of table 32c + (s + n) mod 32
+ *             when that table is < L, else 0.  Keys are grouped in chunks of 32
+ *             and a chunk stores its rows piece-major: the 16-byte piece p of
+ *             the row of key 32m + j sits at [m][p][j].  (The rotation lets
+ *             the 32 lanes of a warp, scoring keys 32m .. 32m + 31, read 32
+ *             different tables in every lookup; the chunking makes each
+ *             lane's 16-byte load part of one contiguous 512-byte warp load.)
  *   vnorm     device out, [B][Hkv][Ncap] float32, 16-byte aligned.
- * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Ncap % 16 == 0;
+ * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Ncap % 32 == 0;
  * 0 <= n_begin <= n_end <= Ncap.  n_begin == n_end queues nothing.
  * Bucket ids are exact except where some |<W_{l,p}, k>| is within float32
  * accumulation error of 0 (below ~1e-6 * ||k|| for d = 128).
@@ -142,7 +146,7 @@ size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t 
  *              if given, the scores of step 2 land here (entries n >= N are
  *              unspecified).
  * Preconditions: d == 128; 1 <= P <= 8; 1 <= L <= 128; Hq % Hkv == 0;
- * 1 <= Hq / Hkv <= 16; Ncap % 16 == 0; 1 <= k <= N <= Ncap; N < 2^31.
+ * 1 <= Hq / Hkv <= 16; Ncap % 32 == 0; 1 <= k <= N <= Ncap; N < 2^31.
  * Inputs must be finite; non-finite values give an unspecified selection.
  */
 int socket_decode(const void* q, int q_dtype, const uint16_t* W,

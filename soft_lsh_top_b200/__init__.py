@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
-    "socket_last_error", "socket_version", "socket_ids_row_bytes", "socket_set_step_events", "library_path", "load_library",
+    "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
 
@@ -135,7 +135,7 @@ def socket_hash_keys(K: torch.Tensor, V: torch.Tensor, W: torch.Tensor, ids: tor
     """Hash keys [n_begin, n_end) of every unit into ``ids`` and ``vnorm``.
 
     K, V: [B, Hkv, Ncap, 128] (float32 or bfloat16); W: [L, P, 128] bfloat16;
-    ids: [B, Hkv, Ncap, socket_ids_row_bytes(L)] uint8 (rotated rows, see the header); vnorm: [B, Hkv, Ncap] float32.
+    ids: [B, Hkv, Ncap/32, Lr/16, 32, 16] uint8, Lr = socket_ids_row_bytes(L) (see the header); vnorm: [B, Hkv, Ncap] float32.
     """
     lib = load_library()
     B, Hkv, Ncap, d = K.shape
@@ -144,7 +144,7 @@ def socket_hash_keys(K: torch.Tensor, V: torch.Tensor, W: torch.Tensor, ids: tor
     _check(K, "K", (B, Hkv, Ncap, d), device=dev)
     _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
     _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
-    _check(ids, "ids", (B, Hkv, Ncap, socket_ids_row_bytes(L)), dtype=torch.uint8, device=dev)
+    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
     _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
     n_end = Ncap if n_end is None else int(n_end)
     with torch.cuda.device(dev):
@@ -160,6 +160,11 @@ def socket_ids_row_bytes(L: int) -> int:
     return n
 
 
+def ids_shape(B: int, Hkv: int, Ncap: int, L: int) -> tuple:
+    """Shape of the bucket-id array: [B, Hkv, Ncap/32, Lr/16, 32, 16]."""
+    return (B, Hkv, Ncap // 32, socket_ids_row_bytes(L) // 16, 32, 16)
+
+
 def socket_decode_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, d: int, L: int, P: int, k: int) -> int:
     n = int(load_library().socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k))
     if n == 0:
@@ -173,7 +178,7 @@ def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: to
                   scores_out: torch.Tensor | None = None, stream=None) -> None:
     """One decode step (soft assignment, scoring, top-k, sparse attention).
 
-    q: [B, Hq, 128]; W: [L, P, 128] bfloat16; ids: [B, Hkv, Ncap, socket_ids_row_bytes(L)] uint8 (rotated rows, see the header);
+    q: [B, Hq, 128]; W: [L, P, 128] bfloat16; ids: [B, Hkv, Ncap/32, Lr/16, 32, 16] uint8, Lr = socket_ids_row_bytes(L) (see the header);
     vnorm: [B, Hkv, Ncap] float32; K, V: [B, Hkv, Ncap, 128];
     workspace: uint8 tensor of >= socket_decode_workspace_size() bytes;
     idx_out: [B, Hkv, k] int32; out: [B, Hq, 128] float32;
@@ -186,7 +191,7 @@ def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: to
     dev = q.device
     _check(q, "q", (B, Hq, d), device=dev)
     _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
-    _check(ids, "ids", (B, Hkv, Ncap, socket_ids_row_bytes(L)), dtype=torch.uint8, device=dev)
+    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
     _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
     _check(K, "K", (B, Hkv, Ncap, d), device=dev)
     _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
@@ -220,7 +225,7 @@ def socket_decode_static(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vn
     dev = q.device
     _check(q, "q", (B, Hq, d), device=dev)
     _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
-    _check(ids, "ids", (B, Hkv, Ncap, socket_ids_row_bytes(L)), dtype=torch.uint8, device=dev)
+    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
     _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
     _check(K, "K", (B, Hkv, Ncap, d), device=dev)
     _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
@@ -252,7 +257,7 @@ def socket_set_step_events(events) -> None:
 
 def alloc_cache_index(B: int, Hkv: int, Ncap: int, L: int, device) -> tuple[torch.Tensor, torch.Tensor]:
     """Bucket-id and value-norm buffers for a cache of Ncap keys per unit."""
-    ids = torch.empty(B, Hkv, Ncap, socket_ids_row_bytes(L), dtype=torch.uint8, device=device)
+    ids = torch.empty(ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=device)
     vnorm = torch.empty(B, Hkv, Ncap, dtype=torch.float32, device=device)
     return ids, vnorm
 

@@ -56,7 +56,7 @@ int check_common(int64_t B, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P)
     if (L < 1 || L > SOCKET_MAX_L) return fail(SOCKET_EUNSUPPORTED, "L=%d outside [1, 128]", L);
     if (B < 1 || Hkv < 1) return fail(SOCKET_EINVAL, "B=%lld and Hkv=%lld must be >= 1", (long long)B, (long long)Hkv);
     if (B * Hkv > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hkv=%lld above 65535", (long long)(B * Hkv));
-    if (Ncap < 16 || Ncap % 16 != 0) return fail(SOCKET_EINVAL, "Ncap=%lld must be a positive multiple of 16", (long long)Ncap);
+    if (Ncap < 32 || Ncap % 32 != 0) return fail(SOCKET_EINVAL, "Ncap=%lld must be a positive multiple of 32", (long long)Ncap);
     if (Ncap >= (int64_t(1) << 31)) return fail(SOCKET_EUNSUPPORTED, "Ncap=%lld must be < 2^31", (long long)Ncap);
     return SOCKET_OK;
 }

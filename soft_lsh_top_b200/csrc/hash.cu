@@ -104,9 +104,16 @@ __global__ __launch_bounds__(kThreads) void hash_kernel(const KT* __restrict__ K
         }
     }
     __syncthreads();
-    // Keys n0 .. n0 + nk - 1 are consecutive rows of the unit's id array.
-    uint4* dst = reinterpret_cast<uint4*>(ids + (u * Ncap + n0) * Lr);
-    for (int e = tid; e < nk * Lr / 16; e += kThreads) dst[e] = reinterpret_cast<const uint4*>(idrow)[e];
+    // Chunked layout: piece p (16 bytes) of key n = 32m + j sits at [m][p][j];
+    // neighbouring threads write neighbouring keys' pieces.
+    const int pieces = Lr / 16;
+    uint8_t* idu = ids + u * Ncap * Lr;
+    for (int e = tid; e < nk * pieces; e += kThreads) {
+        const int p = e / nk, k = e % nk;
+        const int64_t nn = n0 + k;
+        *reinterpret_cast<uint4*>(idu + ((nn >> 5) * pieces + p) * 512 + (nn & 31) * 16) =
+            *reinterpret_cast<const uint4*>(idrow + k * Lr + 16 * p);
+    }
 }
 
 }  // namespace

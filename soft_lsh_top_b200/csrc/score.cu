@@ -14,8 +14,10 @@
 // its fp32 norm from HBM and performs L random lookups into 2^P-entry tables.
 // The lookups go to shared memory, conflict-free for any ids, without
 // replicating the tables:
-//   * ids are stored key-major and rotated: slot s of block c (32 tables) of
-//     key n holds the id of table 32c + (s + n) mod 32;
+//   * every key has an id row rotated by the key: slot s of block c (32
+//     tables) of key n holds the id of table 32c + (s + n) mod 32; rows are
+//     stored in chunks of 32 keys, piece-major, so the 32 lanes' 16-byte loads
+//     of one piece form one contiguous 512-byte warp load;
 //   * a block's tables sit in a 64 KB region as float[bucket][64 columns],
 //     column j holding table 32c + j mod 32 (written in that form by the
 //     soft-table kernel and copied in with one bulk copy);
@@ -27,10 +29,10 @@
 // the packed id word (id into byte 1, lane column in byte 0) gives the row
 // address and the round's column is the load's immediate offset: a lookup is
 // one PRMT, one LDS and one FADD.  Each thread keeps KEYS keys in flight with
-// the next batch's id rows loading behind them and the batch after that
-// prefetched into L2.  The grid is persistent (one CTA per SM) and splits the
-// flattened (unit, 32-key chunk) range evenly; a CTA stages the tables of
-// each unit it touches (two units at once when a unit needs one region).
+// the next batch's id pieces loading behind them.  The grid is persistent
+// (one CTA per SM) and splits the flattened (unit, 32-key chunk) range
+// evenly; a CTA stages the tables of each unit it touches (two units at once
+// when a unit needs one region).
 #include "common.cuh"
 #include "internal.h"
 #include "socket_attn.h"
@@ -158,20 +160,15 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 #pragma unroll
             for (int j = 0; j < KEYS; ++j) {
                 const int n = key_at(b, j);
-                const uint4* p = reinterpret_cast<const uint4*>(idu + (int64_t)n * Lr + 32 * a.blk0);
+                // piece 2 blk0 + i of key n: chunk n / 32, lane n % 32
+                const uint8_t* p = idu + (int64_t)(n >> 5) * 32 * Lr + (2 * a.blk0) * 512 + (n & 31) * 16;
 #pragma unroll
-                for (int i = 0; i < V; ++i) v[j][i] = ldg_stream_u4(p + i);
+                for (int i = 0; i < V; ++i) v[j][i] = ldg_stream_u4(p + 512 * i);
                 vn[j] = LAST ? ldg_stream_f32(vu + n) : 0.0f;
             }
         };
         // Score batch b from its id words, store, and count it.
         auto score = [&](const uint4 (&v)[KEYS][V], const float (&vn)[KEYS], int b) {
-            if (lane < KEYS && (b + 2) * KEYS + lane < cnt) {
-                // L2 prefetch of the id rows two batches ahead.
-                const int c = cbeg + warp + kWarps * ((b + 2) * KEYS + lane);
-                const int rows = min(32, N - c * 32);
-                prefetch_l2_bulk(idu + (int64_t)c * 32 * Lr, (uint32_t)(rows * Lr));
-            }
             float acc[KEYS];
 #pragma unroll
             for (int j = 0; j < KEYS; ++j) acc[j] = FIRST ? 0.0f : __ldcg(su + key_at(b, j));

@@ -32,27 +32,44 @@ OUT_ATOL = 2e-3
 
 def row_slots(L, ncap):
     """Slot of table l in key n's id row, [L, ncap]: 32 (l // 32) + (l - n) mod 32
-    (the rotated key-major layout documented for socket_hash_keys)."""
+    (the rotation documented for socket_hash_keys)."""
     l = np.arange(L)[:, None]
     n = np.arange(ncap)[None, :]
     return 32 * (l // 32) + (l % 32 - n) % 32
 
 
+def _chunked_index(L, ncap):
+    """For table l and key n, the flat byte offset of its id inside a unit's
+    chunked array [ncap/32][Lr/16][32][16]: chunk n // 32, piece s // 16,
+    lane n % 32, byte s % 16 with s = row_slots(L, ncap)."""
+    Lr = 32 * ((L + 31) // 32)
+    s = row_slots(L, ncap)
+    n = np.arange(ncap)[None, :]
+    return (((n // 32) * (Lr // 16) + s // 16) * 32 + n % 32) * 16 + s % 16
+
+
 def ids_to_rows(tab_ids, L):
-    """Table-major ids [..., L, ncap] -> rotated rows [..., ncap, Lr] (padding 0)."""
+    """Table-major ids [..., L, ncap] -> chunked rows [..., ncap/32, Lr/16, 32, 16] (padding 0)."""
     ncap = tab_ids.shape[-1]
     Lr = 32 * ((L + 31) // 32)
-    rows = np.zeros(tab_ids.shape[:-2] + (ncap, Lr), dtype=np.uint8)
-    n = np.broadcast_to(np.arange(ncap)[None, :], (L, ncap))
-    rows[..., n, row_slots(L, ncap)] = tab_ids
-    return rows
+    flat = np.zeros(tab_ids.shape[:-2] + (ncap * Lr,), dtype=np.uint8)
+    flat[..., _chunked_index(L, ncap)] = tab_ids
+    return flat.reshape(tab_ids.shape[:-2] + (ncap // 32, Lr // 16, 32, 16))
 
 
 def rows_to_ids(rows, L):
-    """Rotated rows [..., ncap, Lr] -> table-major ids [..., L, ncap]."""
-    ncap = rows.shape[-2]
-    n = np.broadcast_to(np.arange(ncap)[None, :], (L, ncap))
-    return rows[..., n, row_slots(L, ncap)]
+    """Chunked rows [..., ncap/32, Lr/16, 32, 16] -> table-major ids [..., L, ncap]."""
+    ncap = rows.shape[-4] * 32
+    flat = rows.reshape(rows.shape[:-4] + (-1,))
+    return flat[..., _chunked_index(L, ncap)]
+
+
+def padding_bytes(L, ncap):
+    """Mask [ncap * Lr] of the chunked array's bytes that hold no table's id."""
+    Lr = 32 * ((L + 31) // 32)
+    used = np.zeros(ncap * Lr, dtype=bool)
+    used[_chunked_index(L, ncap)] = True
+    return ~used
 
 
 def gpu_hash(inp, w, n_begin=0, n_end=None):
@@ -97,13 +114,17 @@ def oracle_hash_units(inp, w, units, n_begin=0, n_end=None):
 
 
 def check_hash(gpu_rows, gpu_vn, orc_ids, orc_vn, margin, n_begin, n_end):
-    """gpu_rows [U, ncap, Lr], gpu_vn [U, ncap]: numpy for the same units as the
-    oracle arrays.  Slots of tables >= L must hold 0."""
+    """gpu_rows [U, ncap/32, Lr/16, 32, 16], gpu_vn [U, ncap]: numpy for the same
+    units as the oracle arrays.  Bytes of tables >= L must hold 0 for the
+    hashed keys."""
     L = orc_ids.shape[1]
-    ncap = gpu_rows.shape[1]
-    used = np.zeros(gpu_rows.shape[1:], dtype=bool)
-    used[np.broadcast_to(np.arange(ncap)[None, :], (L, ncap)), row_slots(L, ncap)] = True
-    assert not np.any(gpu_rows[:, n_begin:n_end][:, ~used[n_begin:n_end]]), "padding slots not zero"
+    ncap = gpu_rows.shape[1] * 32
+    Lr = gpu_rows.shape[2] * 16
+    pad = padding_bytes(L, ncap).reshape(ncap // 32, Lr // 16, 32, 16)
+    keys = np.zeros((ncap // 32, 1, 32, 1), dtype=bool)
+    keys.reshape(-1)[n_begin:n_end] = True
+    flat = gpu_rows.reshape(gpu_rows.shape[0], -1)
+    assert not np.any(flat[:, (pad & keys).reshape(-1)]), "padding slots not zero"
     gpu_ids = rows_to_ids(gpu_rows, L)
     g = gpu_ids[..., n_begin:n_end]
     o = orc_ids[..., n_begin:n_end]

@@ -76,6 +76,7 @@ def decode(lib, **kw):
     (dict(k=65), EINVAL),
     (dict(N=80), EINVAL),
     (dict(Ncap=70, N=64), EINVAL),
+    (dict(Ncap=48, N=48), EINVAL),
     (dict(tau=0.0), EINVAL),
     (dict(tau=-1.0), EINVAL),
     (dict(tau=float("nan")), EINVAL),
@@ -110,6 +111,7 @@ def hash_call(lib, **kw):
     (dict(n_end=65), EINVAL),
     (dict(n_begin=-1), EINVAL),
     (dict(Ncap=60, n_end=60), EINVAL),
+    (dict(Ncap=48, n_end=48), EINVAL),
     (dict(kv_dtype=3), EINVAL),
     (dict(vnorm=P16 + 4), EINVAL),
     (dict(W=None), EINVAL),
@@ -143,6 +145,10 @@ def test_python_binding_checks_shapes_before_the_library():
         s.socket_hash_keys(torch.zeros(1, 1, 16, 128), torch.zeros(1, 1, 16, 128),
                            torch.zeros(4, 8, 128, dtype=torch.bfloat16),
                            torch.zeros(1, 1, 4, 16, dtype=torch.uint8), torch.zeros(1, 1, 16))
+    with pytest.raises((ValueError, TypeError)):   # ids in the unchunked [.., Ncap, Lr] shape
+        s.socket_hash_keys(torch.zeros(1, 1, 32, 128), torch.zeros(1, 1, 32, 128),
+                           torch.zeros(4, 8, 128, dtype=torch.bfloat16),
+                           torch.zeros(1, 1, 32, 32, dtype=torch.uint8), torch.zeros(1, 1, 32))
 
 
 def test_ids_row_bytes(lib):
@@ -153,10 +159,11 @@ def test_ids_row_bytes(lib):
 
 @pytest.mark.parametrize("L", [1, 7, 32, 33, 60, 128])
 def test_rotated_id_rows(L):
-    """The documented id-row layout: a bijection between tables and used slots,
-    and, in every slot, the 32 keys 32m .. 32m + 31 name 32 different tables,
-    the one periodic column lane + r of the expanded soft table holds."""
-    from parity import ids_to_rows, row_slots, rows_to_ids
+    """The documented id layout: a bijection between tables and used bytes;
+    in every slot the 32 keys 32m .. 32m + 31 name 32 different tables, the one
+    periodic column lane + r of the expanded soft table holds; and piece p of
+    the chunk's 32 keys is one contiguous 512-byte run."""
+    from parity import ids_to_rows, padding_bytes, row_slots, rows_to_ids
     ncap = 96
     slot = row_slots(L, ncap)                                       # [L, ncap]
     for n in range(ncap):
@@ -175,7 +182,13 @@ def test_rotated_id_rows(L):
             live = want < L
             assert np.array_equal(t[live], want[live]) and np.all(t[~live] == -1)
     rng = np.random.default_rng(5)
-    ids = rng.integers(0, 256, size=(3, L, ncap), dtype=np.uint8)
+    ids = rng.integers(1, 256, size=(3, L, ncap), dtype=np.uint8)
     rows = ids_to_rows(ids, L)
-    assert rows.shape == (3, ncap, Lr)
+    assert rows.shape == (3, ncap // 32, Lr // 16, 32, 16)
     assert np.array_equal(rows_to_ids(rows, L), ids)
+    # key n's row, read back piece by piece, is table_of's row
+    for n in (0, 5, 31, 32, 95):
+        row = rows[0, n // 32, :, n % 32, :].reshape(-1)
+        for s in range(Lr):
+            assert row[s] == (ids[0, table_of[n, s], n] if table_of[n, s] >= 0 else 0)
+    assert padding_bytes(L, ncap).sum() == ncap * (Lr - L)

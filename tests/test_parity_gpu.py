@@ -48,7 +48,7 @@ def test_hash_matches_oracle(small):
     w, inp, units, orc_ids, orc_vn, margin = small
     ids, vnorm = gpu_hash(inp, w)
     torch.cuda.synchronize()
-    g_ids = ids.reshape(w.U, w.ncap, -1).cpu().numpy()
+    g_ids = ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy()
     g_vn = vnorm.reshape(w.U, w.ncap).cpu().numpy()
     check_hash(g_ids, g_vn, orc_ids, orc_vn, margin, 0, w.N)
 
@@ -56,7 +56,8 @@ def test_hash_matches_oracle(small):
 def _decode_on_oracle_index(small, **kw):
     w, inp, units, orc_ids, orc_vn, _ = small
     orc_vn32 = orc_vn.astype(np.float32)
-    ids = torch.from_numpy(ids_to_rows(orc_ids, w.L)).reshape(inp["K"].shape[0], w.Hkv, w.ncap, -1).to(DEV)
+    ids = torch.from_numpy(ids_to_rows(orc_ids, w.L)).reshape(inp["K"].shape[0], w.Hkv, w.ncap // 32, -1, 32,
+                                                               16).to(DEV)
     vn = torch.from_numpy(orc_vn32).reshape(inp["K"].shape[0], w.Hkv, w.ncap).to(DEV)
     idx, out, sc = gpu_decode(inp, w, ids, vn, **kw)
     return check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, **kw)

@@ -61,8 +61,8 @@ class Workload:
 
     @property
     def ncap(self) -> int:
-        """Cache capacity per unit: live keys plus appends, rounded up to 16."""
-        return round_up(self.N + self.appends, 16)
+        """Cache capacity per unit: live keys plus appends, rounded up to 32."""
+        return round_up(self.N + self.appends, 32)
 
     @property
     def torch_dtype(self):
