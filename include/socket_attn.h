@@ -64,7 +64,7 @@ extern "C" {
  */
 #define SOCKET_WS_ERROR_OFFSET 0
 #define SOCKET_DEVERR_GATHER_TIMEOUT 0x1u  /* attention: a key/value row gather */
-#define SOCKET_DEVERR_TABLE_TIMEOUT  0x2u  /* scoring: a soft-table copy into shared memory */
+#define SOCKET_DEVERR_TABLE_TIMEOUT  0x2u  /* scoring: a copy into shared memory (soft tables, ids) */
 
 /*
  * socket_hash_keys -- prefill hashing ([ES] step 1 "Pre-cálculo (Prellenado)";

@@ -46,9 +46,9 @@ constexpr uint32_t kRegionBytes = 1u << 16;  // [256 buckets][64 columns] floats
 constexpr int kRegions = 2;
 constexpr int kHistBins = kScoreHistBins;  // unit histogram of score bit patterns >> kHistShift
 constexpr int kHistShift = kScoreHistShift;
-// The regions sit at 64 KB-aligned shared addresses; the dynamic allocation
-// spans three 64 KB windows so two aligned regions fit wherever it starts.
-constexpr int kSmemBytes = 3 * (int)kRegionBytes;
+// The regions sit at 64 KB-aligned shared addresses inside the dynamic
+// allocation; the histogram and the copy rings use the space around them.
+constexpr int kSmemBytes = 226 * 1024;
 constexpr uint32_t kMaxPolls = 1u << 22;
 
 __device__ __forceinline__ float lds_f32(uint32_t addr)
@@ -56,6 +56,18 @@ __device__ __forceinline__ float lds_f32(uint32_t addr)
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
+}
+
+__device__ __forceinline__ uint4 lds_u4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i)
@@ -86,22 +98,53 @@ struct ScoreArgs {
     int64_t chunks_per_unit, total_chunks, chunks_per_cta;
 };
 
-// NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: keys per thread
-// per batch; FIRST / LAST: whether this launch starts / finishes the sum
-// (launches in between pass partial sums through the score buffer).
-template <int NBLK, int KEYS, bool FIRST, bool LAST>
+// NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: 32-key chunks
+// per warp per batch; NS: batches in a warp's copy ring; FIRST / LAST:
+// whether this launch starts / finishes the sum (launches in between pass
+// partial sums through the score buffer).
+template <int NBLK, int KEYS, int NS, bool FIRST, bool LAST>
 __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 {
-    constexpr int V = 2 * NBLK;              // 16-byte id words per key
-    constexpr int kSlots = kRegions / NBLK;  // units staged at once
+    constexpr int V = 2 * NBLK;                            // 16-byte id pieces per key
+    constexpr int kSlots = kRegions / NBLK;                // units staged at once
+    constexpr uint32_t kChunkIds = 1024u * NBLK;           // id bytes of a chunk in this launch
+    constexpr uint32_t kChunkBytes = kChunkIds + (LAST ? 128u : 0u);  // + the chunk's norms
+    constexpr uint32_t kStageBytes = KEYS * kChunkBytes;
+    constexpr uint32_t kRingBytes = NS * kStageBytes;
+    constexpr uint32_t kHistBytes = LAST ? kHistBins * 4u : 0u;
     extern __shared__ __align__(1024) char smem[];
-    __shared__ uint32_t shist[kHistBins];
     __shared__ uint32_t red[kWarps];
     __shared__ __align__(8) uint64_t bar[kSlots];
+    __shared__ __align__(8) uint64_t ring_bar[kWarps][NS];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint32_t region0 = (smem_addr(smem) + kRegionBytes - 1) & ~(kRegionBytes - 1);
-    char* region0_ptr = smem + (region0 - smem_addr(smem));
+    const uint32_t sbase = smem_addr(smem);
+    const uint32_t region0 = (sbase + kRegionBytes - 1) & ~(kRegionBytes - 1);
+    char* region0_ptr = smem + (region0 - sbase);
+
+    // The histogram and the warps' copy rings fill the space below the two
+    // table regions, then the space above them.
+    uint32_t lo = sbase, hi = region0 + kRegions * kRegionBytes;
+    const uint32_t lo_end = region0, hi_end = sbase + kSmemBytes;
+    auto place = [&](uint32_t bytes) -> uint32_t {
+        if (lo + bytes <= lo_end) { lo += bytes; return lo - bytes; }
+        if (hi + bytes <= hi_end) { hi += bytes; return hi - bytes; }
+        return 0u;
+    };
+    const uint32_t hist_s = LAST ? place(kHistBytes) : sbase;
+    uint32_t ring_s = 0;
+    bool fits = hist_s != 0u;
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t r = place(kRingBytes);
+        fits = fits && r != 0u;
+        if (w == warp) ring_s = r;
+    }
+    if (!fits) {  // cannot happen with the sizes launched; reported, not trapped
+        if (tid == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
+        return;
+    }
+    uint32_t* shist = reinterpret_cast<uint32_t*>(smem + (hist_s - sbase));
+    char* ring = smem + (ring_s - sbase);
 
     const int64_t c0 = (int64_t)blockIdx.x * a.chunks_per_cta;
     const int64_t c1 = min64(a.total_chunks, c0 + a.chunks_per_cta);
@@ -119,6 +162,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         for (int b = tid; b < kHistBins; b += kThreads) shist[b] = 0;
     if (tid == 0) {
         for (int s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
+        for (int w = 0; w < kWarps; ++w)
+            for (int s = 0; s < NS; ++s) mbar_init(&ring_bar[w][s], 1);
         fence_mbarrier_init();
     }
     __syncthreads();
@@ -138,6 +183,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     };
 
     uint32_t mx = 0;
+    uint32_t seq = 0;      // batches this warp has taken from its ring so far
+    bool failed = false;   // a bounded wait of this warp expired
     for (int k = 0; k < nseg; ++k) {
         const int64_t u = u_first + k;
         const int cbeg = (int)(max64(c0, u * cpu) - u * cpu);
@@ -153,25 +200,70 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         const int key0 = (cbeg + warp) * 32 + lane;  // this lane's key of m = 0
         constexpr int kKeyStride = kWarps * 32;       // keys between m and m + 1
 
-        // Key of batch b, slot j; clamped to the warp's last chunk and to a
-        // live key so that loads stay inside the unit's rows.
-        auto key_at = [&](int b, int j) { return min(key0 + kKeyStride * min(b * KEYS + j, cnt - 1), N - 1); };
-        auto load = [&](uint4 (&v)[KEYS][V], float (&vn)[KEYS], int b) {
+        // Lane 0: copy batch b's chunks (this launch's id pieces and, in the
+        // last launch, the norms) into ring stage (seq + b) % NS.  Chunks past
+        // the warp's last repeat it; the unit's last chunk may run past N
+        // (rows below Ncap, never scored).
+        auto issue = [&](int b) {
+            const uint32_t st = (seq + b) % NS;
+            char* dst = ring + st * kStageBytes;
+            mbar_arrive_expect_tx(&ring_bar[warp][st], kStageBytes);
 #pragma unroll
             for (int j = 0; j < KEYS; ++j) {
-                const int n = key_at(b, j);
-                // piece 2 blk0 + i of key n: chunk n / 32, lane n % 32
-                const uint8_t* p = idu + (int64_t)(n >> 5) * 32 * Lr + (2 * a.blk0) * 512 + (n & 31) * 16;
-#pragma unroll
-                for (int i = 0; i < V; ++i) v[j][i] = ldg_stream_u4(p + 512 * i);
-                vn[j] = LAST ? ldg_stream_f32(vu + n) : 0.0f;
+                const int c = cbeg + warp + kWarps * min(b * KEYS + j, cnt - 1);
+                bulk_copy_g2s(dst + j * kChunkBytes, idu + (int64_t)c * 32 * Lr + (2 * a.blk0) * 512, kChunkIds,
+                              &ring_bar[warp][st]);
+                if (LAST) bulk_copy_g2s(dst + j * kChunkBytes + kChunkIds, vu + (int64_t)c * 32, 128u, &ring_bar[warp][st]);
             }
         };
-        // Score batch b from its id words, store, and count it.
-        auto score = [&](const uint4 (&v)[KEYS][V], const float (&vn)[KEYS], int b) {
+        __syncwarp();
+        if (lane == 0 && !failed) {
+            if (k > 0) fence_proxy_async_shared();  // the stages were read in the previous segment
+            for (int b = 0; b < min(NS, nbatch); ++b) issue(b);
+        }
+        if (k == 0) {
+            // The soft tables (and, after the first launch, the partial sums)
+            // come from the previous kernel on the stream.
+            pdl_wait();
+            if (tid == 0)
+                for (int kk = 0; kk < min(kSlots, nseg); ++kk) issue_tables(kk);
+        }
+        // Waits give up after a bounded number of polls; a warp gives up as a
+        // whole so it never splits around __syncwarp.
+        const bool tables_ok = mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
+        if (__any_sync(kFullMask, !tables_ok)) {
+            if (lane == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
+            mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
+            failed = true;
+        }
+
+        int b = 0;
+        for (; b < nbatch && !failed; ++b) {
+            const uint32_t st = (seq + b) % NS;
+            const bool ids_ok = mbar_wait_bounded(&ring_bar[warp][st], ((seq + b) / NS) & 1u, kMaxPolls);
+            if (__any_sync(kFullMask, !ids_ok)) {
+                if (lane == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
+                failed = true;
+                break;
+            }
+            const uint32_t sa = ring_s + st * kStageBytes;
+            uint4 v[KEYS][V];
+            float vn[KEYS];
+#pragma unroll
+            for (int j = 0; j < KEYS; ++j) {
+#pragma unroll
+                for (int i = 0; i < V; ++i) v[j][i] = lds_u4(sa + j * kChunkBytes + i * 512 + lane * 16);
+                vn[j] = LAST ? lds_f32(sa + j * kChunkBytes + kChunkIds + lane * 4) : 0.0f;
+            }
+            __syncwarp();
+            if (lane == 0 && b + NS < nbatch) {
+                fence_proxy_async_shared();  // the reads above precede the next copy into this stage
+                issue(b + NS);
+            }
             float acc[KEYS];
 #pragma unroll
-            for (int j = 0; j < KEYS; ++j) acc[j] = FIRST ? 0.0f : __ldcg(su + key_at(b, j));
+            for (int j = 0; j < KEYS; ++j)
+                acc[j] = FIRST ? 0.0f : __ldcg(su + min(key0 + kKeyStride * min(b * KEYS + j, cnt - 1), N - 1));
 #pragma unroll
             for (int bl = 0; bl < NBLK; ++bl) {
                 const uint32_t base = region0 + (uint32_t)(slot * NBLK + bl) * kRegionBytes + ((uint32_t)lane << 2);
@@ -201,32 +293,13 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                     }
                 }
             }
-        };
-
-        uint4 ia[KEYS][V], ib[KEYS][V];
-        float va[KEYS], vb[KEYS];
-        if (nbatch > 0) load(ia, va, 0);
-        if (k == 0) {
-            // The soft tables (and, after the first launch, the partial sums)
-            // come from the previous kernel on the stream.
-            pdl_wait();
-            if (tid == 0)
-                for (int kk = 0; kk < min(kSlots, nseg); ++kk) issue_tables(kk);
         }
-        if (!mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls)) {
-            if (tid == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
-            // Let the copies in flight land before the CTA exits.
-            mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
-            return;
+        if (failed) {
+            // Let this warp's copies in flight land before anything moves on.
+            for (int bb = b; bb < min(nbatch, b + NS); ++bb)
+                mbar_wait_bounded(&ring_bar[warp][(seq + bb) % NS], ((seq + bb) / NS) & 1u, kMaxPolls);
         }
-        // Two id buffers in turn: batch b + 1 loads while batch b is scored.
-        for (int b = 0; b < nbatch; b += 2) {
-            if (b + 1 < nbatch) load(ib, vb, b + 1);
-            score(ia, va, b);
-            if (b + 1 >= nbatch) break;
-            if (b + 2 < nbatch) load(ia, va, b + 2);
-            score(ib, vb, b + 1);
-        }
+        seq += nbatch;
 
         if (LAST) {
             // The unit's largest live score and its score histogram.
@@ -257,10 +330,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     }
 }
 
-template <int NBLK, int KEYS, bool FIRST, bool LAST>
+template <int NBLK, int KEYS, int NS, bool FIRST, bool LAST>
 cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
 {
-    auto kern = score_kernel<NBLK, KEYS, FIRST, LAST>;
+    auto kern = score_kernel<NBLK, KEYS, NS, FIRST, LAST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, args);
@@ -311,11 +384,14 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
         a.last = b0 + nb == a.nblk;
         cudaError_t e;
         if (nb == 1)
-            e = a.first ? launch_one<1, 4, true, true>(a, grid, stream) : launch_one<1, 4, false, true>(a, grid, stream);
+            e = a.first ? launch_one<1, 2, 2, true, true>(a, grid, stream)
+                        : launch_one<1, 2, 2, false, true>(a, grid, stream);
         else if (a.first)
-            e = a.last ? launch_one<2, 2, true, true>(a, grid, stream) : launch_one<2, 2, true, false>(a, grid, stream);
+            e = a.last ? launch_one<2, 1, 2, true, true>(a, grid, stream)
+                       : launch_one<2, 1, 2, true, false>(a, grid, stream);
         else
-            e = a.last ? launch_one<2, 2, false, true>(a, grid, stream) : launch_one<2, 2, false, false>(a, grid, stream);
+            e = a.last ? launch_one<2, 1, 2, false, true>(a, grid, stream)
+                       : launch_one<2, 1, 2, false, false>(a, grid, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
