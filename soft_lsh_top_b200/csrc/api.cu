@@ -184,7 +184,7 @@ size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t 
         g_last_error = saved;
         return 0;
     }
-    s.nsplit = (k + attention_chunk_rows(SOCKET_F32) - 1) / attention_chunk_rows(SOCKET_F32);
+    s.nsplit = (k + 15) / 16;  // attention splits never exceed ceil(k / 16)
     return decode_workspace_layout(s).total;
 }
 
@@ -206,8 +206,8 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
         !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
         return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
     if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
-    // Splits are at most ceil(k / chunk rows); the advertised size covers the smallest chunk.
-    s.nsplit = attention_splits(kv_dtype, s.U, k, device_num_sms());
+    // Splits never exceed ceil(k / 16), the count the advertised size covers.
+    s.nsplit = attention_splits(kv_dtype, q_dtype, s.G, s.U, k, device_num_sms());
     const size_t need = socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k);
     if (workspace_bytes < need)
         return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);

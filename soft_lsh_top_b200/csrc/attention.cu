@@ -58,12 +58,14 @@ __device__ __forceinline__ float load1(const float* row, int j) { return row[j];
 // out = sum_s w_s o_s / sum_s w_s l_s.  Weights are staged in shared memory,
 // kThreads splits at a time, and the partial rows are read with many loads in
 // flight.  Thread j handles column j.
-template <int G>
+template <int G, int NT>
 __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
                                            const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                            uint32_t* __restrict__ counters, float* __restrict__ out,
                                            float (*red)[G], float* wsm, uint32_t& s_last)
 {
+    static_assert(kHeadDim % NT == 0 && NT % 32 == 0, "NT threads cover the head dimension evenly");
+    constexpr int kCols = kHeadDim / NT;  // output columns per thread: tid, tid + NT, ...
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __threadfence();
     __syncthreads();
@@ -72,12 +74,12 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
     if (!s_last) return;
     __threadfence();
     // Per head: M = max_s m_s; w_s = exp(m_s - M); out = sum_s w_s o_s / sum_s w_s l_s,
-    // accumulated in split order.  Weights are staged in shared memory, kThreads
+    // accumulated in split order.  Weights are staged in shared memory, NT
     // splits at a time, and the partial rows are read with many loads in flight.
     for (int h = 0; h < G; ++h) {
         const int64_t base = pbase + h * nsplit;
         float m = -INFINITY;
-        for (int sp = tid; sp < nsplit; sp += kThreads) m = fmaxf(m, __ldcg(&part_ml[base + sp]).x);
+        for (int sp = tid; sp < nsplit; sp += NT) m = fmaxf(m, __ldcg(&part_ml[base + sp]).x);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, o));
         __syncthreads();
@@ -85,10 +87,12 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
         __syncthreads();
         float M = red[0][0];
 #pragma unroll
-        for (int w = 1; w < kThreads / 32; ++w) M = fmaxf(M, red[w][0]);
-        float lsum = 0.0f, acc = 0.0f;
-        for (int s0 = 0; s0 < nsplit; s0 += kThreads) {
-            const int cnt = min(kThreads, nsplit - s0);
+        for (int w = 1; w < NT / 32; ++w) M = fmaxf(M, red[w][0]);
+        float lsum = 0.0f, acc[kCols];
+#pragma unroll
+        for (int j = 0; j < kCols; ++j) acc[j] = 0.0f;
+        for (int s0 = 0; s0 < nsplit; s0 += NT) {
+            const int cnt = min(NT, nsplit - s0);
             __syncthreads();
             if (tid < cnt) {
                 const float2 t = __ldcg(&part_ml[base + s0 + tid]);
@@ -97,16 +101,19 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
                 lsum += t.y * w;
             }
             __syncthreads();
-            const float* po = part_o + (base + s0) * kHeadDim + tid;
-            int i = 0;
-            for (; i + 16 <= cnt; i += 16) {
-                float v[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) v[r] = __ldcg(po + (int64_t)(i + r) * kHeadDim);
+            for (int j = 0; j < kCols; ++j) {
+                const float* po = part_o + (base + s0) * kHeadDim + tid + j * NT;
+                int i = 0;
+                for (; i + 16 <= cnt; i += 16) {
+                    float v[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) acc += v[r] * wsm[i + r];
+                    for (int r = 0; r < 16; ++r) v[r] = __ldcg(po + (int64_t)(i + r) * kHeadDim);
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) acc[j] += v[r] * wsm[i + r];
+                }
+                for (; i < cnt; ++i) acc[j] += __ldcg(po + (int64_t)i * kHeadDim) * wsm[i];
             }
-            for (; i < cnt; ++i) acc += __ldcg(po + (int64_t)i * kHeadDim) * wsm[i];
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, o);
@@ -115,8 +122,9 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
         __syncthreads();
         float L = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kThreads / 32; ++w) L += red[w][0];
-        out[(qrow0 + h) * kHeadDim + tid] = acc / L;
+        for (int w = 0; w < NT / 32; ++w) L += red[w][0];
+#pragma unroll
+        for (int j = 0; j < kCols; ++j) out[(qrow0 + h) * kHeadDim + tid + j * NT] = acc[j] / L;
     }
     if (tid == 0) counters[u] = 0u;
 }
@@ -313,27 +321,41 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     for (int h = 0; h < G; ++h) part_o[((pbase + h * nsplit) + split) * kHeadDim + tid] = o[h];
     if (tid < G) part_ml[pbase + tid * nsplit + split] = make_float2(m_run[tid], l_run[tid]);
 
-    merge_unit<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
+    merge_unit<G, kThreads>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
 }
 
 // ---------------------------------------------------------------------------
-// bfloat16 K/V and q, G <= 8: the same chunked online softmax with both
-// contractions on the tensor cores (warp-level mma.sync m16n8k16, bf16 in,
-// fp32 accumulate):
-//   logits^T [64 rows x 8 heads] = K_chunk [64 x 128] * q^T [128 x 8]
-//     (warp w: rows 16w..16w+15; A from ldmatrix, B = q held in registers),
-//   out^T   [128 x 8 heads]      += V_chunk^T [128 x 64] * P^T [64 x 8]
-//     (warp w: columns 32w..32w+31; A from ldmatrix.trans of the value rows,
-//      B = the weights, split into a bfloat16 high part and a bfloat16
-//      remainder so the weights keep ~16 bits).
-// bf16 x bf16 products are exact in fp32, so the logits carry only fp32
-// accumulation error, as on the CUDA cores.  Key/value rows are padded to
-// 272 bytes in shared memory so the 8 rows an ldmatrix phase reads fall in
-// distinct banks.  Heads G..7 of the n = 8 tile are zero padding.
+// bfloat16 K/V and q, G <= 8: flash-decode split-K with every warp on its own
+// 16-key chunks and both contractions on the tensor cores (warp-level
+// mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//   logits^T [16 heads x 16 keys] = q [16 x 128] * K_chunk^T [128 x 16]
+//     (A = q held in registers, heads G..15 zero; B from ldmatrix of the key
+//      rows, which are B's columns);
+//   out^T   [128 x 16 heads]     += V_chunk^T [128 x 16] * P^T [16 x 8]
+//     (A from ldmatrix.trans of the value rows; B = the weights).
+// The logits' accumulator fragment (head lane/4, keys 2 (lane%4) + {0,1}
+// and + 8) is exactly the B fragment the second product needs, so weights
+// never leave registers; the online softmax of a head reduces over one lane
+// quad.  Weights enter the second product as a bfloat16 high part plus a
+// bfloat16 remainder (~16 bits).  bf16 x bf16 products are exact in fp32, so
+// the logits carry only fp32 accumulation error.
+// Each warp gathers its chunks itself (one bulk copy per 256-byte key or
+// value row, into rows padded to 272 bytes so an ldmatrix phase's 8 rows hit
+// distinct banks) on its own two-stage ring of mbarriers: the chunk loop has
+// no CTA-wide barrier.  The two warps of a CTA then merge in shared memory
+// and the last CTA of the unit merges the CTAs' partials.
 // ---------------------------------------------------------------------------
-constexpr int kMmaChunk = 64;
-constexpr int kMmaRowStride = 272;
-constexpr int kMmaStageBytes = 2 * kMmaChunk * kMmaRowStride;
+constexpr int kWChunk = 16;                                // keys per warp chunk
+constexpr int kWStages = 2;
+constexpr int kWRowStride = 272;
+constexpr int kWStageBytes = 2 * kWChunk * kWRowStride;   // keys + values
+constexpr int kWWarps = 2;
+constexpr int kWThreads = 32 * kWWarps;
+constexpr int kWSmemBytes = kWWarps * kWStages * kWStageBytes;
+constexpr int kWCtasPerSm = 6;
+
+// The tensor-core kernel takes bfloat16 q, K, V and groups of up to 8 heads.
+bool warp_path(int kv_dtype, int q_dtype, int G) { return kv_dtype == 1 && q_dtype == 1 && G <= 8; }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
 {
@@ -364,22 +386,19 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 __device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(pack_bf16(x, 0.0f) << 16); }
 
 template <int G>
-__global__ __launch_bounds__(kThreads) void attention_mma_kernel(
+__global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
     const int32_t* __restrict__ idx, int64_t Hq, int64_t Hkv, int64_t Ncap, int k, int nsplit, int rpc,
     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
     uint32_t* __restrict__ err_word, float* __restrict__ out)
 {
-    static_assert(G <= 8, "the n = 8 tile holds up to 8 heads");
+    static_assert(G <= 8, "heads are the M rows 0..7 of the 16-row tile");
     extern __shared__ __align__(128) char smem[];
-    // Logits, then weights; rows padded to 72 floats so the weight fragments
-    // (8 heads x 4 row pairs per warp) read from 32 distinct banks.
-    __shared__ __align__(8) float S[G][kMmaChunk + 8];
-    __shared__ float red[kThreads / 32][G];
-    __shared__ float m_run[G], l_run[G], m_new[G], scale[G];
-    __shared__ __align__(8) uint64_t bar[2];
+    __shared__ __align__(8) uint64_t bar[kWWarps][kWStages];
+    __shared__ float xm[kWWarps][8], xl[kWWarps][8];
+    __shared__ float red[kWWarps][G];
+    __shared__ float wsm[kWThreads];
     __shared__ uint32_t s_last;
-    __shared__ float wsm[kThreads];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t u = blockIdx.x / nsplit;
@@ -387,225 +406,206 @@ __global__ __launch_bounds__(kThreads) void attention_mma_kernel(
     const int64_t b = u / Hkv, kvh = u % Hkv;
     const int r_begin = split * rpc;
     const int r_end = min(k, r_begin + rpc);
-    const int nchunks = (r_end - r_begin + kMmaChunk - 1) / kMmaChunk;
+    const int nch = (r_end - r_begin + kWChunk - 1) / kWChunk;        // chunks of this CTA
+    const int cw = nch > warp ? (nch - warp + kWWarps - 1) / kWWarps : 0;  // chunks of this warp
     const int64_t qrow0 = b * Hq + kvh * G;
-    const uint32_t sbase = smem_addr(smem);
+    char* wsm_base = smem + warp * kWStages * kWStageBytes;
+    const uint32_t wbase = smem_addr(wsm_base);
 
-    // q^T fragments: b0/b1 of k-step ks = q[head lane/4][16 ks + 2 (lane%4) + {0, 1} (+8)].
-    uint32_t qb[8][2];
+    // q as the A operand: row h = lane/4 (< G), channels 16 kk + 2 (lane%4) + {0,1} and + 8.
+    uint32_t qa[8][2];
     {
         const int h = lane >> 2, c = (lane & 3) * 2;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int kk = 0; kk < 8; ++kk) {
             uint32_t v0 = 0, v1 = 0;
             if (h < G) {
-                const uint16_t* qh = q + (qrow0 + h) * kHeadDim + ks * 16 + c;
+                const uint16_t* qh = q + (qrow0 + h) * kHeadDim + kk * 16 + c;
                 v0 = (uint32_t)qh[0] | ((uint32_t)qh[1] << 16);
                 v1 = (uint32_t)qh[8] | ((uint32_t)qh[9] << 16);
             }
-            qb[ks][0] = v0;
-            qb[ks][1] = v1;
+            qa[kk][0] = v0;
+            qa[kk][1] = v1;
         }
     }
-    if (tid < G) {
-        m_run[tid] = -INFINITY;
-        l_run[tid] = 0.0f;
-    }
     if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int w = 0; w < kWWarps; ++w)
+            for (int st = 0; st < kWStages; ++st) mbar_init(&bar[w][st], 1);
         fence_mbarrier_init();
     }
     __syncthreads();
     pdl_wait();  // the selected indices come from the previous kernel on the stream
 
-    // Gather chunk c into stage st: thread i < rows copies one key row and one
-    // value row; value rows past the chunk's end are zeroed (their weights are 0).
-    auto issue = [&](int c, int st) {
-        const int r0 = r_begin + c * kMmaChunk;
-        const int nr = min(kMmaChunk, r_end - r0);
-        char* ks = smem + st * kMmaStageBytes;
-        char* vs = ks + kMmaChunk * kMmaRowStride;
-        if (tid < nr) {
+    // Gather this warp's chunk j into stage st: lane i < 16 copies key row i,
+    // lane 16 + i value row i; value rows past the chunk's end are zeroed
+    // (their weights are 0, and 0 * NaN from stale bytes must not happen).
+    auto issue = [&](int j, int st) {
+        const int r0 = r_begin + (warp + kWWarps * j) * kWChunk;
+        const int nr = min(kWChunk, r_end - r0);
+        const int i = lane & 15;
+        char* dst = wsm_base + st * kWStageBytes + (lane >> 4) * kWChunk * kWRowStride + i * kWRowStride;
+        if (i < nr) {
             // Indices come from the top-k kernel and are < N; clamp anyway so a
             // gather can never leave the unit's cache rows.
-            int32_t r = __ldcg(idx + u * k + r0 + tid);
+            int32_t r = __ldcg(idx + u * k + r0 + i);
             r = (r >= 0 && r < Ncap) ? r : 0;
-            const int64_t row = u * Ncap + r;
-            bulk_copy_g2s(ks + tid * kMmaRowStride, K + row * kHeadDim, kHeadDim * 2, &bar[st]);
-            bulk_copy_g2s(vs + tid * kMmaRowStride, V + row * kHeadDim, kHeadDim * 2, &bar[st]);
-        } else if (tid < kMmaChunk) {
-            uint4* z = reinterpret_cast<uint4*>(vs + tid * kMmaRowStride);
+            const uint16_t* src = (lane < 16 ? K : V) + (u * Ncap + r) * kHeadDim;
+            bulk_copy_g2s(dst, src, kHeadDim * 2, &bar[warp][st]);
+        } else if (lane >= 16) {
+            uint4* z = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-            for (int i = 0; i < kHeadDim * 2 / 16; ++i) z[i] = make_uint4(0, 0, 0, 0);
+            for (int e = 0; e < kHeadDim * 2 / 16; ++e) z[e] = make_uint4(0, 0, 0, 0);
         }
-        if (tid == 0) mbar_arrive_expect_tx(&bar[st], (uint32_t)nr * 2u * kHeadDim * 2u);
+        if (lane == 0) mbar_arrive_expect_tx(&bar[warp][st], (uint32_t)nr * 2u * kHeadDim * 2u);
     };
-    issue(0, 0);
-    if (nchunks > 1) issue(1, 1);
-    __syncthreads();  // zeroed value rows visible
+    if (cw > 0) issue(0, 0);
+    if (cw > 1) issue(1, 1);
+    __syncwarp();  // zeroed value rows visible to the warp
 
-    // out^T accumulators: warp w, m-tiles mt = 2w, 2w+1 (columns 16 mt ..), c[mt][i]:
-    // i = 0,1: column 16 mt + lane/4, heads 2 (lane%4) + {0,1}; i = 2,3: column + 8.
-    float acc[2][4];
+    // out^T accumulators: m-tile mt = channels 16 mt ..; [0], [1]: channel
+    // 16 mt + lane/4, heads 2 (lane%4) + {0,1}; [2], [3]: channel + 8.
+    float acc[8][4];
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[t][i] = 0.0f;
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        const int nrows = min(kMmaChunk, r_end - (r_begin + c * kMmaChunk));
-        const uint32_t ks_addr = sbase + st * kMmaStageBytes;
-        const uint32_t vs_addr = ks_addr + kMmaChunk * kMmaRowStride;
-        if (!mbar_wait_bounded(&bar[st], (uint32_t)((c >> 1) & 1), kMaxPolls)) {
-            if (tid == 0) atomicOr(err_word, SOCKET_DEVERR_GATHER_TIMEOUT);
-            mbar_wait_bounded(&bar[st], (uint32_t)((c >> 1) & 1), kMaxPolls);
-            if (c + 1 < nchunks) mbar_wait_bounded(&bar[st ^ 1], (uint32_t)(((c + 1) >> 1) & 1), kMaxPolls);
-            return;
+        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
+    float m_run = -INFINITY, l_run = 0.0f;  // of head lane/4
+    const int q4 = lane >> 3;
+    // ldmatrix lane address: key row (q4 >> 1) * 8 + lane % 8, channel half q4 & 1
+    const uint32_t lrow = (uint32_t)(((q4 >> 1) * 8 + (lane & 7)) * kWRowStride + (q4 & 1) * 16);
+    const int t2 = (lane & 3) * 2;
+    bool ok = true;
+    for (int j = 0; j < cw; ++j) {
+        const int st = j & 1;
+        const bool got = mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), kMaxPolls);
+        if (__any_sync(kFullMask, !got)) {
+            if (lane == 0) atomicOr(err_word, SOCKET_DEVERR_GATHER_TIMEOUT);
+            mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), kMaxPolls);
+            if (j + 1 < cw) mbar_wait_bounded(&bar[warp][st ^ 1], (uint32_t)(((j + 1) >> 1) & 1), kMaxPolls);
+            ok = false;
+            break;
         }
-        // ---- logits of rows 16 warp .. +15 for all heads.
-        {
-            float cl[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            // ldmatrix x4 lane address: matrix q4 = lane/8 -> (rows +8 if q4 odd, cols +8 if q4 >= 2)
-            const int q4 = lane >> 3;
-            const uint32_t a_row = ks_addr + (uint32_t)((warp * 16 + (q4 & 1) * 8 + (lane & 7)) * kMmaRowStride) +
-                                   (uint32_t)((q4 >> 1) * 16);
+        const int nr = min(kWChunk, r_end - (r_begin + (warp + kWWarps * j) * kWChunk));
+        const uint32_t ks = wbase + st * kWStageBytes, vs = ks + kWChunk * kWRowStride;
+        // ---- logits^T: keys 0-7 (c0) and 8-15 (c1) of head lane/4.
+        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                uint32_t a[4];
-                ldsm_x4(a_row + kk * 32, a);
-                mma_bf16(cl, a, qb[kk][0], qb[kk][1]);
-            }
-            const int r = warp * 16 + (lane >> 2), h = (lane & 3) * 2;
-            if (r < nrows) {
-                if (h < G) S[h][r] = cl[0] * kScale;
-                if (h + 1 < G) S[h + 1][r] = cl[1] * kScale;
-            }
-            if (r + 8 < nrows) {
-                if (h < G) S[h][r + 8] = cl[2] * kScale;
-                if (h + 1 < G) S[h + 1][r + 8] = cl[3] * kScale;
-            }
+        for (int kk = 0; kk < 8; ++kk) {
+            uint32_t bk[4];
+            ldsm_x4(ks + lrow + kk * 32, bk);
+            const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
+            mma_bf16(c0, a, bk[0], bk[1]);
+            mma_bf16(c1, a, bk[2], bk[3]);
         }
-        __syncthreads();
-        // ---- running max per head.
+        float sv[4] = {c0[0] * kScale, c0[1] * kScale, c1[0] * kScale, c1[1] * kScale};
+        sv[0] = t2 < nr ? sv[0] : -INFINITY;
+        sv[1] = t2 + 1 < nr ? sv[1] : -INFINITY;
+        sv[2] = t2 + 8 < nr ? sv[2] : -INFINITY;
+        sv[3] = t2 + 9 < nr ? sv[3] : -INFINITY;
+        // ---- online softmax of head lane/4 over the quad's 16 keys.
+        float mc = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+        mc = fmaxf(mc, __shfl_xor_sync(kFullMask, mc, 1));
+        mc = fmaxf(mc, __shfl_xor_sync(kFullMask, mc, 2));
+        const float m_new = fmaxf(m_run, mc);
+        const float sc = expf(m_run - m_new);  // 0 on the first chunk (m_run = -inf)
+        float p[4];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float v = tid < nrows ? S[h][tid] : -INFINITY;
+        for (int e = 0; e < 4; ++e) p[e] = expf(sv[e] - m_new);
+        float ps = (p[0] + p[1]) + (p[2] + p[3]);
+        ps += __shfl_xor_sync(kFullMask, ps, 1);
+        ps += __shfl_xor_sync(kFullMask, ps, 2);
+        l_run = l_run * sc + ps;
+        m_run = m_new;
+        // ---- rescale: the accumulators hold heads 2 (lane%4) and + 1 (quads 2 (lane%4), + 1).
+        const float sa = __shfl_sync(kFullMask, sc, (lane & 3) * 8);
+        const float sb = __shfl_sync(kFullMask, sc, (lane & 3) * 8 + 4);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(kFullMask, v, off));
-            if (lane == 0) red[warp][h] = v;
+        for (int mt = 0; mt < 8; ++mt) {
+            acc[mt][0] *= sa;
+            acc[mt][1] *= sb;
+            acc[mt][2] *= sa;
+            acc[mt][3] *= sb;
         }
-        __syncthreads();
-        if (tid < G) {
-            float mc = red[0][tid];
+        // ---- weights as B: (keys 2 (lane%4) + {0,1}, head lane/4) and keys + 8.
+        const float h0 = bf16_round(p[0]), h1 = bf16_round(p[1]), h2 = bf16_round(p[2]), h3 = bf16_round(p[3]);
+        const uint32_t bh0 = pack_bf16(h0, h1), bh1 = pack_bf16(h2, h3);
+        const uint32_t bl0 = pack_bf16(p[0] - h0, p[1] - h1), bl1 = pack_bf16(p[2] - h2, p[3] - h3);
 #pragma unroll
-            for (int w = 1; w < kThreads / 32; ++w) mc = fmaxf(mc, red[w][tid]);
-            const float mn = fmaxf(m_run[tid], mc);
-            m_new[tid] = mn;
-            scale[tid] = expf(m_run[tid] - mn);  // 0 on the first chunk (m_run = -inf)
+        for (int mt = 0; mt < 8; ++mt) {
+            uint32_t av[4];
+            ldsm_x4_t(vs + lrow + mt * 32, av);
+            // .trans of (keys (q4>>1)*8.., channels 16 mt + (q4&1)*8..) gives A = V^T in
+            // the order (ch 0-7, k 0-7), (ch 8-15, k 0-7), (ch 0-7, k 8-15), (ch 8-15, k 8-15).
+            mma_bf16(acc[mt], av, bh0, bh1);
+            mma_bf16(acc[mt], av, bl0, bl1);
         }
-        __syncthreads();
-        // ---- weights (0 for rows past the chunk's end) and their sums.
+        // Every lane's reads of this stage precede the next copies into it.
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (j + 2 < cw) issue(j + 2, st);
+    }
+    if (!ok) {
+        m_run = -INFINITY;
+        l_run = 0.0f;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float p = 0.0f;
-            if (tid < kMmaChunk) {
-                if (tid < nrows) p = expf(S[h][tid] - m_new[h]);
-                S[h][tid] = p;
-            }
+        for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(kFullMask, p, off);
-            if (lane == 0) red[warp][h] = p;
-        }
-        __syncthreads();
-        // ---- rescale and add this chunk's weighted values on the tensor cores.
-        {
-            const int hb = (lane & 3) * 2;
-            const float s0 = hb < G ? scale[hb] : 0.0f, s1 = hb + 1 < G ? scale[hb + 1] : 0.0f;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                acc[t][0] *= s0;
-                acc[t][1] *= s1;
-                acc[t][2] *= s0;
-                acc[t][3] *= s1;
-            }
-            const int hn = lane >> 2;  // B fragment head (n index)
-            const int q4 = lane >> 3;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                // P^T fragments: rows 16 kk + 2 (lane%4) + {0,1} (+8), head lane/4.
-                const int r0 = kk * 16 + (lane & 3) * 2;
-                float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-                if (hn < G) {
-                    const float2 pa = *reinterpret_cast<const float2*>(&S[hn][r0]);
-                    const float2 pb = *reinterpret_cast<const float2*>(&S[hn][r0 + 8]);
-                    p0 = pa.x;
-                    p1 = pa.y;
-                    p2 = pb.x;
-                    p3 = pb.y;
-                }
-                const float h0 = bf16_round(p0), h1 = bf16_round(p1), h2 = bf16_round(p2), h3 = bf16_round(p3);
-                const uint32_t bh0 = pack_bf16(h0, h1), bh1 = pack_bf16(h2, h3);
-                const uint32_t bl0 = pack_bf16(p0 - h0, p1 - h1), bl1 = pack_bf16(p2 - h2, p3 - h3);
-                // V^T tile via ldmatrix.trans: matrix q4 -> value rows 16 kk + 8 (q4 >> 1) + lane%8,
-                // columns 16 mt + 8 (q4 & 1).
-                const uint32_t v_row =
-                    vs_addr + (uint32_t)((kk * 16 + (q4 >> 1) * 8 + (lane & 7)) * kMmaRowStride) + (uint32_t)((q4 & 1) * 16);
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const int mt = warp * 2 + t;
-                    uint32_t a[4];
-                    ldsm_x4_t(v_row + mt * 32, a);
-                    mma_bf16(acc[t], a, bh0, bh1);
-                    mma_bf16(acc[t], a, bl0, bl1);
-                }
-            }
-        }
-        if (tid < G) {
-            float lc = 0.0f;
-#pragma unroll
-            for (int w = 0; w < kThreads / 32; ++w) lc += red[w][tid];
-            l_run[tid] = l_run[tid] * scale[tid] + lc;
-            m_run[tid] = m_new[tid];
-        }
-        __syncthreads();  // stage st and S are free again
-        if (c + 2 < nchunks) issue(c + 2, st);
+            for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
     }
 
-    // ---- partials: out^T accumulators -> part_o[(unit, head, split)][column].
+    // ---- merge the two warps: warp 1 leaves (m, l, o^T) in its own stage memory.
+    float* xo = reinterpret_cast<float*>(smem + kWStages * kWStageBytes);  // warp 1's area, [8 heads][128]
+    if (warp == 1) {
+        if ((lane & 3) == 0) {
+            xm[1][lane >> 2] = m_run;
+            xl[1][lane >> 2] = l_run;
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int ch = mt * 16 + (lane >> 2);
+            xo[t2 * kHeadDim + ch] = acc[mt][0];
+            xo[(t2 + 1) * kHeadDim + ch] = acc[mt][1];
+            xo[t2 * kHeadDim + ch + 8] = acc[mt][2];
+            xo[(t2 + 1) * kHeadDim + ch + 8] = acc[mt][3];
+        }
+    } else if ((lane & 3) == 0) {
+        xm[0][lane >> 2] = m_run;
+        xl[0][lane >> 2] = l_run;
+    }
+    __syncthreads();
     const int64_t pbase = u * G * (int64_t)nsplit;
-    {
-        const int hb = (lane & 3) * 2;
+    if (warp == 0) {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int j = (warp * 2 + t) * 16 + (lane >> 2);
-            if (hb < G) {
-                part_o[((pbase + hb * nsplit) + split) * kHeadDim + j] = acc[t][0];
-                part_o[((pbase + hb * nsplit) + split) * kHeadDim + j + 8] = acc[t][2];
-            }
-            if (hb + 1 < G) {
-                part_o[((pbase + (hb + 1) * nsplit) + split) * kHeadDim + j] = acc[t][1];
-                part_o[((pbase + (hb + 1) * nsplit) + split) * kHeadDim + j + 8] = acc[t][3];
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = t2 + hh;
+            if (h < G) {
+                const float M = fmaxf(xm[0][h], xm[1][h]);
+                const float w0 = xm[0][h] == -INFINITY ? 0.0f : expf(xm[0][h] - M);
+                const float w1 = xm[1][h] == -INFINITY ? 0.0f : expf(xm[1][h] - M);
+                float* po = part_o + ((pbase + h * nsplit) + split) * kHeadDim;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    const int ch = mt * 16 + (lane >> 2);
+                    po[ch] = w0 * acc[mt][hh] + w1 * xo[h * kHeadDim + ch];
+                    po[ch + 8] = w0 * acc[mt][2 + hh] + w1 * xo[h * kHeadDim + ch + 8];
+                }
+                if ((lane >> 2) == 0) part_ml[pbase + h * nsplit + split] = make_float2(M, w0 * xl[0][h] + w1 * xl[1][h]);
             }
         }
     }
-    if (tid < G) part_ml[pbase + tid * nsplit + split] = make_float2(m_run[tid], l_run[tid]);
-    merge_unit<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
+    merge_unit<G, kWThreads>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
 }
 
 template <int G>
-cudaError_t launch_mma(const void* q, const void* K, const void* V, const int32_t* idx, const DecodeShape& s,
-                       float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word, float* out,
-                       cudaStream_t stream)
+cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32_t* idx, const DecodeShape& s,
+                        float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word, float* out,
+                        cudaStream_t stream)
 {
-    constexpr int smem = 2 * kMmaStageBytes;
-    static_assert(kMmaChunk == Rows<uint16_t>::kChunk, "splits are sized with the bfloat16 chunk");
-    const int rpc = attention_rows_per_cta(s.k, s.nsplit, kMmaChunk);
-    auto kern = attention_mma_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int rpc = attention_rows_per_cta(s.k, s.nsplit, kWChunk);
+    auto kern = attention_warp_kernel<G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream,
+    e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
                    idx, s.Hq, s.Hkv, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out);
     if (e != cudaSuccess) return e;
@@ -656,13 +656,16 @@ int attention_rows_per_cta(int k, int nsplit, int chunk)
     return (per + chunk - 1) / chunk * chunk;
 }
 
-int attention_splits(int kv_dtype, int64_t U, int k, int num_sms)
+int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num_sms)
 {
-    // About three CTAs per SM in one wave, each over whole chunks.
-    const int chunk = attention_chunk_rows(kv_dtype);
+    // One wave: about kWCtasPerSm two-warp CTAs per SM on the tensor-core path,
+    // three four-warp CTAs per SM otherwise, each over whole chunks.
+    const bool wp = warp_path(kv_dtype, q_dtype, G);
+    const int chunk = wp ? kWChunk : attention_chunk_rows(kv_dtype);
+    const int per_sm = wp ? kWCtasPerSm : 3;
     const int max_splits = (k + chunk - 1) / chunk;
-    int64_t want = (3 * (int64_t)num_sms + U - 1) / U;
-    int splits = (int)max64(1, min64(want, max_splits));
+    const int64_t want = max64(1, (int64_t)per_sm * num_sms / U);
+    const int splits = (int)max64(1, min64(want, max_splits));
     const int rpc = attention_rows_per_cta(k, splits, chunk);
     return (k + rpc - 1) / rpc;
 }
@@ -671,9 +674,9 @@ cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const vo
                              const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
                              uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream)
 {
-    if (kv_dtype == 1 && q_dtype == 1 && s.G <= 8) {
+    if (warp_path(kv_dtype, q_dtype, s.G)) {
 #define SOCKET_MMA_CASE(g) \
-    case g: return launch_mma<g>(q, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
+    case g: return launch_warp<g>(q, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
         switch (s.G) {
             SOCKET_MMA_CASE(1) SOCKET_MMA_CASE(2) SOCKET_MMA_CASE(3) SOCKET_MMA_CASE(4)
             SOCKET_MMA_CASE(5) SOCKET_MMA_CASE(6) SOCKET_MMA_CASE(7) SOCKET_MMA_CASE(8)

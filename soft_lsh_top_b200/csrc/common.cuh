@@ -78,6 +78,13 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
         : "memory");
 }
 
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) writes to the same memory.
+__device__ __forceinline__ void fence_proxy_async_shared()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Hint the L2 to start fetching [src, src + bytes); bytes a multiple of 16.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes)
 {

@@ -45,8 +45,8 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s);
 
 // Rows of one attention chunk (the gather unit of the attention kernel).
 int attention_chunk_rows(int kv_dtype);
-// Attention CTAs per unit for these sizes (<= ceil(k / chunk rows)).
-int attention_splits(int kv_dtype, int64_t U, int k, int num_sms);
+// Attention CTAs per unit for these sizes (<= ceil(k / 16)).
+int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num_sms);
 int attention_rows_per_cta(int k, int nsplit, int chunk);
 int device_num_sms();
 

@@ -65,11 +65,6 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr)
     return v;
 }
 
-__device__ __forceinline__ void fence_proxy_async_shared()
-{
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int i)
 {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
@@ -216,11 +211,11 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                 if (LAST) bulk_copy_g2s(dst + j * kChunkBytes + kChunkIds, vu + (int64_t)c * 32, 128u, &ring_bar[warp][st]);
             }
         };
+        // The stages were read in the previous segment: fence every lane's reads.
+        fence_proxy_async_shared();
         __syncwarp();
-        if (lane == 0 && !failed) {
-            if (k > 0) fence_proxy_async_shared();  // the stages were read in the previous segment
+        if (lane == 0 && !failed)
             for (int b = 0; b < min(NS, nbatch); ++b) issue(b);
-        }
         if (k == 0) {
             // The soft tables (and, after the first launch, the partial sums)
             // come from the previous kernel on the stream.
@@ -255,11 +250,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                 for (int i = 0; i < V; ++i) v[j][i] = lds_u4(sa + j * kChunkBytes + i * 512 + lane * 16);
                 vn[j] = LAST ? lds_f32(sa + j * kChunkBytes + kChunkIds + lane * 4) : 0.0f;
             }
+            // Every lane's reads of this stage precede the next copy into it.
+            fence_proxy_async_shared();
             __syncwarp();
-            if (lane == 0 && b + NS < nbatch) {
-                fence_proxy_async_shared();  // the reads above precede the next copy into this stage
-                issue(b + NS);
-            }
+            if (lane == 0 && b + NS < nbatch) issue(b + NS);
             float acc[KEYS];
 #pragma unroll
             for (int j = 0; j < KEYS; ++j)
