@@ -34,6 +34,8 @@ constexpr int kBatch = 8;                             // 16-byte loads in flight
 constexpr int kMaxCluster = 16;
 constexpr int kWindowShift = 15;                      // multi-pass first digit: 2^15 ulps (1/256 octave)
 constexpr int kCand = kTopkCandidates;
+constexpr int kBitmapKeys = 65536;                    // fast path compacts from a bitmap of up to this many keys
+constexpr int kBitmapWords = kBitmapKeys / 32;
 
 // Block-wide exclusive prefix sum of one uint32 per thread; also returns the total.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t& total)
@@ -73,6 +75,9 @@ struct Shared {
         __align__(16) uint32_t slice[kBins];
         uint2 cand[kCand];  // (global index, bit pattern) of the unit's candidates
     };
+    // Candidate path: bit i set for key lo + i of the slice if it is selected
+    // (first every key in or above the threshold bin, then pruned).
+    uint32_t bits[kBitmapWords];
 };
 
 // Finds, over bins given in descending order as per-thread runs of `nb`
@@ -293,9 +298,13 @@ __device__ uint32_t select_multipass(cg::cluster_group& cluster, const uint32_t*
 // with two more radix digits (11 + 8 bits) in its own shared memory -- the
 // same exact threshold t and tie count everywhere.  The CTA's output offset
 // follows from the "sure" counts of lower-ranked CTAs (distributed shared
-// memory) and the candidate list, and it writes its selected indices in
-// index order.  If the threshold bin holds more than kTopkCandidates keys,
-// the cluster takes the multi-pass path instead.
+// memory) and the candidate list.  The same single read of the scores marks
+// every key in or above bin d0 in a bitmap of the CTA's slice; the slice's
+// candidates below t (and ties past the tie budget, by index) are cleared,
+// and the CTA writes the set bits in index order from one block scan over
+// the words' popcounts.  Slices over kBitmapKeys keys re-read the scores
+// instead (compact).  If the threshold bin holds more than kTopkCandidates
+// keys, the cluster takes the multi-pass path.
 __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restrict__ scores,
                                                         const uint32_t* __restrict__ unit_max,
                                                         const uint32_t* __restrict__ unit_hist,
@@ -303,7 +312,8 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
                                                         int64_t Ncap, int N, int k, int R,
                                                         int32_t* __restrict__ idx_out)
 {
-    __shared__ Shared sh;
+    extern __shared__ __align__(16) char topk_smem[];
+    Shared& sh = *reinterpret_cast<Shared*>(topk_smem);
     cg::cluster_group cluster = cg::this_cluster();
     const unsigned rank = cluster.block_rank(), C = cluster.num_blocks();
     const int tid = threadIdx.x;
@@ -374,9 +384,17 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
         budget = need > ties_before ? need - ties_before : 0u;
         cluster.sync();  // no remote shared-memory access after this point
     } else {
-        // ---- candidates of this slice -> the unit list; count keys above bin d0.
+        // ---- candidates of this slice -> the unit list; count keys above bin d0;
+        // mark every key in or above bin d0 in the slice bitmap.
+        const bool use_bits = n <= kBitmapKeys;
+        const int words = (n + 31) / 32;
+        if (use_bits) {
+            for (int w = tid; w < words; w += kThreads) sh.bits[w] = 0u;
+            __syncthreads();
+        }
+        const int lane = tid & 31;
         uint32_t sure = 0;
-        for (int base = tid * 4; base < n; base += kThreads * 4 * kBatch) {
+        for (int base = tid * 4; base - tid * 4 < n; base += kThreads * 4 * kBatch) {
             uint4 v[kBatch];
 #pragma unroll
             for (int b = 0; b < kBatch; ++b) {
@@ -387,17 +405,27 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
             for (int b = 0; b < kBatch; ++b) {
                 const int i = base + b * kThreads * 4;
                 const uint32_t vals[4] = {v[b].x, v[b].y, v[b].z, v[b].w};
+                uint32_t nib = 0;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if (i + e < n) {
                         const uint32_t top = vals[e] >> kScoreHistShift;
                         sure += top > d0;
+                        nib |= (uint32_t)(top >= d0) << e;
                         if (top == d0) {
                             const uint32_t slot = atomicAdd(cand_cnt + u, 1u);
                             if (slot < (uint32_t)kCand)
                                 cand[u * kCand + slot] = make_uint2((uint32_t)(lo + i + e), vals[e]);
                         }
                     }
+                }
+                if (use_bits) {
+                    // Lanes 8m .. 8m + 7 hold the 32 consecutive keys of one bitmap word.
+                    uint32_t word = nib << ((lane & 7) * 4);
+                    word |= __shfl_xor_sync(kFullMask, word, 1);
+                    word |= __shfl_xor_sync(kFullMask, word, 2);
+                    word |= __shfl_xor_sync(kFullMask, word, 4);
+                    if ((lane & 7) == 0 && i < n) sh.bits[i >> 5] = word;
                 }
             }
         }
@@ -444,19 +472,63 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
         need = krem;
         // Keys before this slice that are selected: sure keys of lower CTAs,
         // candidates above t before lo, and ties at t before lo (up to need).
-        uint32_t gt_before = 0, eq_before = 0;
+        uint32_t gt_before = 0, eq_before = 0, eq_all = 0;
         for (int i = tid; i < nc; i += kThreads) {
             const uint2 e = sh.cand[i];
             if ((int)e.x < lo) {
                 gt_before += e.y > t;
                 eq_before += e.y == t;
             }
+            eq_all += e.y == t;
         }
-        uint32_t tg, te;
+        uint32_t tg, te, tall;
         block_exclusive_scan(gt_before, sh.warp_sums, tg);
         block_exclusive_scan(eq_before, sh.warp_sums, te);
+        block_exclusive_scan(eq_all, sh.warp_sums, tall);
         out_base = sure_before + tg + min(te, need);
         budget = need > te ? need - te : 0u;
+        if (use_bits) {
+            // Prune the slice's candidates: keep those above t, and ties at t
+            // whose rank by index among all of the unit's ties is below need.
+            for (int i = tid; i < nc; i += kThreads) {
+                const uint2 e = sh.cand[i];
+                if ((int)e.x < lo || (int)e.x >= hi) continue;
+                bool keep = e.y > t;
+                if (e.y == t) {
+                    if (tall <= need) {
+                        keep = true;
+                    } else {
+                        uint32_t rank_t = 0;
+                        for (int j = 0; j < nc; ++j) rank_t += sh.cand[j].y == t && sh.cand[j].x < e.x;
+                        keep = rank_t < need;
+                    }
+                }
+                if (!keep) atomicAnd(&sh.bits[(e.x - lo) >> 5], ~(1u << ((e.x - lo) & 31)));
+            }
+            __syncthreads();
+            // Selected keys in index order: each thread takes consecutive words.
+            constexpr int kWordsPerThread = kBitmapWords / kThreads;
+            const int w0 = tid * kWordsPerThread;
+            uint32_t cnt = 0;
+#pragma unroll
+            for (int q = 0; q < kWordsPerThread; ++q) cnt += w0 + q < words ? __popc(sh.bits[w0 + q]) : 0u;
+            uint32_t total;
+            uint32_t pos = out_base + block_exclusive_scan(cnt, sh.warp_sums, total);
+#pragma unroll
+            for (int q = 0; q < kWordsPerThread; ++q) {
+                if (w0 + q >= words) break;
+                uint32_t x = sh.bits[w0 + q];
+                while (x) {
+                    const int bit = __ffs(x) - 1;
+                    x &= x - 1;
+                    // pos < k always holds when the threshold is exact; the guard
+                    // keeps every store inside the unit's k slots regardless.
+                    if (pos < (uint32_t)k) out[pos] = lo + 32 * (w0 + q) + bit;
+                    ++pos;
+                }
+            }
+            return;
+        }
     }
     compact(su, lo, hi, t, budget, out_base, k, out, sh);
 }
@@ -472,10 +544,12 @@ cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const uin
     const int R = (int)(((s.N + C - 1) / C + 31) / 32 * 32);
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Shared));
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(s.U * C));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = sizeof(Shared);
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
