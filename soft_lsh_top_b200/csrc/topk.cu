@@ -70,6 +70,7 @@ struct Shared {
     uint32_t warp_sums[32];
     uint32_t digit, krem, sure, total, pick, pick_above, grand;
     uint32_t counts[2];
+    uint32_t nlocal, local_base;  // this CTA's candidates, and their offset in the unit list
     __align__(16) uint32_t hist[kBins];
     union {  // the multi-pass path uses `slice`, the candidate path `cand`
         __align__(16) uint32_t slice[kBins];
@@ -77,7 +78,7 @@ struct Shared {
     };
     // Candidate path: bit i set for key lo + i of the slice if it is selected
     // (first every key in or above the threshold bin, then pruned).
-    uint32_t bits[kBitmapWords];
+    __align__(16) uint32_t bits[kBitmapWords];
 };
 
 // Finds, over bins given in descending order as per-thread runs of `nb`
@@ -388,10 +389,10 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
         // mark every key in or above bin d0 in the slice bitmap.
         const bool use_bits = n <= kBitmapKeys;
         const int words = (n + 31) / 32;
-        if (use_bits) {
+        if (use_bits)
             for (int w = tid; w < words; w += kThreads) sh.bits[w] = 0u;
-            __syncthreads();
-        }
+        if (tid == 0) sh.nlocal = 0;
+        __syncthreads();
         const int lane = tid & 31;
         uint32_t sure = 0;
         for (int base = tid * 4; base - tid * 4 < n; base += kThreads * 4 * kBatch) {
@@ -413,9 +414,9 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
                         sure += top > d0;
                         nib |= (uint32_t)(top >= d0) << e;
                         if (top == d0) {
-                            const uint32_t slot = atomicAdd(cand_cnt + u, 1u);
-                            if (slot < (uint32_t)kCand)
-                                cand[u * kCand + slot] = make_uint2((uint32_t)(lo + i + e), vals[e]);
+                            // The unit's bin holds <= kCand keys, so the slice's do too.
+                            const uint32_t slot = atomicAdd(&sh.nlocal, 1u);
+                            if (slot < (uint32_t)kCand) sh.cand[slot] = make_uint2((uint32_t)(lo + i + e), vals[e]);
                         }
                     }
                 }
@@ -430,8 +431,18 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
             }
         }
         uint32_t sure_total;
-        block_exclusive_scan(sure, sh.warp_sums, sure_total);
-        if (tid == 0) sh.sure = sure_total;
+        block_exclusive_scan(sure, sh.warp_sums, sure_total);  // (its barriers also order sh.nlocal)
+        if (tid == 0) {
+            sh.sure = sure_total;
+            sh.local_base = atomicAdd(cand_cnt + u, min(sh.nlocal, (uint32_t)kCand));
+        }
+        __syncthreads();
+        {
+            // Append this slice's candidates to the unit list with one atomic per CTA.
+            const uint32_t nl = min(sh.nlocal, (uint32_t)kCand), lb = sh.local_base;
+            for (uint32_t i = tid; i < nl; i += kThreads)
+                if (lb + i < (uint32_t)kCand) cand[u * kCand + lb + i] = sh.cand[i];
+        }
         __threadfence();
         cluster.sync();  // candidate list complete; sure counts visible
         if (tid == 0) {
@@ -506,18 +517,27 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
                 if (!keep) atomicAnd(&sh.bits[(e.x - lo) >> 5], ~(1u << ((e.x - lo) & 31)));
             }
             __syncthreads();
-            // Selected keys in index order: each thread takes consecutive words.
+            // Selected keys in index order: each thread takes consecutive words
+            // (read 16 bytes at a time; words past the slice are zero).
             constexpr int kWordsPerThread = kBitmapWords / kThreads;
             const int w0 = tid * kWordsPerThread;
+            uint32_t wv[kWordsPerThread];
+#pragma unroll
+            for (int q = 0; q < kWordsPerThread; q += 4) {
+                const uint4 x4 = w0 + q < words ? *reinterpret_cast<const uint4*>(&sh.bits[w0 + q]) : make_uint4(0, 0, 0, 0);
+                wv[q] = x4.x;
+                wv[q + 1] = w0 + q + 1 < words ? x4.y : 0u;
+                wv[q + 2] = w0 + q + 2 < words ? x4.z : 0u;
+                wv[q + 3] = w0 + q + 3 < words ? x4.w : 0u;
+            }
             uint32_t cnt = 0;
 #pragma unroll
-            for (int q = 0; q < kWordsPerThread; ++q) cnt += w0 + q < words ? __popc(sh.bits[w0 + q]) : 0u;
+            for (int q = 0; q < kWordsPerThread; ++q) cnt += __popc(wv[q]);
             uint32_t total;
             uint32_t pos = out_base + block_exclusive_scan(cnt, sh.warp_sums, total);
 #pragma unroll
             for (int q = 0; q < kWordsPerThread; ++q) {
-                if (w0 + q >= words) break;
-                uint32_t x = sh.bits[w0 + q];
+                uint32_t x = wv[q];
                 while (x) {
                     const int bit = __ffs(x) - 1;
                     x &= x - 1;
