@@ -289,28 +289,39 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         step(s)
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, per-kernel events recorded by the library.
+    # ---- timed region: K steps back to back (kernels chain by programmatic
+    # dependent launch; nothing is recorded between them).
     K = args.steps
-    nk = 4
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
-    for row in evs:  # torch creates the CUDA event on first record
-        for e in row:
-            e.record()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
         start.record()
         for s in range(K):
-            sk.socket_set_step_events(evs[s])
             step(s)
         end.record()
         torch.cuda.synchronize()
-    sk.socket_set_step_events([])
     barrier(world)
     ms_total = max_over_ranks(start.elapsed_time(end), world)
+    assert sk.read_device_error(ws) == 0
+
+    # ---- per-kernel durations: a second pass with events recorded by the
+    # library between the kernels, on the launching stream.  The events
+    # serialise the kernels, so these are each kernel's own time.
+    KD = min(K, 200)
+    nk = 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(KD)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    for s in range(KD):
+        sk.socket_set_step_events(evs[s])
+        step(s)
+    torch.cuda.synchronize()
+    sk.socket_set_step_events([])
     names = ["soft_tables", "score", "topk", "attention"]
-    kern_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(K))
+    kern_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(KD))
                for i, n in enumerate(names)}
     assert sk.read_device_error(ws) == 0
 

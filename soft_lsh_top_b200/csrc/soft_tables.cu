@@ -56,6 +56,14 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // Rows ordered (head, table, plane); thread pair (2r, 2r + 1) takes row r.
+    // This kernel may be launched before the previous kernel on the stream
+    // has finished (programmatic dependent launch): q and W may come from
+    // it, so nothing is read before the wait.  The scoring kernel may start
+    // once the wait is over (its early id loads then see every earlier
+    // kernel's writes).
+    pdl_wait();
+    pdl_launch_dependents();
+
     const int rows = G * nt * P;
     const int half = tid & 1;
     int r = tid >> 1;
@@ -67,19 +75,6 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         for (int c = 0; c < kHalf / 8; ++c) wv[c] = __ldg(w + c);
     };
     if (r < rows) load_w(r);
-
-    if (blockIdx.y == 0) {
-        if (tid == 0) {
-            counters[u] = 0u;
-            unit_max[u] = 0u;
-            cand_cnt[u] = 0u;
-            if (u == 0) *err_word = 0u;
-        }
-        uint4* h = reinterpret_cast<uint4*>(unit_hist + u * kScoreHistBins);
-        for (int i = tid; i < kScoreHistBins / 4; i += kThreads) h[i] = make_uint4(0, 0, 0, 0);
-    }
-    // Let the scoring kernel start its table-independent prologue.
-    pdl_launch_dependents();
 
     const QT* qu = q + (b * Hq + kvh * G) * kHeadDim;
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
@@ -137,6 +132,16 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     }
     __syncthreads();
 
+    if (blockIdx.y == 0) {
+        if (tid == 0) {
+            counters[u] = 0u;
+            unit_max[u] = 0u;
+            cand_cnt[u] = 0u;
+            if (u == 0) *err_word = 0u;
+        }
+        uint4* h = reinterpret_cast<uint4*>(unit_hist + u * kScoreHistBins);
+        for (int i = tid; i < kScoreHistBins / 4; i += kThreads) h[i] = make_uint4(0, 0, 0, 0);
+    }
     const int nblk = (L + 31) / 32;
     float* tu = tables + u * nblk * (int64_t)NB * 64;
     for (int e = tid; e < nt * NB; e += kThreads) {
@@ -168,14 +173,11 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
 {
     dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
     if (q_dtype == 1)
-        soft_tables_kernel<uint16_t><<<grid, kThreads, 0, stream>>>(
-            static_cast<const uint16_t*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
-            unit_max, unit_hist, cand_cnt);
-    else
-        soft_tables_kernel<float><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters,
-            unit_max, unit_hist, cand_cnt);
-    return cudaGetLastError();
+        return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), 0, stream,
+                          static_cast<const uint16_t*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word,
+                          counters, unit_max, unit_hist, cand_cnt);
+    return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), 0, stream, static_cast<const float*>(q), W,
+                      s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt);
 }
 
 }  // namespace socket_attn
