@@ -436,10 +436,16 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     __syncthreads();
     pdl_wait();  // the selected indices come from the previous kernel on the stream
 
+    // Row index of this lane's row (lane % 16) of chunk j, or -1 past the end.
+    auto row_index = [&](int j) -> int32_t {
+        const int r0 = r_begin + (warp + kWWarps * j) * kWChunk;
+        const int i = lane & 15;
+        return (j < cw && i < r_end - r0) ? __ldcg(idx + u * k + r0 + i) : -1;
+    };
     // Gather this warp's chunk j into stage st: lane i < 16 copies key row i,
     // lane 16 + i value row i; value rows past the chunk's end are zeroed
     // (their weights are 0, and 0 * NaN from stale bytes must not happen).
-    auto issue = [&](int j, int st) {
+    auto issue = [&](int j, int st, int32_t r) {
         const int r0 = r_begin + (warp + kWWarps * j) * kWChunk;
         const int nr = min(kWChunk, r_end - r0);
         const int i = lane & 15;
@@ -447,7 +453,6 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         if (i < nr) {
             // Indices come from the top-k kernel and are < N; clamp anyway so a
             // gather can never leave the unit's cache rows.
-            int32_t r = __ldcg(idx + u * k + r0 + i);
             r = (r >= 0 && r < Ncap) ? r : 0;
             const uint16_t* src = (lane < 16 ? K : V) + (u * Ncap + r) * kHeadDim;
             bulk_copy_g2s(dst, src, kHeadDim * 2, &bar[warp][st]);
@@ -458,8 +463,8 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         }
         if (lane == 0) mbar_arrive_expect_tx(&bar[warp][st], (uint32_t)nr * 2u * kHeadDim * 2u);
     };
-    if (cw > 0) issue(0, 0);
-    if (cw > 1) issue(1, 1);
+    if (cw > 0) issue(0, 0, row_index(0));
+    if (cw > 1) issue(1, 1, row_index(1));
     __syncwarp();  // zeroed value rows visible to the warp
 
     // out^T accumulators: m-tile mt = channels 16 mt ..; [0], [1]: channel
@@ -477,6 +482,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     bool ok = true;
     for (int j = 0; j < cw; ++j) {
         const int st = j & 1;
+        const int32_t next_row = row_index(j + 2);  // in flight while chunk j is used
         const bool got = mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), kMaxPolls);
         if (__any_sync(kFullMask, !got)) {
             if (lane == 0) atomicOr(err_word, SOCKET_DEVERR_GATHER_TIMEOUT);
@@ -542,7 +548,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         // Every lane's reads of this stage precede the next copies into it.
         fence_proxy_async_shared();
         __syncwarp();
-        if (j + 2 < cw) issue(j + 2, st);
+        if (j + 2 < cw) issue(j + 2, st, next_row);
     }
     if (!ok) {
         m_run = -INFINITY;

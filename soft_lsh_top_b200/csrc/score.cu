@@ -28,11 +28,14 @@
 // A region starts at a 64 KB-aligned shared address, so one byte-permute of
 // the packed id word (id into byte 1, lane column in byte 0) gives the row
 // address and the round's column is the load's immediate offset: a lookup is
-// one PRMT, one LDS and one FADD.  Each thread keeps KEYS keys in flight with
-// the next batch's id pieces loading behind them.  The grid is persistent
-// (one CTA per SM) and splits the flattened (unit, 32-key chunk) range
-// evenly; a CTA stages the tables of each unit it touches (two units at once
-// when a unit needs one region).
+// one PRMT, one LDS and one FADD.  Each warp streams its batches (KEYS
+// consecutive 32-key chunks of id pieces and norms, one bulk copy each) into
+// its own ring of shared-memory stages on mbarriers, and reads them back with
+// conflict-free 16-byte loads; ids and norms stream through L2 with an
+// evict-first policy and the scores are stored evict-last, so top-k reads
+// them from L2.  The grid is persistent (one CTA per SM) and splits the
+// flattened (unit, 32-key chunk) range evenly; a CTA stages the tables of
+// each unit it touches (two units at once when a unit needs one region).
 #include "common.cuh"
 #include "internal.h"
 #include "socket_attn.h"
@@ -178,6 +181,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     };
 
     uint32_t mx = 0;
+    // Ids and norms stream through L2 once; the scores stay there for top-k.
+    const uint64_t pol_stream = l2_policy_evict_first(), pol_keep = l2_policy_evict_last();
     uint32_t seq = 0;      // batches this warp has taken from its ring so far
     bool failed = false;   // a bounded wait of this warp expired
     for (int k = 0; k < nseg; ++k) {
@@ -185,31 +190,39 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         const int cbeg = (int)(max64(c0, u * cpu) - u * cpu);
         const int nch = (int)(min64(c1, (u + 1) * cpu) - u * cpu) - cbeg;
         const int slot = k % kSlots;
-        // This warp's chunks: cbeg + warp + kWarps * m for m < cnt; batch b
-        // holds m = KEYS b .. KEYS b + KEYS - 1.
-        const int cnt = nch > warp ? (nch - warp + kWarps - 1) / kWarps : 0;
-        const int nbatch = (cnt + KEYS - 1) / KEYS;
+        // Batch b of this warp holds the KEYS consecutive chunks starting at
+        // cbeg + (warp + kWarps b) KEYS (the last group of the segment may be
+        // shorter); m = KEYS b + j indexes its chunks.
+        const int ngroups = (nch + KEYS - 1) / KEYS;
+        const int nbatch = ngroups > warp ? (ngroups - warp + kWarps - 1) / kWarps : 0;
+        auto chunk_at = [&](int m) { return cbeg + (warp + kWarps * (m / KEYS)) * KEYS + (m % KEYS); };
+        const int cend = cbeg + nch;
         const uint8_t* idu = a.ids + u * a.Ncap * Lr;
         const float* vu = a.vnorm + u * a.Ncap;
         float* su = a.scores + u * a.Ncap;
-        const int key0 = (cbeg + warp) * 32 + lane;  // this lane's key of m = 0
-        constexpr int kKeyStride = kWarps * 32;       // keys between m and m + 1
 
         // Lane 0: copy batch b's chunks (this launch's id pieces and, in the
-        // last launch, the norms) into ring stage (seq + b) % NS.  Chunks past
-        // the warp's last repeat it; the unit's last chunk may run past N
-        // (rows below Ncap, never scored).
+        // last launch, the norms) into ring stage (seq + b) % NS, laid out as
+        // [KEYS chunks of ids][KEYS x 32 norms].  When the launch covers the
+        // whole id row, the chunks' ids are one contiguous run.  The unit's
+        // last chunk may run past N (rows below Ncap, never scored).
         auto issue = [&](int b) {
             const uint32_t st = (seq + b) % NS;
             char* dst = ring + st * kStageBytes;
-            mbar_arrive_expect_tx(&ring_bar[warp][st], kStageBytes);
-#pragma unroll
-            for (int j = 0; j < KEYS; ++j) {
-                const int c = cbeg + warp + kWarps * min(b * KEYS + j, cnt - 1);
-                bulk_copy_g2s(dst + j * kChunkBytes, idu + (int64_t)c * 32 * Lr + (2 * a.blk0) * 512, kChunkIds,
-                              &ring_bar[warp][st]);
-                if (LAST) bulk_copy_g2s(dst + j * kChunkBytes + kChunkIds, vu + (int64_t)c * 32, 128u, &ring_bar[warp][st]);
+            const int c0 = chunk_at(b * KEYS);
+            const int nv = min(KEYS, cend - c0);
+            mbar_arrive_expect_tx(&ring_bar[warp][st], (uint32_t)nv * kChunkBytes);
+            if (NBLK == a.nblk) {
+                bulk_copy_g2s_hint(dst, idu + (int64_t)c0 * 32 * Lr, (uint32_t)nv * kChunkIds, &ring_bar[warp][st],
+                                   pol_stream);
+            } else {
+                for (int j = 0; j < nv; ++j)
+                    bulk_copy_g2s_hint(dst + j * kChunkIds, idu + (int64_t)(c0 + j) * 32 * Lr + (2 * a.blk0) * 512,
+                                       kChunkIds, &ring_bar[warp][st], pol_stream);
             }
+            if (LAST)
+                bulk_copy_g2s_hint(dst + KEYS * kChunkIds, vu + (int64_t)c0 * 32, (uint32_t)nv * 128u,
+                                   &ring_bar[warp][st], pol_stream);
         };
         // The stages were read in the previous segment: fence every lane's reads.
         fence_proxy_async_shared();
@@ -247,8 +260,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 #pragma unroll
             for (int j = 0; j < KEYS; ++j) {
 #pragma unroll
-                for (int i = 0; i < V; ++i) v[j][i] = lds_u4(sa + j * kChunkBytes + i * 512 + lane * 16);
-                vn[j] = LAST ? lds_f32(sa + j * kChunkBytes + kChunkIds + lane * 4) : 0.0f;
+                for (int i = 0; i < V; ++i) v[j][i] = lds_u4(sa + j * kChunkIds + i * 512 + lane * 16);
+                vn[j] = LAST ? lds_f32(sa + KEYS * kChunkIds + j * 128 + lane * 4) : 0.0f;
             }
             // Every lane's reads of this stage precede the next copy into it.
             fence_proxy_async_shared();
@@ -257,7 +270,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
             float acc[KEYS];
 #pragma unroll
             for (int j = 0; j < KEYS; ++j)
-                acc[j] = FIRST ? 0.0f : __ldcg(su + min(key0 + kKeyStride * min(b * KEYS + j, cnt - 1), N - 1));
+                acc[j] = FIRST ? 0.0f : __ldcg(su + min(min(chunk_at(b * KEYS + j), cend - 1) * 32 + lane, N - 1));
 #pragma unroll
             for (int bl = 0; bl < NBLK; ++bl) {
                 const uint32_t base = region0 + (uint32_t)(slot * NBLK + bl) * kRegionBytes + ((uint32_t)lane << 2);
@@ -275,11 +288,11 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
             }
 #pragma unroll
             for (int j = 0; j < KEYS; ++j) {
-                const int m = b * KEYS + j;
-                const int n = key0 + kKeyStride * m;
-                if (m < cnt && n < N) {
+                const int c = chunk_at(b * KEYS + j);
+                const int n = c * 32 + lane;
+                if (c < cend && n < N) {
                     const float sc = LAST ? acc[j] * vn[j] : acc[j];
-                    su[n] = sc;
+                    st_global_hint(su + n, sc, pol_keep);
                     if (LAST) {
                         const uint32_t bits = __float_as_uint(sc);
                         mx = max(mx, bits);
