@@ -385,6 +385,75 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 }
 __device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(pack_bf16(x, 0.0f) << 16); }
 
+// The unit's last CTA merges the splits' partials: head h is merged by warp
+// h % kWWarps with no CTA barrier.  For each head, M = max_s m_s, the weights
+// w_s = exp(m_s - M) live in the lanes (split s in lane s % 32, a tile of 32
+// splits at a time) and reach the others by shuffle, and each lane
+// accumulates four output columns from 16-byte loads of every split's row,
+// in split order: out = sum_s w_s o_s / sum_s w_s l_s.
+template <int G>
+__device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
+                                                 const float* __restrict__ part_o, const float2* __restrict__ part_ml,
+                                                 uint32_t* __restrict__ counters, float* __restrict__ out,
+                                                 uint32_t& s_last)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&counters[u], 1u) == (uint32_t)(nsplit - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int h = warp; h < G; h += kWWarps) {
+        const int64_t base = pbase + h * nsplit;
+        float M = -INFINITY;
+        for (int s0 = 0; s0 < nsplit; s0 += 32)
+            if (s0 + lane < nsplit) M = fmaxf(M, __ldcg(&part_ml[base + s0 + lane]).x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, o));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float lsum = 0.0f;
+        for (int s0 = 0; s0 < nsplit; s0 += 32) {
+            const int cnt = min(32, nsplit - s0);
+            float w = 0.0f;
+            if (lane < cnt) {
+                const float2 t = __ldcg(&part_ml[base + s0 + lane]);
+                w = t.x == -INFINITY ? 0.0f : expf(t.x - M);
+                lsum += t.y * w;
+            }
+            const float4* po = reinterpret_cast<const float4*>(part_o + (base + s0) * kHeadDim) + lane;
+            int i = 0;
+            for (; i + 8 <= cnt; i += 8) {
+                float4 v[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r) v[r] = __ldcg(po + (int64_t)(i + r) * (kHeadDim / 4));
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const float wr = __shfl_sync(kFullMask, w, i + r);
+                    acc.x += wr * v[r].x;
+                    acc.y += wr * v[r].y;
+                    acc.z += wr * v[r].z;
+                    acc.w += wr * v[r].w;
+                }
+            }
+            for (; i < cnt; ++i) {
+                const float4 v = __ldcg(po + (int64_t)i * (kHeadDim / 4));
+                const float wr = __shfl_sync(kFullMask, w, i);
+                acc.x += wr * v.x;
+                acc.y += wr * v.y;
+                acc.z += wr * v.z;
+                acc.w += wr * v.w;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, o);
+        const float inv = 1.0f / lsum;
+        reinterpret_cast<float4*>(out + (qrow0 + h) * kHeadDim)[lane] =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    if (tid == 0) counters[u] = 0u;
+}
+
 template <int G>
 __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
@@ -396,8 +465,6 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     extern __shared__ __align__(128) char smem[];
     __shared__ __align__(8) uint64_t bar[kWWarps][kWStages];
     __shared__ float xm[kWWarps][8], xl[kWWarps][8];
-    __shared__ float red[kWWarps][G];
-    __shared__ float wsm[kWThreads];
     __shared__ uint32_t s_last;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -599,7 +666,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
             }
         }
     }
-    merge_unit<G, kWThreads>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
+    merge_unit_warps<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, s_last);
 }
 
 template <int G>
