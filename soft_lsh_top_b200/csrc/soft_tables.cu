@@ -64,6 +64,16 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     pdl_wait();
     pdl_launch_dependents();
 
+    // The unit's G query rows in 16-byte pieces (8 bf16 or 4 fp32 each), one
+    // load per thread, issued before the hyperplane loads.
+    constexpr int kPer16 = 16 / (int)sizeof(QT);             // elements per piece
+    const int npieces = G * kHeadDim / kPer16;               // <= 512 for G <= 16
+    const uint4* qu4 = reinterpret_cast<const uint4*>(q + (b * Hq + kvh * G) * kHeadDim);
+    uint4 qv[(kMaxGroup * kHeadDim / kPer16 + kThreads - 1) / kThreads];
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(qv) / sizeof(qv[0])); ++i)
+        if (tid + i * kThreads < npieces) qv[i] = __ldg(qu4 + tid + i * kThreads);
+
     const int rows = G * nt * P;
     const int half = tid & 1;
     int r = tid >> 1;
@@ -76,10 +86,23 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     };
     if (r < rows) load_w(r);
 
-    const QT* qu = q + (b * Hq + kvh * G) * kHeadDim;
-    for (int e = tid; e < G * kHeadDim; e += kThreads) {
-        if constexpr (sizeof(QT) == 2) qd[e / kHeadDim][e % kHeadDim] = (double)bf16_to_f32(qu[e]);
-        else qd[e / kHeadDim][e % kHeadDim] = (double)qu[e];
+#pragma unroll
+    for (int i = 0; i < (int)(sizeof(qv) / sizeof(qv[0])); ++i) {
+        const int piece = tid + i * kThreads;
+        if (piece < npieces) {
+            double* dst = &qd[0][0] + piece * kPer16;  // qd rows are contiguous
+            const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if constexpr (sizeof(QT) == 2) {
+                    const float2 f = bf16x2_to_f32x2(w4[e]);
+                    dst[2 * e] = (double)f.x;
+                    dst[2 * e + 1] = (double)f.y;
+                } else {
+                    dst[e] = (double)__uint_as_float(w4[e]);
+                }
+            }
+        }
     }
     __syncthreads();
     for (int h = warp; h < G; h += kThreads / 32) {

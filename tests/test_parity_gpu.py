@@ -32,6 +32,11 @@ SMALL = {
     "bf16_single_head": wl.Workload(name="g1", B=2, Hq=2, Hkv=2, N=4099, L=8, P=8, tau=0.3, k=200, seed=7005),
     "bf16_group8_p7": wl.Workload(name="g8", B=1, Hq=16, Hkv=2, N=5000, L=10, P=7, tau=0.5, k=300, seed=7006),
     "bf16_group16": wl.Workload(name="g16", B=1, Hq=16, Hkv=1, N=3000, L=6, P=8, tau=0.4, k=129, seed=7007),
+    # more than 64 tables: the scoring runs in two launches that pass partial
+    # sums through the score buffer (three and four 32-table blocks).
+    "bf16_l80_p7": wl.Workload(name="l80", B=1, Hq=4, Hkv=2, N=2500, L=80, P=7, tau=0.4, k=150, seed=7008),
+    "f32_l128_group2": wl.Workload(name="l128", B=1, Hq=4, Hkv=2, N=1800, L=128, P=5, tau=0.6, k=90, dtype="f32",
+                                   seed=7009),
 }
 
 
@@ -100,6 +105,21 @@ def test_all_ties_select_lowest_indices():
     torch.testing.assert_close(out, torch.ones_like(out), atol=1e-6, rtol=0)
 
 
+def test_all_ties_candidate_path():
+    """All scores equal with the unit's keys within the candidate capacity:
+    the threshold bin holds every key and the ties are ranked by index."""
+    w = wl.Workload(name="ties_small", B=1, Hq=4, Hkv=2, N=3000, L=5, P=8, tau=0.3, k=333, seed=7010)
+    inp = wl.make_inputs(w, DEV)
+    inp["q"].zero_()
+    inp["V"].fill_(1.0)
+    ids, vnorm = gpu_hash(inp, w)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    want = torch.arange(w.k, dtype=torch.int32, device=DEV)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            assert torch.equal(idx[b, h], want)
+
+
 def test_decode_is_deterministic():
     w = SMALL["ragged_multitile"]
     inp = wl.make_inputs(w, DEV)
@@ -125,6 +145,16 @@ def _full_size(w, sample_units):
     g_vn = torch.stack([vnorm[u // w.Hkv, u % w.Hkv] for u in sample_units]).cpu().numpy()
     check_hash(g_ids, g_vn, orc_ids, orc_vn, margin, 0, w.N)
     return inp, ids, vnorm, orc_ids, orc_vn.astype(np.float32)
+
+
+def test_topk_slices_above_bitmap_capacity():
+    """N above 16 x 65536: each top-k CTA's slice exceeds the bitmap, so the
+    selection is written by the compaction pass over the scores."""
+    w = wl.Workload(name="wide", B=1, Hq=4, Hkv=1, N=1_100_000, L=8, P=6, tau=0.5, k=512, seed=7011)
+    inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, [0])
+    substitute_units(ids, vnorm, w, [0], orc_ids, orc_vn32)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    check_decode(inp, w, orc_ids, orc_vn32, [0], idx, out, sc)
 
 
 def test_batch8_128k_sampled_units_and_needles():
