@@ -150,12 +150,20 @@ class ClockSampler:
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world: int, steps: int, ms_max: float) -> float:
+    """Steps per second of the whole job: every rank ran `steps` steps of its
+    own data (weak scaling), and the job took the slowest rank's time."""
+    return world * steps / (ms_max * 1e-3)
 
 
 def barrier(world: int):
@@ -361,7 +369,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
                                                             "soft_lsh_top_b200/csrc/common.cuh"])
         result = {
-            "metric": METRIC, "value": world * K / (ms_total * 1e-3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "metric": METRIC, "value": whole_job_rate(world, K, ms_total), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "L": w.L,
@@ -378,7 +386,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                          "attention_gbs": attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9},
             "gpu_launches": nk * K,
             "clocks": clocks.summary(),
-            "e2e": {"value": world * K / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": whole_job_rate(world, K, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }
         if world == 1 and not args.no_cpu_baseline:
