@@ -501,6 +501,9 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         fence_mbarrier_init();
     }
     __syncthreads();
+    // The grid fits in one wave, so the next decode's first kernel may be
+    // placed now; it waits for this grid to finish before it reads anything.
+    pdl_launch_dependents();
     pdl_wait();  // the selected indices come from the previous kernel on the stream
 
     // Row index of this lane's row (lane % 16) of chunk j, or -1 past the end.

@@ -324,6 +324,9 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const float* __restri
     const int lo = (int)min64((int64_t)rank * R, N), hi = (int)min64((int64_t)lo + R, N);
     const int n = hi - lo;
 
+    // The grid fits in one wave, so the attention kernel's CTAs may be placed
+    // now; they wait for this grid to finish before they read anything.
+    pdl_launch_dependents();
     pdl_wait();  // scores, maxima and histograms come from the previous kernel on the stream
 
     // ---- the unit histogram: bin d0 of the k-th largest score.
