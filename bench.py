@@ -56,6 +56,15 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback 6650 GB/s (earlier measurement on this pool)"
 
 
+def tensor_peak() -> float:
+    """Measured dense bf16 TFLOP/s (burst) of MEASURED_PEAKS.json, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
+
+
 def profiled_traffic(kernel: str, workload: str, src_files):
     """DRAM bytes per launch from a committed ncu summary, if the kernel source
     is unchanged since the counters were taken; else None."""
@@ -179,15 +188,18 @@ def barrier(world: int):
 def oracle_decode_timing(w, K, V, q, W, units_kvh, min_seconds=2.0, reps_max=50):
     """Hash the sampled units with the oracle (untimed), then time the oracle
     decode of those units (OpenMP across units).  K, V: [Hkv, Ncap, d] CPU
-    tensors of one batch row; q: [Hq, d].  Returns (seconds per rep, units, threads)."""
+    tensors of one batch row; q: [Hq, d].  Returns (seconds per rep, units,
+    threads, seconds to hash the units)."""
     import oracle
     S = len(units_kvh)
     ids = np.zeros((S, w.L, w.ncap), dtype=np.uint8)
     vn = np.zeros((S, w.ncap), dtype=np.float32)
+    th = time.perf_counter()
     for i, h in enumerate(units_kvh):
         a, v, _ = oracle.hash_keys(K[h, : w.N], V[h, : w.N], W, w.L, w.P)
         ids[i, :, : w.N] = a
         vn[i, : w.N] = v.astype(np.float32)
+    hash_s = time.perf_counter() - th
     qs = torch.stack([q[h * w.G:(h + 1) * w.G] for h in units_kvh])
     Ks = torch.stack([K[h] for h in units_kvh])
     Vs = torch.stack([V[h] for h in units_kvh])
@@ -200,16 +212,17 @@ def oracle_decode_timing(w, K, V, q, W, units_kvh, min_seconds=2.0, reps_max=50)
         el = time.perf_counter() - t0
         if el >= min_seconds or reps >= reps_max:
             break
-    return el / reps, S, threads
+    return el / reps, S, threads, hash_s
 
 
 def cpu_baseline(w, inp):
     units = list(range(min(w.Hkv, 8)))
     K = inp["K"][0].cpu()
     V = inp["V"][0].cpu()
-    t, S, threads = oracle_decode_timing(w, K, V, inp["q"][0].cpu(), inp["W"].cpu(), units)
+    t, S, threads, hash_s = oracle_decode_timing(w, K, V, inp["q"][0].cpu(), inp["W"].cpu(), units)
     value = 1.0 / (t * w.U / S)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "hash_keys_per_s": S * w.N / hash_s,
             "sample": f"{S} of {w.U} (batch, kv-head) units at full N={w.N}, oracle decode (soft tables, scores, "
                       f"top-k, attention) in fp64, {t * 1e3:.1f} ms per sample; steps/s scaled by {w.U}/{S}"}
 
@@ -333,6 +346,21 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                for i, n in enumerate(names)}
     assert sk.read_device_error(ws) == 0
 
+    # ---- prefill: hashing a whole layer (socket_hash_keys), for the hash
+    # kernel's roofline.  Not part of the decode step.
+    inp0, ids0, vn0 = layers[0]
+    for _ in range(2):
+        sk.socket_hash_keys(inp0["K"], inp0["V"], inp0["W"], ids0, vn0, 0, w.N)
+    torch.cuda.synchronize()
+    RH = 5
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record()
+    for _ in range(RH):
+        sk.socket_hash_keys(inp0["K"], inp0["V"], inp0["W"], ids0, vn0, 0, w.N)
+    h1.record()
+    torch.cuda.synchronize()
+    hash_ms = max_over_ranks(h0.elapsed_time(h1) / RH, world)
+
     # ---- end to end through the public API with host buffers.
     q_host = [torch.empty_like(l[0]["q"], device="cpu").pin_memory() for l in layers]
     for l, qh in zip(layers, q_host):
@@ -366,6 +394,21 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         score_bytes = w.U * w.N * (w.L + 4)
         score_gbs = score_bytes / (kern_ms["score"] * 1e-3) / 1e9
         attn_bytes = w.U * 2 * w.k * w.d * w.elem_bytes
+        keys = w.U * w.N
+        hash_bytes = keys * (2 * w.d * w.elem_bytes + sk.socket_ids_row_bytes(w.L) + 4)
+        hash_flops = 2.0 * keys * w.d * w.L * w.P
+        bf16_peak = tensor_peak()
+        hash_gbs = hash_bytes / (hash_ms * 1e-3) / 1e9
+        hash_tflops = hash_flops / (hash_ms * 1e-3) / 1e12
+        prefill = {
+            "what": "socket_hash_keys over the whole layer (all units, N keys each); not in the decode step",
+            "kernel": "hash_mma_kernel" if w.dtype == "bf16" else "hash_kernel",
+            "keys": keys, "ms": hash_ms, "keys_per_s": world * keys / (hash_ms * 1e-3),
+            "algorithmic_bytes": hash_bytes, "gbs": hash_gbs, "hbm_frac": hash_gbs / peak,
+            "flops": hash_flops, "tflops": hash_tflops,
+            "tensor_frac": hash_tflops / bf16_peak if w.dtype == "bf16" else None,
+            "bound": "hbm" if hash_bytes / (peak * 1e9) >= hash_flops / (bf16_peak * 1e12) else "tensor",
+        }
         traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
                                                             "soft_lsh_top_b200/csrc/common.cuh"])
         result = {
@@ -386,6 +429,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                          "attention_gbs": attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9},
             "gpu_launches": nk * K,
             "clocks": clocks.summary(),
+            "prefill": prefill,
             "e2e": {"value": whole_job_rate(world, K, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }
