@@ -310,6 +310,26 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         step(s)
     torch.cuda.synchronize()
 
+    # One CUDA graph holds R consecutive decode steps, one per layer, so the
+    # kernels chain by programmatic dependent launch across steps as well
+    # (graph edges); the timed loop replays it K // R times and runs the
+    # K % R remaining steps as direct calls.
+    graph, launch = None, "direct C-ABI calls, one stream"
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for li in range(R):
+                    step(li)
+            for _ in range(max(1, args.warmup // R)):
+                graph.replay()
+            torch.cuda.synchronize()
+            assert sk.read_device_error(ws) == 0
+            launch = f"CUDA graph replay ({R} decode steps per graph, one per layer)"
+        except Exception as exc:  # capture unsupported here: time direct calls
+            graph = None
+            launch = f"direct C-ABI calls, one stream (graph capture failed: {type(exc).__name__})"
+
     # ---- timed region: K steps back to back (kernels chain by programmatic
     # dependent launch; nothing is recorded between them).
     K = args.steps
@@ -318,10 +338,17 @@ def run_socket(args, world: int, rank: int, local_rank: int):
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
         start.record()
-        for s in range(K):
-            step(s)
+        if graph is not None:
+            for _ in range(K // R):
+                graph.replay()
+            for s in range(K % R):
+                step(s)
+        else:
+            for s in range(K):
+                step(s)
         end.record()
         torch.cuda.synchronize()
+    graph = None
     barrier(world)
     ms_total = max_over_ranks(start.elapsed_time(end), world)
     assert sk.read_device_error(ws) == 0
@@ -418,7 +445,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "L": w.L,
                        "P": w.P, "tau": w.tau, "k": w.k, "kv_dtype": w.dtype, "parallelism": f"replicas{world}",
                        "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB per step, {R} rotating layers "
-                             "of independent data", "launch": "direct C-ABI calls, one stream"},
+                             "of independent data", "launch": launch},
             "bytes_per_step": bytes_step,
             "step_hbm_gbs": bytes_step / (ms_step * 1e-3) / 1e9,
             "step_roofline_frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak,
@@ -453,6 +480,7 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=3, help="independently drawn layers rotated across steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
+    ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA graph replay")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

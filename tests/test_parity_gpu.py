@@ -120,6 +120,30 @@ def test_all_ties_candidate_path():
             assert torch.equal(idx[b, h], want)
 
 
+def test_decode_in_a_cuda_graph_matches_direct_calls():
+    """A decode captured in a CUDA graph (the kernels' dependent launches become
+    graph edges) reproduces a direct call bit for bit."""
+    w = SMALL["llama_32k"]
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)
+    ws, idx, out = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, DEV)
+    run = lambda: sk.socket_decode(inp["q"], inp["W"], ids, vnorm, inp["K"], inp["V"], w.N, w.tau, w.k, ws, idx, out)
+    run()
+    torch.cuda.synchronize()
+    want_idx, want_out = idx.clone(), out.clone()
+    idx.fill_(-1)
+    out.fill_(float("nan"))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert sk.read_device_error(ws) == 0
+    assert torch.equal(idx, want_idx)
+    assert torch.equal(out.view(torch.int32), want_out.view(torch.int32))
+
+
 def test_decode_is_deterministic():
     w = SMALL["ragged_multitile"]
     inp = wl.make_inputs(w, DEV)
