@@ -137,7 +137,10 @@ size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t 
  *   ids, vnorm device, as written by socket_hash_keys.
  *   K, V       device, [B][Hkv][Ncap][d] of kv_dtype, 16-byte aligned.
  *   N          live keys per unit (the same for every unit), k <= N <= Ncap.
- *   tau        temperature, finite and > 0.
+ *   tau        temperature, finite and >= 0.  tau = 0 is hard LSH: each
+ *              query is hashed like a key (bit p = [<W_{l,p}, q> > 0]) and
+ *              p_{h,l} is 1 on that bucket and 0 elsewhere, so a key's score
+ *              is vnorm times its collision count over tables and heads.
  *   workspace  device scratch of >= socket_decode_workspace_size() bytes,
  *              256-byte aligned.
  *   idx_out    device out, [B][Hkv][k] int32, ascending per unit.

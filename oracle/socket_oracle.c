@@ -127,6 +127,11 @@ void oracle_hash(const void* K, const void* V, int kv_dtype, int64_t n, int d,
  *   logit(b) = sum_p s_{b,p} z_{l,p} / tau,  s_{b,p} = +1 if bit p of b else -1
  *   p_l(b)   = exp(logit(b) - max) / sum_b' exp(logit(b') - max)
  *
+ * tau = 0 is hard LSH ([ES] "Enunciado del Problema" / "Fundamento Teórico",
+ * the hard-hash collision count the soft score generalises): the query is
+ * hashed like a key, bit p = [<W_{l,p}, q> > 0], and all mass sits on that
+ * bucket, so the score counts the tables where key and query collide.
+ *
  * q: d stored elements (dtype q_dtype).  prob: [L][2^P].
  */
 void oracle_soft_assign(const void* q, int q_dtype, int d,
@@ -140,6 +145,19 @@ void oracle_soft_assign(const void* q, int q_dtype, int d,
     }
     double qnorm = sqrt(qq);
     double z[8];
+    if (tau == 0.0) {
+        for (int l = 0; l < L; ++l) {
+            int hb = 0;
+            for (int p = 0; p < P; ++p) {
+                const double* w = W + ((int64_t)l * P + p) * d;
+                double y = 0.0;
+                for (int j = 0; j < d; ++j) y += w[j] * load_elem(q, q_dtype, j);
+                if (y > 0.0) hb |= 1 << p;
+            }
+            for (int b = 0; b < nb; ++b) prob[(int64_t)l * nb + b] = b == hb ? 1.0 : 0.0;
+        }
+        return;
+    }
     double* logit = (double*)malloc(sizeof(double) * nb);
     for (int l = 0; l < L; ++l) {
         for (int p = 0; p < P; ++p) {

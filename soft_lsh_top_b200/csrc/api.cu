@@ -199,7 +199,7 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
     if (st != SOCKET_OK) return st;
     if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype))
         return fail(SOCKET_EINVAL, "q_dtype=%d / kv_dtype=%d unknown", q_dtype, kv_dtype);
-    if (!(tau > 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and > 0", tau);
+    if (!(tau >= 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and >= 0", tau);
     if (!q || !W || !ids || !vnorm || !K || !V || !idx_out || !out || !workspace)
         return fail(SOCKET_EINVAL, "null pointer argument");
     if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(K, 16) ||

@@ -135,10 +135,16 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         y += __shfl_xor_sync(kFullMask, y, 1);
         if (live && half == 0) {
             const int lt = (r / P) % nt, p = r % P;
-            const double z = qnorm[h] > 0.0 ? y / qnorm[h] : 0.0;
-            const double x = 2.0 * z / tau;
-            sig[h][lt][p][1] = 1.0 / (1.0 + exp(-x));  // sign +1: bit set
-            sig[h][lt][p][0] = 1.0 / (1.0 + exp(x));   // sign -1: bit clear
+            if (tau == 0.0) {
+                // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
+                sig[h][lt][p][1] = y > 0.0 ? 1.0 : 0.0;
+                sig[h][lt][p][0] = y > 0.0 ? 0.0 : 1.0;
+            } else {
+                const double z = qnorm[h] > 0.0 ? y / qnorm[h] : 0.0;
+                const double x = 2.0 * z / tau;
+                sig[h][lt][p][1] = 1.0 / (1.0 + exp(-x));  // sign +1: bit set
+                sig[h][lt][p][0] = 1.0 / (1.0 + exp(x));   // sign -1: bit clear
+            }
         }
         if (r + kThreads / 2 < rows) load_w(r + kThreads / 2);
     }

@@ -245,6 +245,29 @@ def pin_score_hard_collision_count(lib):
     assert count.max() >= 1
 
 
+def pin_hard_mode_is_collision_count(lib):
+    """tau = 0, hard LSH ([ES] "Enunciado del Problema": binary collision
+    signals; [DE] "Der alte Weg (Harte LSH)"): each head's query is hashed like
+    a key, p is one-hot on that bucket, and the score is ||v|| times the number
+    of (head, table) pairs where key and query collide -- counted here by brute
+    force from the hash of the keys and of the queries."""
+    rng = np.random.default_rng(19)
+    L, P, d, n, G = 7, 5, 16, 300, 3
+    W, q, K, V = _unit_case(rng, G, n, d, L, P)
+    ids, vn, _ = oracle.hash_keys(K, V, W, L, P, lib=lib)
+    vn32 = vn.astype(np.float32)
+    qids = oracle.hash_keys(q, q, W, L, P, lib=lib)[0]            # [L, G]
+    for h in range(G):
+        prob = oracle.soft_assign(q[h], W, L, P, 0.0, lib=lib)
+        want = np.zeros_like(prob)
+        want[np.arange(L), qids[:, h]] = 1.0
+        assert np.array_equal(prob, want)
+    count = sum(np.sum(ids == qids[:, h][:, None], axis=0) for h in range(G))
+    _, _, sc, _ = oracle.decode_unit(q, W, L, P, 0.0, ids, vn32, K, V, n, 5, lib=lib)
+    assert np.array_equal(sc, vn32.astype(np.float64) * count)
+    assert count.max() >= 1
+
+
 def pin_score_heads_add(lib):
     """Grouped heads share one selection and their scores add: the score of a
     2-head group equals the sum of each head's score alone."""

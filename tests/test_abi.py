@@ -77,7 +77,6 @@ def decode(lib, **kw):
     (dict(N=80), EINVAL),
     (dict(Ncap=70, N=64), EINVAL),
     (dict(Ncap=48, N=48), EINVAL),
-    (dict(tau=0.0), EINVAL),
     (dict(tau=-1.0), EINVAL),
     (dict(tau=float("nan")), EINVAL),
     (dict(tau=float("inf")), EINVAL),

@@ -72,7 +72,7 @@ def test_decode_matches_oracle(small):
     _decode_on_oracle_index(small)
 
 
-@pytest.mark.parametrize("variant", ["k1", "k_eq_n", "tau_0.01", "tau_5", "n_not_ncap"])
+@pytest.mark.parametrize("variant", ["k1", "k_eq_n", "tau_0.01", "tau_5", "tau_0_hard", "n_not_ncap"])
 def test_decode_edge_cases(small, variant):
     w = small[0]
     if variant == "k1":
@@ -83,6 +83,8 @@ def test_decode_edge_cases(small, variant):
         _decode_on_oracle_index(small, tau=0.01)
     elif variant == "tau_5":
         _decode_on_oracle_index(small, tau=5.0)
+    elif variant == "tau_0_hard":
+        _decode_on_oracle_index(small, tau=0.0)
     else:
         n = w.N - 13
         _decode_on_oracle_index(small, N=n, k=min(w.k, n))
