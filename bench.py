@@ -388,6 +388,44 @@ def run_socket(args, world: int, rank: int, local_rank: int):
     torch.cuda.synchronize()
     hash_ms = max_over_ranks(h0.elapsed_time(h1) / RH, world)
 
+    # ---- one selection per query head (socket_decode_per_head) on the same
+    # layers: direct calls, then a pass with events between the kernels.
+    ws_h, idx_h, out_h = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, dev, per_head=True)
+
+    def step_h(s):
+        inp, ids, vn = layers[s % R]
+        sk.socket_decode_per_head(inp["q"], inp["W"], ids, vn, inp["K"], inp["V"], w.N, w.tau, w.k,
+                                  ws_h, idx_h, out_h)
+
+    for s in range(args.warmup):
+        step_h(s)
+    torch.cuda.synchronize()
+    KH = min(K, 100)
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    p0.record()
+    for s in range(KH):
+        step_h(s)
+    p1.record()
+    torch.cuda.synchronize()
+    ph_ms = max_over_ranks(p0.elapsed_time(p1), world)
+    KHD = min(KH, 50)
+    evs_h = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(KHD)]
+    for row in evs_h:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    for s in range(KHD):
+        sk.socket_set_step_events(evs_h[s])
+        step_h(s)
+    torch.cuda.synchronize()
+    sk.socket_set_step_events([])
+    ph_kern = {n: statistics.fmean(evs_h[s][i].elapsed_time(evs_h[s][i + 1]) for s in range(KHD))
+               for i, n in enumerate(names)}
+    assert sk.read_device_error(ws_h) == 0
+    del ws_h, idx_h, out_h, evs_h
+    torch.cuda.empty_cache()
+
     # ---- end to end through the public API with host buffers.
     q_host = [torch.empty_like(l[0]["q"], device="cpu").pin_memory() for l in layers]
     for l, qh in zip(layers, q_host):
@@ -436,6 +474,18 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "tensor_frac": hash_tflops / bf16_peak if w.dtype == "bf16" else None,
             "bound": "hbm" if hash_bytes / (peak * 1e9) >= hash_flops / (bf16_peak * 1e12) else "tensor",
         }
+        # Per-head scoring reads each kv unit's ids and norms once (its heads'
+        # CTAs stream them side by side) and writes a score row per head.
+        ph_score_bytes = w.U * w.N * (w.L + 4) + w.U * w.G * w.N * 4
+        ph_score_gbs = ph_score_bytes / (ph_kern["score"] * 1e-3) / 1e9
+        per_head = {
+            "what": "socket_decode_per_head: one selection per query head (B*Hq units) on the same layers; "
+                    "direct calls",
+            "steps_per_s": whole_job_rate(world, KH, ph_ms), "ms_per_step": ph_ms / KH, "steps": KH,
+            "kernels_ms": ph_kern,
+            "score": {"algorithmic_bytes": ph_score_bytes, "gbs": ph_score_gbs, "frac": ph_score_gbs / peak},
+            "attention_gbs": w.U * w.G * 2 * w.k * w.d * w.elem_bytes / (ph_kern["attention"] * 1e-3) / 1e9,
+        }
         traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
                                                             "soft_lsh_top_b200/csrc/common.cuh"])
         result = {
@@ -457,6 +507,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "gpu_launches": nk * K,
             "clocks": clocks.summary(),
             "prefill": prefill,
+            "per_head": per_head,
             "e2e": {"value": whole_job_rate(world, K, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }

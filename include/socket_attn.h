@@ -161,6 +161,36 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W,
                   int32_t* idx_out, float* out, float* scores_out, void* stream);
 
 /*
+ * socket_decode_per_head_workspace_size / socket_decode_per_head -- the same
+ * step with one selection per query head instead of one per kv head: every
+ * query is scored and selects on its own, as the pages state the method for
+ * a single query ([ES] "Mecanismo Central: LSH Suave" steps 2-4: each new
+ * query induces its own bucket distribution, its own scores and its own
+ * top-k).  For query head h of batch row b, with kv head h / (Hq / Hkv):
+ *     score_{b,h}(n) = vnorm(n) * sum_l p_{h,l}(id_l(n))
+ * then top-k and exact attention of head h over its own k keys.  With
+ * Hq == Hkv this is socket_decode.
+ *
+ *   Arguments as for socket_decode, except:
+ *   idx_out    device out, [B][Hq][k] int32, ascending per query head.
+ *   scores_out device out or NULL, [B][Hq][Ncap] float32, 16-byte aligned.
+ *   workspace  >= socket_decode_per_head_workspace_size() bytes.
+ * Preconditions: those of socket_decode, and B * Hq <= 65535.
+ * The Hq / Hkv heads of a kv head read its ids and norms from HBM about once
+ * (their scoring runs side by side); the lookups, the selections and the
+ * gathers are per head.
+ */
+size_t socket_decode_per_head_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
+                                             int64_t d, int L, int P, int k);
+int socket_decode_per_head(const void* q, int q_dtype, const uint16_t* W,
+                           const uint8_t* ids, const float* vnorm,
+                           const void* K, const void* V, int kv_dtype,
+                           int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d,
+                           int L, int P, double tau, int k,
+                           void* workspace, size_t workspace_bytes,
+                           int32_t* idx_out, float* out, float* scores_out, void* stream);
+
+/*
  * socket_decode_static -- socket_decode for callers that cannot allocate
  * device memory.  The paper has no counterpart: this is a packaging variant
  * of socket_decode, same arguments minus the workspace, same results.

@@ -266,3 +266,24 @@ def decode(q, W, L: int, P: int, tau: float, ids, vnorm_f32, K, V, n: int, k: in
                       ncap, n, _ptr(Ks), _ptr(Vs), kdt, int(k), _ptr(idx), _ptr(out),
                       _ptr(sc) if sc is not None else None)
     return idx, out, sc
+
+
+def decode_per_head(q, W, L: int, P: int, tau: float, ids, vnorm_f32, K, V, n: int, k: int,
+                    want_scores: bool = True, lib=None):
+    """Steps 2-4 with one selection per query head: the method as the pages
+    state it for a single query ([ES] "Mecanismo Central: LSH Suave" steps
+    2-4 -- each new query induces its own bucket distribution, scores and
+    top-k).  Head g of unit u is run as a unit of its own, with the one query
+    row q[u, g] over u's ids, norms, keys and values; no arithmetic is added.
+
+    q: [U, G, d]; ids: [U, L, ncap]; vnorm_f32: [U, ncap]; K, V: [U, ncap, d].
+    Returns (idx [U, G, k], out [U, G, d], scores [U, G, n] or None).
+    """
+    qs, _ = _stored(q)
+    Ks, _ = _stored(K)
+    Vs, _ = _stored(V)
+    U, G, d = qs.shape
+    rep = lambda a: np.repeat(np.asarray(a), G, axis=0)  # unit u -> units u G .. u G + G - 1
+    idx, out, sc = decode(qs.reshape(U * G, 1, d), W, L, P, tau, rep(ids), rep(vnorm_f32), rep(Ks), rep(Vs),
+                          n, k, want_scores=want_scores, lib=lib)
+    return idx.reshape(U, G, k), out.reshape(U, G, d), (sc.reshape(U, G, n) if sc is not None else None)

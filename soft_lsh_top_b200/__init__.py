@@ -20,6 +20,7 @@ import torch
 
 __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
+    "socket_decode_per_head", "socket_decode_per_head_workspace_size",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -65,6 +66,10 @@ def load_library(path: str | None = None):
     lib.socket_decode.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64,
                                   _int, _int, _dbl, _int, _vp, _sz, _vp, _vp, _vp, _vp]
     lib.socket_decode.restype = _int
+    lib.socket_decode_per_head_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]
+    lib.socket_decode_per_head_workspace_size.restype = _sz
+    lib.socket_decode_per_head.argtypes = lib.socket_decode.argtypes
+    lib.socket_decode_per_head.restype = _int
     lib.socket_decode_static.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
                                          _i64, _int, _int, _dbl, _int, _vp, _vp, _vp, _vp]
     lib.socket_decode_static.restype = _int
@@ -172,11 +177,49 @@ def socket_decode_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, d: int, L
     return n
 
 
+def socket_decode_per_head_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, d: int, L: int, P: int,
+                                          k: int) -> int:
+    n = int(load_library().socket_decode_per_head_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k))
+    if n == 0:
+        raise ValueError("invalid sizes for socket_decode_per_head")
+    return n
+
+
+def _decode(per_head: bool, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream):
+    lib = load_library()
+    B, Hq, d = q.shape
+    _, Hkv, Ncap, _ = K.shape
+    L, P, _ = W.shape
+    dev = q.device
+    sel = Hq if per_head else Hkv  # selections per batch row
+    _check(q, "q", (B, Hq, d), device=dev)
+    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
+    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
+    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
+    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
+    _check(idx_out, "idx_out", (B, sel, k), dtype=torch.int32, device=dev)
+    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1 or not workspace.is_cuda or workspace.device != dev:
+        raise ValueError("workspace must be a 1-D uint8 CUDA tensor on the inputs' device")
+    if scores_out is not None:
+        _check(scores_out, "scores_out", (B, sel, Ncap), dtype=torch.float32, device=dev)
+    fn = lib.socket_decode_per_head if per_head else lib.socket_decode
+    with torch.cuda.device(dev):
+        _raise(fn(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(),
+                  K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P,
+                  float(tau), int(k), workspace.data_ptr(), workspace.numel(),
+                  idx_out.data_ptr(), out.data_ptr(),
+                  scores_out.data_ptr() if scores_out is not None else None,
+                  _stream_handle(stream)))
+
+
 def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
                   K: torch.Tensor, V: torch.Tensor, N: int, tau: float, k: int,
                   workspace: torch.Tensor, idx_out: torch.Tensor, out: torch.Tensor,
                   scores_out: torch.Tensor | None = None, stream=None) -> None:
-    """One decode step (soft assignment, scoring, top-k, sparse attention).
+    """One decode step (soft assignment, scoring, top-k, sparse attention),
+    one selection per kv head.
 
     q: [B, Hq, 128]; W: [L, P, 128] bfloat16; ids: [B, Hkv, Ncap/32, Lr/16, 32, 16] uint8, Lr = socket_ids_row_bytes(L) (see the header);
     vnorm: [B, Hkv, Ncap] float32; K, V: [B, Hkv, Ncap, 128];
@@ -184,30 +227,17 @@ def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: to
     idx_out: [B, Hkv, k] int32; out: [B, Hq, 128] float32;
     scores_out: optional [B, Hkv, Ncap] float32.
     """
-    lib = load_library()
-    B, Hq, d = q.shape
-    _, Hkv, Ncap, _ = K.shape
-    L, P, _ = W.shape
-    dev = q.device
-    _check(q, "q", (B, Hq, d), device=dev)
-    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
-    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
-    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
-    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
-    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
-    _check(idx_out, "idx_out", (B, Hkv, k), dtype=torch.int32, device=dev)
-    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
-    if workspace.dtype != torch.uint8 or workspace.dim() != 1 or not workspace.is_cuda or workspace.device != dev:
-        raise ValueError("workspace must be a 1-D uint8 CUDA tensor on the inputs' device")
-    if scores_out is not None:
-        _check(scores_out, "scores_out", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
-    with torch.cuda.device(dev):
-        _raise(lib.socket_decode(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(),
-                                 K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P,
-                                 float(tau), int(k), workspace.data_ptr(), workspace.numel(),
-                                 idx_out.data_ptr(), out.data_ptr(),
-                                 scores_out.data_ptr() if scores_out is not None else None,
-                                 _stream_handle(stream)))
+    _decode(False, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream)
+
+
+def socket_decode_per_head(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
+                           K: torch.Tensor, V: torch.Tensor, N: int, tau: float, k: int,
+                           workspace: torch.Tensor, idx_out: torch.Tensor, out: torch.Tensor,
+                           scores_out: torch.Tensor | None = None, stream=None) -> None:
+    """socket_decode with one selection per query head: idx_out [B, Hq, k],
+    scores_out optional [B, Hq, Ncap], workspace of
+    >= socket_decode_per_head_workspace_size() bytes; the rest as socket_decode."""
+    _decode(True, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream)
 
 
 def socket_decode_static(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
@@ -262,11 +292,12 @@ def alloc_cache_index(B: int, Hkv: int, Ncap: int, L: int, device) -> tuple[torc
     return ids, vnorm
 
 
-def alloc_decode_buffers(B: int, Hq: int, Hkv: int, Ncap: int, L: int, P: int, k: int, device):
-    """(workspace, idx_out, out) for socket_decode at these sizes."""
-    ws = torch.empty(socket_decode_workspace_size(B, Hq, Hkv, Ncap, HEAD_DIM, L, P, k), dtype=torch.uint8,
-                     device=device)
-    idx = torch.empty(B, Hkv, k, dtype=torch.int32, device=device)
+def alloc_decode_buffers(B: int, Hq: int, Hkv: int, Ncap: int, L: int, P: int, k: int, device,
+                         per_head: bool = False):
+    """(workspace, idx_out, out) for socket_decode (per_head: socket_decode_per_head) at these sizes."""
+    size = socket_decode_per_head_workspace_size if per_head else socket_decode_workspace_size
+    ws = torch.empty(size(B, Hq, Hkv, Ncap, HEAD_DIM, L, P, k), dtype=torch.uint8, device=device)
+    idx = torch.empty(B, Hq if per_head else Hkv, k, dtype=torch.int32, device=device)
     out = torch.empty(B, Hq, HEAD_DIM, dtype=torch.float32, device=device)
     return ws, idx, out
 

@@ -83,9 +83,38 @@ int fill_shape(DecodeShape& s, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap,
     s.k = k;
     s.G = (int)(Hq / Hkv);
     s.U = B * Hkv;
+    s.share = 1;
     s.NB = 1 << P;
     s.nsplit = 0;
     return SOCKET_OK;
+}
+
+// Every query head selects its own keys: each head is a unit of one query
+// row, and the Hq / Hkv units of a kv head read that head's ids, norms, keys
+// and values.
+void select_per_head(DecodeShape& s)
+{
+    s.share = s.G;
+    s.U = s.B * s.Hq;
+    s.G = 1;
+}
+
+size_t workspace_size(bool per_head, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P,
+                      int k)
+{
+    DecodeShape s;
+    const std::string saved = g_last_error;
+    // N = k is the smallest valid N; the layout does not depend on N.
+    if (fill_shape(s, B, Hq, Hkv, Ncap, k, d, L, P, k) != SOCKET_OK) {
+        g_last_error = saved;
+        return 0;
+    }
+    if (per_head) {
+        if (B * Hq > 65535) return 0;
+        select_per_head(s);
+    }
+    s.nsplit = (k + 15) / 16;  // attention splits never exceed ceil(k / 16)
+    return decode_workspace_layout(s).total;
 }
 
 }  // namespace
@@ -128,6 +157,65 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 8 * (size_t)s.U * s.G * s.nsplit);
     w.total = off;
     return w;
+}
+
+// One decode step; per_head: every query head selects its own keys.
+int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
+           const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N,
+           int64_t d, int L, int P, double tau, int k, void* workspace, size_t workspace_bytes, int32_t* idx_out,
+           float* out, float* scores_out, cudaStream_t cs)
+{
+    g_last_error.clear();
+    DecodeShape s;
+    int st = fill_shape(s, B, Hq, Hkv, Ncap, N, d, L, P, k);
+    if (st != SOCKET_OK) return st;
+    if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype))
+        return fail(SOCKET_EINVAL, "q_dtype=%d / kv_dtype=%d unknown", q_dtype, kv_dtype);
+    if (!(tau >= 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and >= 0", tau);
+    if (!q || !W || !ids || !vnorm || !K || !V || !idx_out || !out || !workspace)
+        return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(K, 16) ||
+        !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
+        return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
+    if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
+    if (per_head) {
+        if (B * Hq > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hq=%lld above 65535", (long long)(B * Hq));
+        select_per_head(s);
+    }
+    // Splits never exceed ceil(k / 16), the count the advertised size covers.
+    s.nsplit = attention_splits(kv_dtype, q_dtype, s.G, s.U, k, device_num_sms());
+    const size_t need = workspace_size(per_head, B, Hq, Hkv, Ncap, d, L, P, k);
+    if (workspace_bytes < need)
+        return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+
+    const DecodeWorkspace w = decode_workspace_layout(s);
+    char* base = static_cast<char*>(workspace);
+    uint32_t* err_word = reinterpret_cast<uint32_t*>(base + w.err);
+    uint32_t* counters = reinterpret_cast<uint32_t*>(base + w.counters);
+    float* tables = reinterpret_cast<float*>(base + w.tables);
+    float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
+    uint32_t* unit_max = reinterpret_cast<uint32_t*>(base + w.unit_max);
+    uint32_t* unit_hist = reinterpret_cast<uint32_t*>(base + w.unit_hist);
+    uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
+    uint2* cand = reinterpret_cast<uint2*>(base + w.cand);
+    float* part_o = reinterpret_cast<float*>(base + w.part_o);
+    float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
+
+    if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt, cs), "soft-table kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, err_word, cs), "score kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");
+    if (st != SOCKET_OK) return st;
+    if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
+    st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,
+                                      out, cs),
+                     "attention kernel launch");
+    if (st != SOCKET_OK) return st;
+    return cuda_status(mark_step(4, cs), "step event record");
 }
 
 }  // namespace socket_attn
@@ -177,15 +265,13 @@ int socket_ids_row_bytes(int L) { return (L >= 1 && L <= SOCKET_MAX_L) ? ids_row
 size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P,
                                     int k)
 {
-    DecodeShape s;
-    const std::string saved = g_last_error;
-    // N = k is the smallest valid N; the layout does not depend on N.
-    if (fill_shape(s, B, Hq, Hkv, Ncap, k, d, L, P, k) != SOCKET_OK) {
-        g_last_error = saved;
-        return 0;
-    }
-    s.nsplit = (k + 15) / 16;  // attention splits never exceed ceil(k / 16)
-    return decode_workspace_layout(s).total;
+    return workspace_size(false, B, Hq, Hkv, Ncap, d, L, P, k);
+}
+
+size_t socket_decode_per_head_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L,
+                                             int P, int k)
+{
+    return workspace_size(true, B, Hq, Hkv, Ncap, d, L, P, k);
 }
 
 int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
@@ -193,54 +279,17 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
                   int64_t N, int64_t d, int L, int P, double tau, int k, void* workspace, size_t workspace_bytes,
                   int32_t* idx_out, float* out, float* scores_out, void* stream)
 {
-    g_last_error.clear();
-    DecodeShape s;
-    int st = fill_shape(s, B, Hq, Hkv, Ncap, N, d, L, P, k);
-    if (st != SOCKET_OK) return st;
-    if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype))
-        return fail(SOCKET_EINVAL, "q_dtype=%d / kv_dtype=%d unknown", q_dtype, kv_dtype);
-    if (!(tau >= 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and >= 0", tau);
-    if (!q || !W || !ids || !vnorm || !K || !V || !idx_out || !out || !workspace)
-        return fail(SOCKET_EINVAL, "null pointer argument");
-    if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(K, 16) ||
-        !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
-        return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
-    if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
-    // Splits never exceed ceil(k / 16), the count the advertised size covers.
-    s.nsplit = attention_splits(kv_dtype, q_dtype, s.G, s.U, k, device_num_sms());
-    const size_t need = socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k);
-    if (workspace_bytes < need)
-        return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    return decode(false, q, q_dtype, W, ids, vnorm, K, V, kv_dtype, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, workspace,
+                  workspace_bytes, idx_out, out, scores_out, static_cast<cudaStream_t>(stream));
+}
 
-    const DecodeWorkspace w = decode_workspace_layout(s);
-    char* base = static_cast<char*>(workspace);
-    uint32_t* err_word = reinterpret_cast<uint32_t*>(base + w.err);
-    uint32_t* counters = reinterpret_cast<uint32_t*>(base + w.counters);
-    float* tables = reinterpret_cast<float*>(base + w.tables);
-    float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
-    uint32_t* unit_max = reinterpret_cast<uint32_t*>(base + w.unit_max);
-    uint32_t* unit_hist = reinterpret_cast<uint32_t*>(base + w.unit_hist);
-    uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
-    uint2* cand = reinterpret_cast<uint2*>(base + w.cand);
-    float* part_o = reinterpret_cast<float*>(base + w.part_o);
-    float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-
-    if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt, cs), "soft-table kernel launch");
-    if (st != SOCKET_OK) return st;
-    if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, err_word, cs), "score kernel launch");
-    if (st != SOCKET_OK) return st;
-    if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");
-    if (st != SOCKET_OK) return st;
-    if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,
-                                      out, cs),
-                     "attention kernel launch");
-    if (st != SOCKET_OK) return st;
-    return cuda_status(mark_step(4, cs), "step event record");
+int socket_decode_per_head(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
+                           const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hq, int64_t Hkv,
+                           int64_t Ncap, int64_t N, int64_t d, int L, int P, double tau, int k, void* workspace,
+                           size_t workspace_bytes, int32_t* idx_out, float* out, float* scores_out, void* stream)
+{
+    return decode(true, q, q_dtype, W, ids, vnorm, K, V, kv_dtype, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, workspace,
+                  workspace_bytes, idx_out, out, scores_out, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

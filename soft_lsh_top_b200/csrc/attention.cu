@@ -140,7 +140,7 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
 template <typename KT, int G>
 __global__ __launch_bounds__(kThreads) void attention_kernel(
     const void* __restrict__ q, int q_dtype, const KT* __restrict__ K, const KT* __restrict__ V,
-    const int32_t* __restrict__ idx, int64_t Hq, int64_t Hkv, int64_t Ncap, int k, int nsplit, int rpc,
+    const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
     uint32_t* __restrict__ err_word, float* __restrict__ out)
 {
@@ -160,12 +160,12 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t u = blockIdx.x / nsplit;
     const int split = blockIdx.x % nsplit;
-    const int64_t b = u / Hkv, kvh = u % Hkv;
+    const int64_t ukv = u / share;  // the unit's key/value rows
     const int r_begin = split * rpc;
     const int r_end = min(k, r_begin + rpc);
     const int nchunks = (r_end - r_begin + kChunk - 1) / kChunk;
 
-    const int64_t qrow0 = b * Hq + kvh * G;
+    const int64_t qrow0 = u * G;  // the unit's query rows of [B][Hq]
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
         const int64_t off = qrow0 * kHeadDim + e;
         qs[e / kHeadDim][e % kHeadDim] = q_dtype == 1 ? bf16_to_f32(static_cast<const uint16_t*>(q)[off])
@@ -194,7 +194,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
             // gather can never leave the unit's cache rows.
             int32_t r = __ldcg(idx + u * k + r0 + tid);
             r = (r >= 0 && r < Ncap) ? r : 0;
-            const int64_t row = u * Ncap + r;
+            const int64_t row = ukv * Ncap + r;
             bulk_copy_g2s(ks + tid * kRowBytes, K + row * kHeadDim, kRowBytes, &bar[st]);
             bulk_copy_g2s(vs + tid * kRowBytes, V + row * kHeadDim, kRowBytes, &bar[st]);
         }
@@ -438,7 +438,7 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
 template <int G>
 __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
-    const int32_t* __restrict__ idx, int64_t Hq, int64_t Hkv, int64_t Ncap, int k, int nsplit, int rpc,
+    const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
     uint32_t* __restrict__ err_word, float* __restrict__ out)
 {
@@ -451,12 +451,12 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t u = blockIdx.x / nsplit;
     const int split = blockIdx.x % nsplit;
-    const int64_t b = u / Hkv, kvh = u % Hkv;
+    const int64_t ukv = u / share;  // the unit's key/value rows
     const int r_begin = split * rpc;
     const int r_end = min(k, r_begin + rpc);
     const int nch = (r_end - r_begin + kWChunk - 1) / kWChunk;        // chunks of this CTA
     const int cw = nch > warp ? (nch - warp + kWWarps - 1) / kWWarps : 0;  // chunks of this warp
-    const int64_t qrow0 = b * Hq + kvh * G;
+    const int64_t qrow0 = u * G;  // the unit's query rows of [B][Hq]
     char* wsm_base = smem + warp * kWStages * kWStageBytes;
     const uint32_t wbase = smem_addr(wsm_base);
 
@@ -505,7 +505,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
             // Indices come from the top-k kernel and are < N; clamp anyway so a
             // gather can never leave the unit's cache rows.
             r = (r >= 0 && r < Ncap) ? r : 0;
-            const uint16_t* src = (lane < 16 ? K : V) + (u * Ncap + r) * kHeadDim;
+            const uint16_t* src = (lane < 16 ? K : V) + (ukv * Ncap + r) * kHeadDim;
             bulk_copy_g2s(dst, src, kHeadDim * 2, &bar[warp][st]);
         } else if (lane >= 16) {
             uint4* z = reinterpret_cast<uint4*>(dst);
@@ -664,7 +664,7 @@ cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                   idx, s.Hq, s.Hkv, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out);
+                   idx, s.share, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -680,7 +680,7 @@ cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, c
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream, q, q_dtype,
-                   static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.Hq, s.Hkv, s.Ncap, s.k, s.nsplit, rpc,
+                   static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.share, s.Ncap, s.k, s.nsplit, rpc,
                    part_o, part_ml, counters, err_word, out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

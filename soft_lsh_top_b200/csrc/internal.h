@@ -11,8 +11,9 @@ namespace socket_attn {
 struct DecodeShape {
     int64_t B, Hq, Hkv, Ncap, N, d;
     int L, P, k;
-    int G;         // Hq / Hkv
-    int64_t U;     // B * Hkv
+    int G;         // query heads per unit: Hq / Hkv, or 1 when every head selects its own keys
+    int64_t U;     // units: B * Hkv, or B * Hq when every head selects its own keys
+    int share;     // units reading one kv unit's ids, norms, keys and values (1, or Hq / Hkv)
     int NB;        // 2^P
     int nsplit;    // attention splits per unit
 };

@@ -34,8 +34,13 @@
 // conflict-free 16-byte loads; ids and norms stream through L2 with an
 // evict-first policy and the scores are stored evict-last, so top-k reads
 // them from L2.  The grid is persistent (one CTA per SM) and splits the
-// flattened (unit, 32-key chunk) range evenly; a CTA stages the tables of
+// flattened (kv unit, 32-key chunk) range evenly; a CTA stages the tables of
 // each unit it touches (two units at once when a unit needs one region).
+// When every query head selects its own keys, the `share` units of a kv
+// unit (one per head) read the same ids and norms: the grid is then groups
+// of `share` CTAs, CTA h of a group scoring head h over the group's chunk
+// range, so the group's CTAs stream the same id chunks at about the same
+// time and all but the first read of each chunk is served from L2.
 #include "common.cuh"
 #include "internal.h"
 #include "socket_attn.h"
@@ -82,18 +87,19 @@ __device__ __forceinline__ float ldg_stream_f32(const float* p)
 
 struct ScoreArgs {
     const float* tables;  // [U][nblk][NB][64] expanded soft tables
-    const uint8_t* ids;   // [U][Ncap][32 nblk] rotated id rows
-    const float* vnorm;   // [U][Ncap]
+    const uint8_t* ids;   // [U / share][Ncap][32 nblk] rotated id rows
+    const float* vnorm;   // [U / share][Ncap]
     float* scores;        // [U][Ncap]
     uint32_t* unit_max;
     uint32_t* unit_hist;
     uint32_t* err_word;
+    int share;            // units per kv unit (CTAs per group)
     int nblk;             // 32-table blocks of L
     int blk0;             // first block of this launch
     int NB;
     int first, last;      // first / last launch of the step (partial sums between)
     int64_t Ncap, N;
-    int64_t chunks_per_unit, total_chunks, chunks_per_cta;
+    int64_t chunks_per_unit, total_chunks, chunks_per_cta;  // over kv units; per group of CTAs
 };
 
 // NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: 32-key chunks
@@ -144,11 +150,12 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     uint32_t* shist = reinterpret_cast<uint32_t*>(smem + (hist_s - sbase));
     char* ring = smem + (ring_s - sbase);
 
-    const int64_t c0 = (int64_t)blockIdx.x * a.chunks_per_cta;
+    const int h = (int)(blockIdx.x % (unsigned)a.share);  // this CTA's unit within each kv unit
+    const int64_t c0 = (int64_t)(blockIdx.x / (unsigned)a.share) * a.chunks_per_cta;
     const int64_t c1 = min64(a.total_chunks, c0 + a.chunks_per_cta);
     if (c0 >= c1) return;
     const int cpu = (int)a.chunks_per_unit;
-    const int64_t u_first = c0 / cpu;
+    const int64_t u_first = c0 / cpu;  // first kv unit
     const int nseg = (int)((c1 - 1) / cpu - u_first + 1);
     const int Lr = 32 * a.nblk;  // id row bytes
     const int N = (int)a.N;
@@ -169,7 +176,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     // Bulk copy of segment k's table blocks into its slot's regions.
     auto issue_tables = [&](int k) {
         const int s = k % kSlots;
-        const int64_t u = u_first + k;
+        const int64_t u = (u_first + k) * a.share + h;
         mbar_arrive_expect_tx(&bar[s], NBLK * region_bytes);
         for (int bl = 0; bl < NBLK; ++bl) {
             const char* src = reinterpret_cast<const char*>(a.tables) +
@@ -186,9 +193,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     uint32_t seq = 0;      // batches this warp has taken from its ring so far
     bool failed = false;   // a bounded wait of this warp expired
     for (int k = 0; k < nseg; ++k) {
-        const int64_t u = u_first + k;
-        const int cbeg = (int)(max64(c0, u * cpu) - u * cpu);
-        const int nch = (int)(min64(c1, (u + 1) * cpu) - u * cpu) - cbeg;
+        const int64_t ukv = u_first + k;
+        const int64_t u = ukv * a.share + h;
+        const int cbeg = (int)(max64(c0, ukv * cpu) - ukv * cpu);
+        const int nch = (int)(min64(c1, (ukv + 1) * cpu) - ukv * cpu) - cbeg;
         const int slot = k % kSlots;
         // Batch b of this warp holds the KEYS consecutive chunks starting at
         // cbeg + (warp + kWarps b) KEYS (the last group of the segment may be
@@ -197,8 +205,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         const int nbatch = ngroups > warp ? (ngroups - warp + kWarps - 1) / kWarps : 0;
         auto chunk_at = [&](int m) { return cbeg + (warp + kWarps * (m / KEYS)) * KEYS + (m % KEYS); };
         const int cend = cbeg + nch;
-        const uint8_t* idu = a.ids + u * a.Ncap * Lr;
-        const float* vu = a.vnorm + u * a.Ncap;
+        const uint8_t* idu = a.ids + ukv * a.Ncap * Lr;
+        const float* vu = a.vnorm + ukv * a.Ncap;
         float* su = a.scores + u * a.Ncap;
 
         // Lane 0: copy batch b's chunks (this launch's id pieces and, in the
@@ -376,12 +384,15 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     a.NB = s.NB;
     a.Ncap = s.Ncap;
     a.N = s.N;
+    a.share = s.share;
     a.chunks_per_unit = (s.N + 31) / 32;
-    a.total_chunks = s.U * a.chunks_per_unit;
-    // At least one chunk per warp per CTA; at most one CTA per SM.
+    a.total_chunks = (s.U / s.share) * a.chunks_per_unit;
+    // At least one chunk per warp per CTA; at most one CTA per SM; groups of
+    // `share` CTAs.
     const int64_t want = (a.total_chunks + kWarps - 1) / kWarps;
-    const int grid = (int)max64(1, min64(device_num_sms(), want));
-    a.chunks_per_cta = (a.total_chunks + grid - 1) / grid;
+    const int64_t groups = max64(1, min64(device_num_sms() / s.share, want));
+    const int grid = (int)(groups * s.share);
+    a.chunks_per_cta = (a.total_chunks + groups - 1) / groups;
     // Blocks two at a time (two 64 KB regions); partial sums pass through
     // the score buffer between launches when L > 64.
     for (int b0 = 0; b0 < a.nblk; b0 += kRegions) {

@@ -38,7 +38,7 @@ constexpr int kHalf = kHeadDim / 2;  // channels per thread of a dot product
 //      whose column j holds table 32c + j mod 32 (tables past L are zero).
 template <typename QT>
 __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
-    const QT* __restrict__ q, const uint16_t* __restrict__ W, int64_t Hq, int64_t Hkv, int G, int L,
+    const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L,
     int P, double tau, float* __restrict__ tables, uint32_t* __restrict__ err_word,
     uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
     uint32_t* __restrict__ cand_cnt)
@@ -48,8 +48,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     __shared__ double sig[kMaxGroup][kTablesPerBlock][kMaxP][2];
     __shared__ double nib[kMaxGroup][kTablesPerBlock][2][16];
 
-    const int64_t u = blockIdx.x;
-    const int64_t b = u / Hkv, kvh = u % Hkv;
+    const int64_t u = blockIdx.x;  // the unit's query rows are u G .. u G + G - 1 of [B][Hq]
     const int l0 = blockIdx.y * kTablesPerBlock;
     const int nt = min(kTablesPerBlock, L - l0);
     const int NB = 1 << P;
@@ -68,7 +67,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     // load per thread, issued before the hyperplane loads.
     constexpr int kPer16 = 16 / (int)sizeof(QT);             // elements per piece
     const int npieces = G * kHeadDim / kPer16;               // <= 512 for G <= 16
-    const uint4* qu4 = reinterpret_cast<const uint4*>(q + (b * Hq + kvh * G) * kHeadDim);
+    const uint4* qu4 = reinterpret_cast<const uint4*>(q + u * G * kHeadDim);
     uint4 qv[(kMaxGroup * kHeadDim / kPer16 + kThreads - 1) / kThreads];
 #pragma unroll
     for (int i = 0; i < (int)(sizeof(qv) / sizeof(qv[0])); ++i)
@@ -203,10 +202,10 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
     dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
     if (q_dtype == 1)
         return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), 0, stream,
-                          static_cast<const uint16_t*>(q), W, s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word,
+                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, tables, err_word,
                           counters, unit_max, unit_hist, cand_cnt);
     return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), 0, stream, static_cast<const float*>(q), W,
-                      s.Hq, s.Hkv, s.G, s.L, s.P, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt);
+                      s.G, s.L, s.P, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt);
 }
 
 }  // namespace socket_attn

@@ -284,6 +284,36 @@ def pin_score_heads_add(lib):
     assert not np.allclose(s0, s1)
 
 
+def pin_per_head_selection(lib):
+    """One selection per query head: head g's scores split the grouped score
+    by head (they add up to it), its k keys are the k largest of its own
+    scores with ties to the lower index (a stable sort here), and its output
+    is softmax attention over them (numpy, fp64)."""
+    rng = np.random.default_rng(21)
+    L, P, d, n, G, U, k = 6, 5, 16, 257, 3, 2, 9
+    W = rng.standard_normal((L, P, d))
+    q = rng.standard_normal((U, G, d))
+    K = rng.standard_normal((U, n, d))
+    V = rng.standard_normal((U, n, d))
+    hashed = [oracle.hash_keys(K[u], V[u], W, L, P, lib=lib) for u in range(U)]
+    ids = np.stack([h[0] for h in hashed])
+    vn32 = np.stack([h[1].astype(np.float32) for h in hashed])
+    tau = 0.4
+    idx, out, sc = oracle.decode_per_head(q, W, L, P, tau, ids, vn32, K, V, n, k, lib=lib)
+    _, _, gsc = oracle.decode(q, W, L, P, tau, ids, vn32, K, V, n, k, lib=lib)
+    assert np.allclose(sc.sum(axis=1), gsc, rtol=1e-13)
+    for u in range(U):
+        for g in range(G):
+            order = np.argsort(-sc[u, g], kind="stable")
+            assert np.array_equal(idx[u, g], np.sort(order[:k]))
+            sel = idx[u, g]
+            logits = K[u, sel] @ q[u, g] / np.sqrt(d)
+            w = np.exp(logits - logits.max())
+            w /= w.sum()
+            assert np.allclose(out[u, g], w @ V[u, sel], rtol=1e-12, atol=1e-13)
+    assert any(not np.array_equal(idx[u, 0], idx[u, g]) for u in range(U) for g in range(1, G))
+
+
 def pin_score_uniform_query(lib):
     """A zero query puts probability 2^-P on every bucket, so every key scores
     G * L * 2^-P * ||v|| whatever its bucket ids."""

@@ -81,16 +81,18 @@ def gpu_hash(inp, w, n_begin=0, n_end=None):
     return ids, vnorm
 
 
-def gpu_decode(inp, w, ids, vnorm, N=None, tau=None, k=None, q=None):
+def gpu_decode(inp, w, ids, vnorm, N=None, tau=None, k=None, q=None, per_head=False):
+    """socket_decode (per_head: socket_decode_per_head) with the scores kept."""
     dev = inp["K"].device
     B = inp["K"].shape[0]
     N = w.N if N is None else N
     k = w.k if k is None else k
     q = inp["q"] if q is None else q
-    ws, idx, out = sk.alloc_decode_buffers(B, w.Hq, w.Hkv, w.ncap, w.L, w.P, k, dev)
-    scores = torch.full((B, w.Hkv, w.ncap), float("nan"), dtype=torch.float32, device=dev)
-    sk.socket_decode(q, inp["W"], ids, vnorm, inp["K"], inp["V"], N, w.tau if tau is None else tau, k,
-                     ws, idx, out, scores_out=scores)
+    ws, idx, out = sk.alloc_decode_buffers(B, w.Hq, w.Hkv, w.ncap, w.L, w.P, k, dev, per_head=per_head)
+    scores = torch.full((B, w.Hq if per_head else w.Hkv, w.ncap), float("nan"), dtype=torch.float32, device=dev)
+    fn = sk.socket_decode_per_head if per_head else sk.socket_decode
+    fn(q, inp["W"], ids, vnorm, inp["K"], inp["V"], N, w.tau if tau is None else tau, k, ws, idx, out,
+       scores_out=scores)
     torch.cuda.synchronize()
     assert sk.read_device_error(ws) == 0
     return idx, out, scores
@@ -158,7 +160,11 @@ def check_unit(q_u, W, L, P, tau, ids_u, vn_u, K_u, V_u, N, k, g_idx, g_out, g_s
     return {"swapped": int(swapped.size), "out_err": float(err)}
 
 
-def check_decode(inp, w, orc_ids, orc_vn32, units, g_idx, g_out, g_sc, N=None, tau=None, k=None, q=None):
+def check_decode(inp, w, orc_ids, orc_vn32, units, g_idx, g_out, g_sc, N=None, tau=None, k=None, q=None,
+                 per_head=False):
+    """Compare sampled kv units.  per_head: the results of
+    socket_decode_per_head, each query head checked as a unit of one query
+    row over its kv head's ids, norms, keys and values."""
     N = w.N if N is None else N
     k = w.k if k is None else k
     tau = w.tau if tau is None else tau
@@ -170,6 +176,13 @@ def check_decode(inp, w, orc_ids, orc_vn32, units, g_idx, g_out, g_sc, N=None, t
         q_u = q[b, h * w.G:(h + 1) * w.G].cpu()
         K_u = inp["K"][b, h].cpu()
         V_u = inp["V"][b, h].cpu()
+        if per_head:
+            for g in range(w.G):
+                r = h * w.G + g
+                stats.append(check_unit(q_u[g:g + 1], Wc, w.L, w.P, tau, orc_ids[i], orc_vn32[i], K_u, V_u, N, k,
+                                        g_idx[b, r].cpu().numpy(), g_out[b, r:r + 1].cpu().numpy(),
+                                        g_sc[b, r].cpu().numpy()))
+            continue
         stats.append(check_unit(q_u, Wc, w.L, w.P, tau, orc_ids[i], orc_vn32[i], K_u, V_u, N, k,
                                 g_idx[b, h].cpu().numpy(), g_out[b, h * w.G:(h + 1) * w.G].cpu().numpy(),
                                 g_sc[b, h].cpu().numpy()))

@@ -54,12 +54,12 @@ def test_version(lib):
 P16 = 0x10000
 
 
-def decode(lib, **kw):
+def decode(lib, entry="socket_decode", **kw):
     a = dict(q=P16, q_dtype=1, W=P16, ids=P16, vnorm=P16, K=P16, V=P16, kv_dtype=1, B=1, Hq=4, Hkv=1, Ncap=64,
              N=64, d=128, L=4, P=8, tau=0.5, k=8, ws=P16, ws_bytes=1 << 30, idx=P16, out=P16, scores=None,
              stream=None)
     a.update(kw)
-    return lib.socket_decode(a["q"], a["q_dtype"], a["W"], a["ids"], a["vnorm"], a["K"], a["V"], a["kv_dtype"],
+    return getattr(lib, entry)(a["q"], a["q_dtype"], a["W"], a["ids"], a["vnorm"], a["K"], a["V"], a["kv_dtype"],
                              a["B"], a["Hq"], a["Hkv"], a["Ncap"], a["N"], a["d"], a["L"], a["P"], a["tau"],
                              a["k"], a["ws"], a["ws_bytes"], a["idx"], a["out"], a["scores"], a["stream"])
 
@@ -90,9 +90,16 @@ def decode(lib, **kw):
     (dict(ws=P16 + 16), EWS),
     (dict(ws_bytes=16), EWS),
 ])
-def test_decode_rejects(lib, kw, status):
-    assert decode(lib, **kw) == status
+@pytest.mark.parametrize("entry", ["socket_decode", "socket_decode_per_head"])
+def test_decode_rejects(lib, entry, kw, status):
+    assert decode(lib, entry, **kw) == status
     assert lib.socket_last_error().decode() != ""
+
+
+def test_per_head_rejects_too_many_query_heads(lib):
+    # 4096 x 32 query-head units exceed the limit; 4096 x 2 kv units would not.
+    assert decode(lib, "socket_decode_per_head", B=4096, Hq=32, Hkv=2) == EUNSUP
+    assert "B*Hq" in lib.socket_last_error().decode()
 
 
 def hash_call(lib, **kw):
@@ -135,6 +142,17 @@ def test_workspace_size(lib):
     assert f(1, 4, 1, 64, 64, 4, 8, 8) == 0          # d != 128
     assert f(1, 4, 1, 64, 128, 4, 8, 100) == 0       # k > Ncap
     assert f(1, 3, 2, 64, 128, 4, 8, 8) == 0         # Hq % Hkv != 0
+
+
+def test_per_head_workspace_size(lib):
+    f, g = lib.socket_decode_workspace_size, lib.socket_decode_per_head_workspace_size
+    # one head per kv head: the same step, the same workspace
+    assert g(2, 4, 4, 4096, 128, 32, 8, 256) == f(2, 4, 4, 4096, 128, 32, 8, 256)
+    # four heads per kv head: a table set, a score row and a selection per head
+    grouped, per_head = f(8, 32, 8, 131072, 128, 32, 8, 2048), g(8, 32, 8, 131072, 128, 32, 8, 2048)
+    assert per_head >= 256 * 131072 * 4 + 256 * 32 * 256 * 4 > grouped
+    assert g(4096, 32, 2, 64, 128, 4, 8, 8) == 0     # B*Hq above 65535
+    assert g(1, 3, 2, 64, 128, 4, 8, 8) == 0         # Hq % Hkv != 0
 
 
 def test_python_binding_checks_shapes_before_the_library():

@@ -59,6 +59,7 @@ def test_hash_matches_oracle(small):
 
 
 def _decode_on_oracle_index(small, **kw):
+    """Decode on the oracle's ids and norms (so that scores compare key by key)."""
     w, inp, units, orc_ids, orc_vn, _ = small
     orc_vn32 = orc_vn.astype(np.float32)
     ids = torch.from_numpy(ids_to_rows(orc_ids, w.L)).reshape(inp["K"].shape[0], w.Hkv, w.ncap // 32, -1, 32,
@@ -72,22 +73,45 @@ def test_decode_matches_oracle(small):
     _decode_on_oracle_index(small)
 
 
-@pytest.mark.parametrize("variant", ["k1", "k_eq_n", "tau_0.01", "tau_5", "tau_0_hard", "n_not_ncap"])
+def test_decode_per_head_matches_oracle(small):
+    """One selection per query head: every head's scores, selection and
+    output against the oracle run on that head alone."""
+    _decode_on_oracle_index(small, per_head=True)
+
+
+def test_per_head_with_one_head_per_kv_head_is_the_grouped_decode():
+    """With Hq == Hkv both entry points compute the same thing, bit for bit."""
+    w = SMALL["bf16_single_head"]
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)
+    idx_a, out_a, sc_a = gpu_decode(inp, w, ids, vnorm)
+    idx_b, out_b, sc_b = gpu_decode(inp, w, ids, vnorm, per_head=True)
+    assert torch.equal(idx_a, idx_b)
+    assert torch.equal(out_a, out_b)
+    assert torch.equal(sc_a[..., :w.N], sc_b[..., :w.N])
+
+
+@pytest.mark.parametrize("variant", ["k1", "k_eq_n", "tau_0.01", "tau_5", "tau_0_hard", "n_not_ncap",
+                                     "per_head_k1", "per_head_tau_0_hard", "per_head_n_not_ncap"])
 def test_decode_edge_cases(small, variant):
     w = small[0]
+    kw = {}
+    if variant.startswith("per_head_"):
+        variant = variant[len("per_head_"):]
+        kw["per_head"] = True
     if variant == "k1":
-        _decode_on_oracle_index(small, k=1)
+        _decode_on_oracle_index(small, k=1, **kw)
     elif variant == "k_eq_n":
-        _decode_on_oracle_index(small, k=w.N)
+        _decode_on_oracle_index(small, k=w.N, **kw)
     elif variant == "tau_0.01":
-        _decode_on_oracle_index(small, tau=0.01)
+        _decode_on_oracle_index(small, tau=0.01, **kw)
     elif variant == "tau_5":
-        _decode_on_oracle_index(small, tau=5.0)
+        _decode_on_oracle_index(small, tau=5.0, **kw)
     elif variant == "tau_0_hard":
-        _decode_on_oracle_index(small, tau=0.0)
+        _decode_on_oracle_index(small, tau=0.0, **kw)
     else:
         n = w.N - 13
-        _decode_on_oracle_index(small, N=n, k=min(w.k, n))
+        _decode_on_oracle_index(small, N=n, k=min(w.k, n), **kw)
 
 
 def test_all_ties_select_lowest_indices():
@@ -207,6 +231,26 @@ def test_batch8_128k_sampled_units_and_needles():
                                    inp["K"][b, h].cpu(), inp["V"][b, h].cpu(), w.N, w.k)[0]
         nd = needles[b, h].cpu().numpy()
         assert np.array_equal(np.isin(nd, idx[b, h].cpu().numpy()), np.isin(nd, o_idx)), u
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_batch8_128k_per_head_sampled_units_and_needles():
+    """One selection per query head at full size: sampled kv units checked
+    head by head against the oracle, and each head's own needles found by its
+    own selection (no competition from the group's other heads)."""
+    w = wl.BATCH8_128K
+    units = [5, 40]
+    inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
+    idx, _, _ = gpu_decode(inp, w, ids, vnorm, per_head=True)
+    needles, m = inp["needles"], w.needles_per_head
+    found = sum(int(torch.isin(needles[b, kvh, g * m:(g + 1) * m].to(torch.int32), idx[b, kvh * w.G + g]).sum())
+                for b in range(w.B) for kvh in range(w.Hkv) for g in range(w.G))
+    recall = found / needles.numel()
+    assert recall >= 0.99, recall
+    substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm, per_head=True)
+    check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, per_head=True)
     del inp
     torch.cuda.empty_cache()
 
