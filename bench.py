@@ -386,6 +386,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         sk.socket_hash_keys(inp0["K"], inp0["V"], inp0["W"], ids0, vn0, 0, w.N)
     h1.record()
     torch.cuda.synchronize()
+    sk.socket_hash_check()
     hash_ms = max_over_ranks(h0.elapsed_time(h1) / RH, world)
 
     # ---- one selection per query head (socket_decode_per_head) on the same
@@ -467,7 +468,8 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         hash_tflops = hash_flops / (hash_ms * 1e-3) / 1e12
         prefill = {
             "what": "socket_hash_keys over the whole layer (all units, N keys each); not in the decode step",
-            "kernel": "hash_mma_kernel" if w.dtype == "bf16" else "hash_kernel",
+            "kernel": ("hash_umma_kernel" if w.L * w.P <= 256 else "hash_mma_kernel") if w.dtype == "bf16"
+                      else "hash_kernel",
             "keys": keys, "ms": hash_ms, "keys_per_s": world * keys / (hash_ms * 1e-3),
             "algorithmic_bytes": hash_bytes, "gbs": hash_gbs, "hbm_frac": hash_gbs / peak,
             "flops": hash_flops, "tflops": hash_tflops,
@@ -478,12 +480,24 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         # CTAs stream them side by side) and writes a score row per head.
         ph_score_bytes = w.U * w.N * (w.L + 4) + w.U * w.G * w.N * 4
         ph_score_gbs = ph_score_bytes / (ph_kern["score"] * 1e-3) / 1e9
+        # Each (head, key, table) is one 4-byte shared-memory lookup: per head
+        # that is the whole lookup stream, bound by the SMs' shared-memory
+        # bandwidth (128 B per clock per SM) at the sampled SM clock.
+        ck = clocks.summary()
+        mhz = ck.get("sm_mhz") or ck.get("sm_max_mhz") or 1965.0
+        n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+        smem_peak = n_sm * 128 * mhz * 1e6 / 1e9
+        lookup_bytes = w.U * w.G * w.N * w.L * 4
+        lookup_gbs = lookup_bytes / (ph_kern["score"] * 1e-3) / 1e9
         per_head = {
             "what": "socket_decode_per_head: one selection per query head (B*Hq units) on the same layers; "
                     "direct calls",
             "steps_per_s": whole_job_rate(world, KH, ph_ms), "ms_per_step": ph_ms / KH, "steps": KH,
             "kernels_ms": ph_kern,
-            "score": {"algorithmic_bytes": ph_score_bytes, "gbs": ph_score_gbs, "frac": ph_score_gbs / peak},
+            "score": {"hbm_algorithmic_bytes": ph_score_bytes, "hbm_gbs": ph_score_gbs, "hbm_frac": ph_score_gbs / peak,
+                      "bound": "smem", "lookup_bytes": lookup_bytes, "achieved": lookup_gbs, "peak": smem_peak,
+                      "unit": "GB/s", "frac": lookup_gbs / smem_peak,
+                      "peak_source": f"derived: {n_sm} SMs x 128 B/clock x {mhz:.0f} MHz (sampled SM clock)"},
             "attention_gbs": w.U * w.G * 2 * w.k * w.d * w.elem_bytes / (ph_kern["attention"] * 1e-3) / 1e9,
         }
         traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",

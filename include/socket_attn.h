@@ -108,6 +108,15 @@ int socket_hash_keys(const void* K, const void* V, int kv_dtype,
 int socket_ids_row_bytes(int L);
 
 /*
+ * socket_hash_check -- waits for `stream`, then reports whether a hashing
+ * kernel of this library gave up on one of its bounded waits since the last
+ * check (SOCKET_ECUDA with a message; its ids and norms are then
+ * unspecified) and clears that record.  SOCKET_OK otherwise.  The record is
+ * per device and process.
+ */
+int socket_hash_check(void* stream);
+
+/*
  * socket_decode_workspace_size -- bytes of device scratch socket_decode needs
  * for these sizes (0 if the sizes are invalid).  The workspace needs no
  * initialisation, must be 256-byte aligned, and may be reused by later calls

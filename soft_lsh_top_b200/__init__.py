@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
-    "socket_decode_per_head", "socket_decode_per_head_workspace_size",
+    "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -61,6 +61,8 @@ def load_library(path: str | None = None):
     lib = ctypes.CDLL(p)
     lib.socket_hash_keys.argtypes = [_vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64, _vp, _int, _int, _vp, _vp, _vp]
     lib.socket_hash_keys.restype = _int
+    lib.socket_hash_check.argtypes = [_vp]
+    lib.socket_hash_check.restype = _int
     lib.socket_decode_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]
     lib.socket_decode_workspace_size.restype = _sz
     lib.socket_decode.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _i64,
@@ -155,6 +157,12 @@ def socket_hash_keys(K: torch.Tensor, V: torch.Tensor, W: torch.Tensor, ids: tor
     with torch.cuda.device(dev):
         _raise(lib.socket_hash_keys(K.data_ptr(), V.data_ptr(), _code(K), B, Hkv, Ncap, int(n_begin), n_end, d,
                                     W.data_ptr(), L, P, ids.data_ptr(), vnorm.data_ptr(), _stream_handle(stream)))
+
+
+def socket_hash_check(stream=None) -> None:
+    """Wait for the stream; raise SocketError if a hashing kernel gave up on a
+    bounded wait since the last check (the record is then cleared)."""
+    _raise(load_library().socket_hash_check(_stream_handle(stream)))
 
 
 def socket_ids_row_bytes(L: int) -> int:

@@ -260,6 +260,16 @@ int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int6
                        "hash kernel launch");
 }
 
+int socket_hash_check(void* stream)
+{
+    g_last_error.clear();
+    uint32_t bits = 0;
+    const int e = hash_device_error(static_cast<cudaStream_t>(stream), &bits);
+    if (e != 0) return cuda_status(static_cast<cudaError_t>(e), "hash error check");
+    if (bits) return fail(SOCKET_ECUDA, "hash kernel: a bounded wait expired (device error bits 0x%x)", bits);
+    return SOCKET_OK;
+}
+
 int socket_ids_row_bytes(int L) { return (L >= 1 && L <= SOCKET_MAX_L) ? ids_row_bytes(L) : 0; }
 
 size_t socket_decode_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int L, int P,

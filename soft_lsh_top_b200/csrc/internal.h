@@ -75,6 +75,10 @@ cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const vo
                              const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
                              uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream);
 
+// Waits for `stream`, then reads and clears the hash kernels' device error
+// bits; returns a cudaError_t value.
+int hash_device_error(cudaStream_t stream, uint32_t* bits);
+
 // Sets the calling thread's socket_last_error() message; returns `status`.
 int record_error(int status, const char* message);
 

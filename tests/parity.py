@@ -78,6 +78,7 @@ def gpu_hash(inp, w, n_begin=0, n_end=None):
     ids.zero_()
     vnorm.zero_()
     sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, n_begin, w.N if n_end is None else n_end)
+    sk.socket_hash_check()
     return ids, vnorm
 
 

@@ -69,6 +69,28 @@ def _decode_on_oracle_index(small, **kw):
     return check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, **kw)
 
 
+@pytest.mark.parametrize("case", ["bf16_single_head", "odd_group3_p5", "bf16_l80_p7"])
+def test_hash_in_ranges_matches_oracle(case):
+    """The cache hashed piecewise -- a long range from an unaligned start, single
+    appended keys, a range inside one 32-key chunk, the rest -- equals the
+    oracle's hash of every key (tensor-core tiles that start anywhere and end
+    ragged; the last case has more hyperplanes than one tensor-core tile and
+    takes the warp-level kernel)."""
+    w = SMALL[case]
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = sk.alloc_cache_index(inp["K"].shape[0], w.Hkv, w.ncap, w.L, DEV)
+    ids.zero_()
+    vnorm.zero_()
+    cuts = sorted({0, 37, 38, 39, 70, 1000, 1001, w.N - 1, w.N})
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, a, b)
+    sk.socket_hash_check()
+    units = list(range(w.U))
+    orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units)
+    check_hash(ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy(), vnorm.reshape(w.U, w.ncap).cpu().numpy(),
+               orc_ids, orc_vn, margin, 0, w.N)
+
+
 def test_decode_matches_oracle(small):
     _decode_on_oracle_index(small)
 
@@ -277,7 +299,7 @@ def test_append_mix_sampled_units():
     for t in range(w.appends):
         sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, w.N + t, w.N + t + 1)
         gpu_decode(inp, w, ids, vnorm, N=w.N + t + 1, q=inp["q_steps"][t])
-    torch.cuda.synchronize()
+    sk.socket_hash_check()
     n_all = w.N + w.appends
     orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units, 0, n_all)
     g_ids = torch.stack([ids[u // w.Hkv, u % w.Hkv] for u in units]).cpu().numpy()
