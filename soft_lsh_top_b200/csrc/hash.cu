@@ -289,7 +289,7 @@ __global__ __launch_bounds__(kMThreads) void hash_mma_kernel(const uint16_t* __r
 // lets its own copies and MMAs land, frees tensor memory and exits.
 // ---------------------------------------------------------------------------
 constexpr int kUKeys = 128;                            // keys per tile (UMMA M)
-constexpr int kUStages = 3;
+constexpr int kUStages = 2;
 constexpr int kUThreads = 320;
 constexpr uint32_t kUBoxBytes = kUKeys * 128u;         // 128 rows x 64 bf16 channels
 constexpr uint32_t kUTileBytes = 2u * kUBoxBytes;      // 32 KB
@@ -379,18 +379,21 @@ struct HashUArgs {
 };
 
 __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                 const __grid_constant__ CUtensorMap tmV,
                                                                  const __grid_constant__ CUtensorMap tmW,
                                                                  const HashUArgs a)
 {
     extern __shared__ __align__(1024) char dsm[];
-    __shared__ __align__(8) uint64_t full[kUStages], empty[kUStages], tfull[2], tempty[2], wbar, done;
+    __shared__ __align__(8) uint64_t full[kUStages], empty[kUStages], tfull[2], tempty[2], vfull[2], vempty[2], wbar,
+        done;
     __shared__ uint32_t tmem_slot;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t raw = smem_addr(dsm);
     const uint32_t sW = (raw + 1023u) & ~1023u;                 // [2 boxes][Np rows][128 B]
     const uint32_t sK = sW + (uint32_t)a.Np * 256u;             // [kUStages][2 boxes][128 rows][128 B]
-    uint32_t* sgn = reinterpret_cast<uint32_t*>(dsm + (sK + kUStages * kUTileBytes - raw));  // [2][128][9]
+    const uint32_t sV = sK + kUStages * kUTileBytes;            // [2 groups][2 boxes][128 rows][128 B]
+    uint32_t* sgn = reinterpret_cast<uint32_t*>(dsm + (sV + 2 * kUTileBytes - raw));  // [2][128][9]
     const int Lr = 32 * ((a.L + 31) / 32);
 
     if (tid == 0) {
@@ -400,7 +403,9 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+            mbar_init(&tempty[b], 4);  // one arrival per epilogue warp of group b
+            mbar_init(&vfull[b], 1);
+            mbar_init(&vempty[b], 4);
         }
         mbar_init(&wbar, 1);
         mbar_init(&done, 1);
@@ -426,8 +431,9 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
             int i = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++i) {
-                const int s = i % kUStages;
-                if (!mbar_wait_bounded(&empty[s], ((i / kUStages) & 1) ^ 1, kUMaxPolls)) {
+                const int s = i % kUStages, g = i & 1;
+                if (!mbar_wait_bounded(&empty[s], ((i / kUStages) & 1) ^ 1, kUMaxPolls) ||
+                    !mbar_wait_bounded(&vempty[g], ((i >> 1) & 1) ^ 1, kUMaxPolls)) {
                     ok = false;
                     break;
                 }
@@ -436,12 +442,16 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
                 mbar_arrive_expect_tx(&full[s], kUTileBytes);
                 tma_load_3d(sK + s * kUTileBytes, &tmK, 0, n0, u, &full[s]);
                 tma_load_3d(sK + s * kUTileBytes + kUBoxBytes, &tmK, 64, n0, u, &full[s]);
+                mbar_arrive_expect_tx(&vfull[g], kUTileBytes);
+                tma_load_3d(sV + g * kUTileBytes, &tmV, 0, n0, u, &vfull[g]);
+                tma_load_3d(sV + g * kUTileBytes + kUBoxBytes, &tmV, 64, n0, u, &vfull[g]);
             }
             if (!ok) atomicOr(&g_hash_err, 1u);
-            // The last copies of every stage have landed before the CTA exits.
+            // The last copies of every stage and buffer have landed before the CTA exits.
             mbar_wait_bounded(&wbar, 0, kUMaxPolls);
             for (int j = max(0, i - kUStages); j < i; ++j)
                 mbar_wait_bounded(&full[j % kUStages], (j / kUStages) & 1, kUMaxPolls);
+            for (int j = max(0, i - 2); j < i; ++j) mbar_wait_bounded(&vfull[j & 1], (j >> 1) & 1, kUMaxPolls);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -486,24 +496,16 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
         uint32_t* srow = sgn + (grp * kUKeys + r) * kUSgnStride;
         srow[8] = 0u;
         const int64_t step = 2 * (int64_t)gridDim.x;
-        uint4 vv[kHeadDim / 8];
-        // The value row of this thread's key in tile t, loaded ahead of use.
-        auto load_v = [&](int64_t t) {
-            if (t >= a.tiles) return;
-            const int64_t u = t / a.tiles_per_unit;
-            const int64_t n = a.n_begin + (t % a.tiles_per_unit) * kUKeys + r;
-            if (n >= a.n_end) return;
-            const uint4* vp = reinterpret_cast<const uint4*>(a.V + (u * a.Ncap + n) * kHeadDim);
-#pragma unroll
-            for (int c = 0; c < kHeadDim / 8; ++c) vv[c] = __ldg(vp + c);
-        };
-        int64_t t = blockIdx.x + grp * (int64_t)gridDim.x;
-        load_v(t);
-        for (int j = 0; t < a.tiles; t += step, ++j) {
+        // This thread's value row: the 16-byte chunks of row r in the group's
+        // two swizzled boxes, read in an order staggered by r so that a warp's
+        // loads spread over all banks (only the sum of squares is taken).
+        const uint32_t vrow = sV + (uint32_t)grp * kUTileBytes + (uint32_t)r * 128u;
+        for (int64_t t = blockIdx.x + grp * (int64_t)gridDim.x, j = 0; t < a.tiles; t += step, ++j) {
             const int64_t u = t / a.tiles_per_unit;
             const int64_t n = a.n_begin + (t % a.tiles_per_unit) * kUKeys + r;
             const bool live = n < a.n_end;
-            const bool ok = mbar_wait_bounded(&tfull[grp], j & 1, kUMaxPolls);
+            const bool ok = mbar_wait_bounded(&vfull[grp], j & 1, kUMaxPolls) &&
+                            mbar_wait_bounded(&tfull[grp], j & 1, kUMaxPolls);
             if (!__all_sync(kFullMask, ok)) {
                 if (lane == 0) atomicOr(&g_hash_err, 1u);
                 break;
@@ -534,7 +536,11 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
                 double s0 = 0.0, s1 = 0.0;
 #pragma unroll
                 for (int c = 0; c < kHeadDim / 8; ++c) {
-                    const uint32_t w4[4] = {vv[c].x, vv[c].y, vv[c].z, vv[c].w};
+                    uint4 x;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w)
+                                 : "r"(vrow + (uint32_t)(c >> 3) * kUBoxBytes + (uint32_t)((c ^ r) & 7) * 16u));
+                    const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = bf16x2_to_f32x2(w4[e]);
@@ -544,7 +550,9 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
                 }
                 a.vnorm[u * a.Ncap + n] = (float)sqrt(s0 + s1);
             }
-            load_v(t + step);
+            fence_proxy_async_shared();  // these reads precede the next tensor copy into the buffer
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vempty[grp]);
             if (!live) continue;
 
             // Rotated id row: slot s of block c holds table 32c + (s + n) mod 32.
@@ -669,14 +677,15 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
         a.Np = (planes + 15) / 16 * 16;
         a.tiles_per_unit = (int)((nkeys + kUKeys - 1) / kUKeys);
         a.tiles = B * Hkv * a.tiles_per_unit;
-        CUtensorMap tmK, tmW;
+        CUtensorMap tmK, tmV, tmW;
         if (encode_rows(&tmK, K, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys) &&
+            encode_rows(&tmV, V, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys) &&
             encode_rows(&tmW, W, (uint64_t)planes, 1, (uint32_t)a.Np)) {
-            const int smem = 1024 + a.Np * 256 + kUStages * (int)kUTileBytes + 2 * kUKeys * kUSgnStride * 4;
+            const int smem = 1024 + a.Np * 256 + (kUStages + 2) * (int)kUTileBytes + 2 * kUKeys * kUSgnStride * 4;
             cudaError_t e = cudaFuncSetAttribute(hash_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
             const int grid = (int)min64(device_num_sms(), a.tiles);
-            hash_umma_kernel<<<grid, kUThreads, smem, stream>>>(tmK, tmW, a);
+            hash_umma_kernel<<<grid, kUThreads, smem, stream>>>(tmK, tmV, tmW, a);
             return cudaGetLastError();
         }
     }
