@@ -427,6 +427,44 @@ def run_socket(args, world: int, rank: int, local_rank: int):
     del ws_h, idx_h, out_h, evs_h
     torch.cuda.empty_cache()
 
+    # ---- decode steps that append one key each (the append-mix workload):
+    # hash + decode as two calls, and the fused socket_decode_append.
+    wa = wl.APPEND_MIX.scaled(seed=wl.APPEND_MIX.seed + 7919 * rank)
+    ia = wl.make_inputs(wa, dev)
+    ids_a, vn_a = sk.alloc_cache_index(wa.B, wa.Hkv, wa.ncap, wa.L, dev)
+    sk.socket_hash_keys(ia["K"], ia["V"], ia["W"], ids_a, vn_a, 0, wa.N)
+    ws_a, idx_a, out_a = sk.alloc_decode_buffers(wa.B, wa.Hq, wa.Hkv, wa.ncap, wa.L, wa.P, wa.k, dev)
+
+    def two_calls(t):
+        sk.socket_hash_keys(ia["K"], ia["V"], ia["W"], ids_a, vn_a, wa.N + t, wa.N + t + 1)
+        sk.socket_decode(ia["q_steps"][t], ia["W"], ids_a, vn_a, ia["K"], ia["V"], wa.N + t + 1, wa.tau, wa.k,
+                         ws_a, idx_a, out_a)
+
+    def fused(t):
+        sk.socket_decode_append(ia["q_steps"][t], ia["W"], ids_a, vn_a, ia["K"], ia["V"], wa.N + t + 1, wa.tau,
+                                wa.k, 1, ws_a, idx_a, out_a)
+
+    append = {"what": "64 decode steps that each append one key (hash + decode), append-mix workload: "
+                      "socket_hash_keys + socket_decode vs the fused socket_decode_append; direct calls",
+              "workload": wa.name, "B": wa.B, "Hq": wa.Hq, "Hkv": wa.Hkv, "N": wa.N, "L": wa.L, "P": wa.P,
+              "k": wa.k}
+    for name, fn in (("two_calls", two_calls), ("fused", fused)):
+        for t in range(wa.appends):  # warm-up (re-hashing a key writes the same bytes)
+            fn(t)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a0.record()
+        for t in range(wa.appends):
+            fn(t)
+        a1.record()
+        torch.cuda.synchronize()
+        ms = a0.elapsed_time(a1)
+        append[name] = {"steps_per_s": wa.appends / (ms * 1e-3), "us_per_step": 1e3 * ms / wa.appends}
+    sk.socket_hash_check()
+    assert sk.read_device_error(ws_a) == 0
+    del ia, ids_a, vn_a, ws_a, idx_a, out_a
+    torch.cuda.empty_cache()
+
     # ---- end to end through the public API with host buffers.
     q_host = [torch.empty_like(l[0]["q"], device="cpu").pin_memory() for l in layers]
     for l, qh in zip(layers, q_host):
@@ -522,6 +560,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "clocks": clocks.summary(),
             "prefill": prefill,
             "per_head": per_head,
+            "append": append,
             "e2e": {"value": whole_job_rate(world, K, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
         }

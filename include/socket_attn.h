@@ -170,6 +170,31 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W,
                   int32_t* idx_out, float* out, float* scores_out, void* stream);
 
 /*
+ * socket_decode_append -- a decode step whose last n_new keys were just
+ * appended: the caller has written keys and values N - n_new .. N - 1 of
+ * every unit into K and V; this call hashes them (step 1, [ES] "Pre-cálculo
+ * (Prellenado)" / [DE] "Vorverarbeitung (Prefill)": their rows of ids and
+ * their vnorm are written, as socket_hash_keys would write them) inside the
+ * step's first kernel, then runs socket_decode over N keys.  One call
+ * replaces socket_hash_keys(N - n_new, N) followed by socket_decode.
+ *
+ *   Arguments as for socket_decode, except that ids and vnorm are also
+ *   written (the rows of the n_new keys) and:
+ *   n_new      1 <= n_new <= min(64, N).
+ * The projections are summed in float32 in another order than the hash
+ * kernels', so an id can differ from socket_hash_keys' only where some
+ * |<W_{l,p}, k>| is within float32 accumulation error of 0.  The workspace is
+ * socket_decode_workspace_size()'s.
+ */
+int socket_decode_append(const void* q, int q_dtype, const uint16_t* W,
+                         uint8_t* ids, float* vnorm,
+                         const void* K, const void* V, int kv_dtype,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d,
+                         int L, int P, double tau, int k, int64_t n_new,
+                         void* workspace, size_t workspace_bytes,
+                         int32_t* idx_out, float* out, float* scores_out, void* stream);
+
+/*
  * socket_decode_per_head_workspace_size / socket_decode_per_head -- the same
  * step with one selection per query head instead of one per kv head: every
  * query is scored and selects on its own, as the pages state the method for

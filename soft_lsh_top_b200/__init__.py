@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
-    "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check",
+    "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check", "socket_decode_append",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -71,6 +71,9 @@ def load_library(path: str | None = None):
     lib.socket_decode_per_head_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64, _int, _int, _int]
     lib.socket_decode_per_head_workspace_size.restype = _sz
     lib.socket_decode_per_head.argtypes = lib.socket_decode.argtypes
+    lib.socket_decode_append.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
+                                         _i64, _int, _int, _dbl, _int, _i64, _vp, _sz, _vp, _vp, _vp, _vp]
+    lib.socket_decode_append.restype = _int
     lib.socket_decode_per_head.restype = _int
     lib.socket_decode_static.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64,
                                          _i64, _int, _int, _dbl, _int, _vp, _vp, _vp, _vp]
@@ -193,7 +196,8 @@ def socket_decode_per_head_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, 
     return n
 
 
-def _decode(per_head: bool, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream):
+def _decode(per_head: bool, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream,
+            n_new: int = 0):
     lib = load_library()
     B, Hq, d = q.shape
     _, Hkv, Ncap, _ = K.shape
@@ -212,14 +216,17 @@ def _decode(per_head: bool, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_ou
         raise ValueError("workspace must be a 1-D uint8 CUDA tensor on the inputs' device")
     if scores_out is not None:
         _check(scores_out, "scores_out", (B, sel, Ncap), dtype=torch.float32, device=dev)
-    fn = lib.socket_decode_per_head if per_head else lib.socket_decode
+    head = (q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(), K.data_ptr(), V.data_ptr(),
+            _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P, float(tau), int(k))
+    tail = (workspace.data_ptr(), workspace.numel(), idx_out.data_ptr(), out.data_ptr(),
+            scores_out.data_ptr() if scores_out is not None else None, _stream_handle(stream))
     with torch.cuda.device(dev):
-        _raise(fn(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(),
-                  K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap, int(N), d, L, P,
-                  float(tau), int(k), workspace.data_ptr(), workspace.numel(),
-                  idx_out.data_ptr(), out.data_ptr(),
-                  scores_out.data_ptr() if scores_out is not None else None,
-                  _stream_handle(stream)))
+        if n_new:
+            _raise(lib.socket_decode_append(*head, int(n_new), *tail))
+        elif per_head:
+            _raise(lib.socket_decode_per_head(*head, *tail))
+        else:
+            _raise(lib.socket_decode(*head, *tail))
 
 
 def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
@@ -236,6 +243,18 @@ def socket_decode(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: to
     scores_out: optional [B, Hkv, Ncap] float32.
     """
     _decode(False, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream)
+
+
+def socket_decode_append(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,
+                         K: torch.Tensor, V: torch.Tensor, N: int, tau: float, k: int, n_new: int,
+                         workspace: torch.Tensor, idx_out: torch.Tensor, out: torch.Tensor,
+                         scores_out: torch.Tensor | None = None, stream=None) -> None:
+    """socket_decode after appending keys N - n_new .. N - 1 to K and V: the
+    step also hashes those keys (writing their ids and vnorm).  Shapes as
+    socket_decode; 1 <= n_new <= 64."""
+    if int(n_new) < 1:
+        raise ValueError("n_new must be >= 1")
+    _decode(False, q, W, ids, vnorm, K, V, N, tau, k, workspace, idx_out, out, scores_out, stream, n_new=int(n_new))
 
 
 def socket_decode_per_head(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor,

@@ -159,11 +159,14 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     return w;
 }
 
-// One decode step; per_head: every query head selects its own keys.
+// One decode step; per_head: every query head selects its own keys; the
+// last n_new keys of every unit are hashed inside the step (ids and norms
+// written through app_ids / app_vnorm) when n_new > 0.
 int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
            const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N,
            int64_t d, int L, int P, double tau, int k, void* workspace, size_t workspace_bytes, int32_t* idx_out,
-           float* out, float* scores_out, cudaStream_t cs)
+           float* out, float* scores_out, cudaStream_t cs, int64_t n_new = 0, uint8_t* app_ids = nullptr,
+           float* app_vnorm = nullptr)
 {
     g_last_error.clear();
     DecodeShape s;
@@ -177,6 +180,8 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(K, 16) ||
         !aligned(V, 16) || !aligned(out, 16) || !aligned(idx_out, 4) || (scores_out && !aligned(scores_out, 16)))
         return fail(SOCKET_EINVAL, "q, W, ids, vnorm, K, V, out, scores_out must be 16-byte aligned, idx_out 4-byte");
+    if (n_new < 0 || n_new > kMaxAppend || n_new > N)
+        return fail(SOCKET_EINVAL, "n_new=%lld outside [0, min(%d, N)]", (long long)n_new, kMaxAppend);
     if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
     if (per_head) {
         if (B * Hq > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hq=%lld above 65535", (long long)(B * Hq));
@@ -202,10 +207,24 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
 
     if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt, cs), "soft-table kernel launch");
+    AppendHash app;
+    if (n_new > 0) {
+        app.K = K;
+        app.V = V;
+        app.kv_dtype = kv_dtype;
+        app.ids = app_ids;
+        app.vnorm = app_vnorm;
+        app.begin = N - n_new;
+        app.end = N;
+    }
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, app, tables, err_word, counters, unit_max, unit_hist,
+                                        cand_cnt, cs),
+                     "soft-table kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, scores, unit_max, unit_hist, err_word, cs), "score kernel launch");
+    const int64_t fresh_chunk = n_new > 0 ? (N - n_new) / 32 : Ncap / 32;
+    st = cuda_status(launch_score(tables, ids, vnorm, s, fresh_chunk, scores, unit_max, unit_hist, err_word, cs),
+                     "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
     st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");
@@ -291,6 +310,19 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W, const uint8_t* 
 {
     return decode(false, q, q_dtype, W, ids, vnorm, K, V, kv_dtype, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, workspace,
                   workspace_bytes, idx_out, out, scores_out, static_cast<cudaStream_t>(stream));
+}
+
+int socket_decode_append(const void* q, int q_dtype, const uint16_t* W, uint8_t* ids, float* vnorm, const void* K,
+                         const void* V, int kv_dtype, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N,
+                         int64_t d, int L, int P, double tau, int k, int64_t n_new, void* workspace,
+                         size_t workspace_bytes, int32_t* idx_out, float* out, float* scores_out, void* stream)
+{
+    if (n_new < 1) {
+        g_last_error.clear();
+        return fail(SOCKET_EINVAL, "n_new=%lld must be >= 1", (long long)n_new);
+    }
+    return decode(false, q, q_dtype, W, ids, vnorm, K, V, kv_dtype, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, workspace,
+                  workspace_bytes, idx_out, out, scores_out, static_cast<cudaStream_t>(stream), n_new, ids, vnorm);
 }
 
 int socket_decode_per_head(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,

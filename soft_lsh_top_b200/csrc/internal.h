@@ -56,15 +56,31 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
                              int64_t Ncap, int64_t n_begin, int64_t n_end, const uint16_t* W,
                              int L, int P, uint8_t* ids, float* vnorm, cudaStream_t stream);
 
-// Also zeroes the error word, the merge counters, the per-unit max scores,
-// the score histograms and the candidate counters.
-cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
-                               double tau, float* tables, uint32_t* err_word, uint32_t* counters,
-                               uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream);
+// Keys [begin, end) of every kv unit, just written to K and V by the caller,
+// hashed inside the decode step (their ids and norms written) before scoring.
+constexpr int kMaxAppend = 64;
+struct AppendHash {
+    const void* K = nullptr;
+    const void* V = nullptr;
+    int kv_dtype = 0;
+    uint8_t* ids = nullptr;
+    float* vnorm = nullptr;
+    int64_t begin = 0, end = 0;  // empty: nothing hashed
+};
 
+// Also zeroes the error word, the merge counters, the per-unit max scores,
+// the score histograms and the candidate counters, and hashes `app`'s keys.
+cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
+                               double tau, const AppendHash& app, float* tables, uint32_t* err_word,
+                               uint32_t* counters, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt,
+                               cudaStream_t stream);
+
+// fresh_chunk: first 32-key chunk of a unit whose ids the preceding soft-table
+// kernel writes in this step (none: a value >= Ncap / 32); such chunks are
+// not fetched before that kernel has completed.
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* err_word,
-                         cudaStream_t stream);
+                         int64_t fresh_chunk, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
+                         uint32_t* err_word, cudaStream_t stream);
 // Bytes of one key's rotated id row (32 per started block of 32 tables).
 int ids_row_bytes(int L);
 

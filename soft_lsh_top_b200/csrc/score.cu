@@ -100,6 +100,7 @@ struct ScoreArgs {
     int first, last;      // first / last launch of the step (partial sums between)
     int64_t Ncap, N;
     int64_t chunks_per_unit, total_chunks, chunks_per_cta;  // over kv units; per group of CTAs
+    int64_t fresh_chunk;  // chunks from here on get ids in this step: not fetched before the wait
 };
 
 // NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: 32-key chunks
@@ -235,12 +236,19 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         // The stages were read in the previous segment: fence every lane's reads.
         fence_proxy_async_shared();
         __syncwarp();
-        if (lane == 0 && !failed)
-            for (int b = 0; b < min(NS, nbatch); ++b) issue(b);
+        // The first segment's first batches are fetched before the wait below,
+        // unless they reach a chunk whose ids the soft-table kernel writes in
+        // this step (keys hashed on append).
+        const int nfirst = min(NS, nbatch);
+        const bool early = k > 0 || nfirst == 0 || chunk_at(nfirst * KEYS - 1) < a.fresh_chunk;
+        if (lane == 0 && !failed && early)
+            for (int b = 0; b < nfirst; ++b) issue(b);
         if (k == 0) {
             // The soft tables (and, after the first launch, the partial sums)
             // come from the previous kernel on the stream.
             pdl_wait();
+            if (lane == 0 && !failed && !early)
+                for (int b = 0; b < nfirst; ++b) issue(b);
             if (tid == 0)
                 for (int kk = 0; kk < min(kSlots, nseg); ++kk) issue_tables(kk);
         }
@@ -369,8 +377,8 @@ int device_num_sms()
 int ids_row_bytes(int L) { return 32 * ((L + 31) / 32); }
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         float* scores, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* err_word,
-                         cudaStream_t stream)
+                         int64_t fresh_chunk, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
+                         uint32_t* err_word, cudaStream_t stream)
 {
     ScoreArgs a;
     a.tables = tables;
@@ -385,6 +393,7 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     a.Ncap = s.Ncap;
     a.N = s.N;
     a.share = s.share;
+    a.fresh_chunk = fresh_chunk;
     a.chunks_per_unit = (s.N + 31) / 32;
     a.total_chunks = (s.U / s.share) * a.chunks_per_unit;
     // At least one chunk per warp per CTA; at most one CTA per SM; groups of

@@ -39,10 +39,11 @@ constexpr int kHalf = kHeadDim / 2;  // channels per thread of a dot product
 template <typename QT>
 __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L,
-    int P, double tau, float* __restrict__ tables, uint32_t* __restrict__ err_word,
-    uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max, uint32_t* __restrict__ unit_hist,
-    uint32_t* __restrict__ cand_cnt)
+    int P, double tau, const AppendHash app, int64_t Ncap, int share, float* __restrict__ tables,
+    uint32_t* __restrict__ err_word, uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max,
+    uint32_t* __restrict__ unit_hist, uint32_t* __restrict__ cand_cnt)
 {
+    __shared__ uint32_t aid[kMaxAppend][kTablesPerBlock];  // ids of the appended keys (bit p <-> plane p)
     __shared__ double qd[kMaxGroup][kHeadDim];
     __shared__ double qnorm[kMaxGroup];
     __shared__ double sig[kMaxGroup][kTablesPerBlock][kMaxP][2];
@@ -191,21 +192,83 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
             row[(l & 31) + 32] = 0.0f;
         }
     }
+
+    // Keys appended in this step (the step 1 hash of those keys, "Pre-cálculo"):
+    // the ids of this CTA's tables, and for the first table block the norms and
+    // the row padding.  Projections in float32 (one warp per (key, table,
+    // plane), four channels per lane, tree sum); norms in float64.  The first
+    // unit of each kv unit does it; the scoring kernel reads these rows only
+    // after this grid has completed.
+    if (app.end > app.begin && u % share == 0) {
+        const int64_t ukv = u / share;
+        const int nk = (int)(app.end - app.begin);
+        const int Lr = 32 * nblk, pieces = Lr / 16;
+        uint8_t* idu = app.ids + ukv * Ncap * Lr;
+        for (int e = tid; e < nk * kTablesPerBlock; e += kThreads) aid[e / kTablesPerBlock][e % kTablesPerBlock] = 0u;
+        __syncthreads();
+        for (int row = warp; row < nk * nt * P; row += kThreads / 32) {
+            const int key = row / (nt * P), lt = (row / P) % nt, p = row % P;
+            const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
+            const uint2 wq = *reinterpret_cast<const uint2*>(W + ((int64_t)(l0 + lt) * P + p) * kHeadDim + 4 * lane);
+            const float2 w01 = bf16x2_to_f32x2(wq.x), w23 = bf16x2_to_f32x2(wq.y);
+            float4 kf;
+            if (app.kv_dtype == 1) {
+                const uint2 kq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.K) + off);
+                const float2 k01 = bf16x2_to_f32x2(kq.x), k23 = bf16x2_to_f32x2(kq.y);
+                kf = make_float4(k01.x, k01.y, k23.x, k23.y);
+            } else {
+                kf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.K) + off);
+            }
+            float y = fmaf(w23.y, kf.w, fmaf(w23.x, kf.z, fmaf(w01.y, kf.y, w01.x * kf.x)));
+            for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(kFullMask, y, o);
+            if (lane == 0 && y > 0.0f) atomicOr(&aid[key][lt], 1u << p);
+        }
+        __syncthreads();
+        // Byte of table l in key n's rotated row: block l / 32, slot (l - n) mod 32.
+        auto id_byte = [&](int64_t n, int l) -> uint8_t* {
+            const int b = (l & ~31) + (((l & 31) - (int)(n & 31)) & 31);
+            return idu + ((n >> 5) * pieces + (b >> 4)) * 512 + (n & 31) * 16 + (b & 15);
+        };
+        for (int e = tid; e < nk * nt; e += kThreads) {
+            const int key = e / nt, lt = e % nt;
+            *id_byte(app.begin + key, l0 + lt) = (uint8_t)aid[key][lt];
+        }
+        if (blockIdx.y == 0) {
+            const int npad = Lr - L;
+            for (int e = tid; e < nk * npad; e += kThreads) *id_byte(app.begin + e / npad, L + e % npad) = 0;
+            for (int key = warp; key < nk; key += kThreads / 32) {
+                const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
+                float4 vf;
+                if (app.kv_dtype == 1) {
+                    const uint2 vq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.V) + off);
+                    const float2 v01 = bf16x2_to_f32x2(vq.x), v23 = bf16x2_to_f32x2(vq.y);
+                    vf = make_float4(v01.x, v01.y, v23.x, v23.y);
+                } else {
+                    vf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.V) + off);
+                }
+                double s = (double)vf.x * vf.x + (double)vf.y * vf.y + (double)vf.z * vf.z + (double)vf.w * vf.w;
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
+                if (lane == 0) app.vnorm[ukv * Ncap + app.begin + key] = (float)sqrt(s);
+            }
+        }
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
-                               double tau, float* tables, uint32_t* err_word, uint32_t* counters,
-                               uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt, cudaStream_t stream)
+                               double tau, const AppendHash& app, float* tables, uint32_t* err_word,
+                               uint32_t* counters, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt,
+                               cudaStream_t stream)
 {
     dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
     if (q_dtype == 1)
         return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), 0, stream,
-                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, tables, err_word,
-                          counters, unit_max, unit_hist, cand_cnt);
+                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables,
+                          err_word, counters, unit_max, unit_hist, cand_cnt);
     return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), 0, stream, static_cast<const float*>(q), W,
-                      s.G, s.L, s.P, tau, tables, err_word, counters, unit_max, unit_hist, cand_cnt);
+                      s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables, err_word, counters, unit_max, unit_hist,
+                      cand_cnt);
 }
 
 }  // namespace socket_attn

@@ -96,6 +96,14 @@ def test_decode_rejects(lib, entry, kw, status):
     assert lib.socket_last_error().decode() != ""
 
 
+@pytest.mark.parametrize("n_new", [0, -1, 65, 9])
+def test_decode_append_rejects_n_new(lib, n_new):
+    # N = 8 keys: n_new may not exceed N, nor 64, nor be below 1.
+    assert lib.socket_decode_append(P16, 1, P16, P16, P16, P16, P16, 1, 1, 4, 1, 64, 8, 128, 4, 8, 0.5, 8, n_new,
+                                    P16, 1 << 30, P16, P16, None, None) == EINVAL
+    assert "n_new" in lib.socket_last_error().decode()
+
+
 def test_per_head_rejects_too_many_query_heads(lib):
     # 4096 x 32 query-head units exceed the limit; 4096 x 2 kv units would not.
     assert decode(lib, "socket_decode_per_head", B=4096, Hq=32, Hkv=2) == EUNSUP

@@ -12,7 +12,7 @@ import torch
 import oracle
 import soft_lsh_top_b200 as sk
 import workloads as wl
-from parity import (check_decode, check_hash, gpu_decode, gpu_hash, ids_to_rows, oracle_hash_units,
+from parity import (check_decode, check_hash, gpu_decode, gpu_hash, ids_to_rows, oracle_hash_units, rows_to_ids,
                     substitute_units)
 
 pytestmark = pytest.mark.gpu
@@ -89,6 +89,40 @@ def test_hash_in_ranges_matches_oracle(case):
     orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units)
     check_hash(ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy(), vnorm.reshape(w.U, w.ncap).cpu().numpy(),
                orc_ids, orc_vn, margin, 0, w.N)
+
+
+@pytest.mark.parametrize("case", ["bf16_single_head", "odd_group3_p5", "f32_group2_p6", "bf16_l80_p7",
+                                  "bf16_group16"])
+def test_decode_append_hashes_and_decodes(case):
+    """socket_decode_append: the step hashes the keys just appended (1, 5, then
+    33 keys, so chunk boundaries are crossed) and decodes over them.  The ids
+    and norms of every key match the oracle's hash (within the float32
+    exemption band), and each step's scores, selection and output match the
+    oracle run on the index the step saw."""
+    w = SMALL[case]
+    inp = wl.make_inputs(w, DEV)
+    B = inp["K"].shape[0]
+    ids, vnorm = sk.alloc_cache_index(B, w.Hkv, w.ncap, w.L, DEV)
+    ids.zero_()
+    vnorm.zero_()
+    n = w.N - 39
+    sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vnorm, 0, n)
+    sk.socket_hash_check()
+    ws, idx, out = sk.alloc_decode_buffers(B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, DEV)
+    units = list(range(w.U))
+    for n_new in (1, 5, 33):
+        n += n_new
+        scores = torch.full((B, w.Hkv, w.ncap), float("nan"), dtype=torch.float32, device=DEV)
+        sk.socket_decode_append(inp["q"], inp["W"], ids, vnorm, inp["K"], inp["V"], n, w.tau, w.k, n_new, ws, idx,
+                                out, scores_out=scores)
+        torch.cuda.synchronize()
+        assert sk.read_device_error(ws) == 0
+        g_ids = rows_to_ids(ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy(), w.L)
+        g_vn = vnorm.reshape(w.U, w.ncap).cpu().numpy()
+        check_decode(inp, w, g_ids, g_vn, units, idx, out, scores, N=n)
+    orc_ids, orc_vn, margin = oracle_hash_units(inp, w, units, 0, n)
+    check_hash(ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy(), vnorm.reshape(w.U, w.ncap).cpu().numpy(),
+               orc_ids, orc_vn, margin, 0, n)
 
 
 def test_decode_matches_oracle(small):
