@@ -445,21 +445,44 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                                 wa.k, 1, ws_a, idx_a, out_a)
 
     append = {"what": "64 decode steps that each append one key (hash + decode), append-mix workload: "
-                      "socket_hash_keys + socket_decode vs the fused socket_decode_append; direct calls",
+                      "socket_hash_keys + socket_decode vs the fused socket_decode_append; each variant's 64 "
+                      "steps captured in one CUDA graph and replayed",
               "workload": wa.name, "B": wa.B, "Hq": wa.Hq, "Hkv": wa.Hkv, "N": wa.N, "L": wa.L, "P": wa.P,
               "k": wa.k}
     for name, fn in (("two_calls", two_calls), ("fused", fused)):
-        for t in range(wa.appends):  # warm-up (re-hashing a key writes the same bytes)
+        for t in range(wa.appends):  # warm-up
             fn(t)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for t in range(wa.appends):
+                fn(t)
+        g.replay()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         a0.record()
-        for t in range(wa.appends):
-            fn(t)
+        for _ in range(3):
+            g.replay()
         a1.record()
         torch.cuda.synchronize()
-        ms = a0.elapsed_time(a1)
+        ms = a0.elapsed_time(a1) / 3
         append[name] = {"steps_per_s": wa.appends / (ms * 1e-3), "us_per_step": 1e3 * ms / wa.appends}
+        del g
+    # Per-kernel times of the decode step of each variant (events between its kernels).
+    for name, fn in (("two_calls", two_calls), ("fused", fused)):
+        ev_a = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(wa.appends)]
+        for row in ev_a:
+            for e in row:
+                e.record()
+        torch.cuda.synchronize()
+        for t in range(wa.appends):
+            sk.socket_set_step_events(ev_a[t])
+            fn(t)
+        torch.cuda.synchronize()
+        sk.socket_set_step_events([])
+        append[name]["decode_kernels_us"] = {n: 1e3 * statistics.fmean(ev_a[t][i].elapsed_time(ev_a[t][i + 1])
+                                                                       for t in range(wa.appends))
+                                             for i, n in enumerate(names)}
     sk.socket_hash_check()
     assert sk.read_device_error(ws_a) == 0
     del ia, ids_a, vn_a, ws_a, idx_a, out_a

@@ -18,18 +18,18 @@ namespace socket_attn {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kTablesPerBlock = 2;
+constexpr int kMaxTablesPerBlock = 8;  // tables per CTA: 2, 4 or 8, chosen at launch
 constexpr int kMaxGroup = 16;
 constexpr int kMaxP = 8;
 constexpr int kHalf = kHeadDim / 2;  // channels per thread of a dot product
+constexpr int kWRow = kHeadDim + 8;  // padded bf16 hyperplane row in shared memory (272 bytes)
 
-// Grid: (U, ceil(L / kTablesPerBlock)).  Block: kThreads.
-//   1. two threads per (head, table, plane) row load the two halves of the
-//      hyperplane row W_{l,p} (issued first, so they are in flight while the
-//      query is staged); the unit's G query rows are widened to float64 and
-//      their norms taken;
-//   2. each pair forms z = <W_{l,p}, q_h>/||q_h|| (its halves added with one
-//      shuffle) and the two per-plane factors sigmoid(+-2z/tau);
+// Grid: (U, ceil(L / tpb)).  Block: kThreads.  Dynamic shared memory sized by G and tpb.
+//   1. the CTA's hyperplane rows are staged in shared memory; the unit's G
+//      query rows are widened to float64 and their norms taken;
+//   2. two threads per (head, table, plane) row form z = <W_{l,p}, q_h>/||q_h||
+//      (their channel halves added with one shuffle) and the two per-plane
+//      factors sigmoid(+-2z/tau), both from one exponential;
 //   3. the per-plane factors of planes 0-3 and 4-7 are multiplied into two
 //      16-entry nibble tables per (head, table);
 //   4. each entry T_l(b) = sum_h lo_h(b & 15) * hi_h(b >> 4) is rounded once
@@ -39,19 +39,23 @@ constexpr int kHalf = kHeadDim / 2;  // channels per thread of a dot product
 template <typename QT>
 __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L,
-    int P, double tau, const AppendHash app, int64_t Ncap, int share, float* __restrict__ tables,
+    int P, int tpb, double tau, const AppendHash app, int64_t Ncap, int share, float* __restrict__ tables,
     uint32_t* __restrict__ err_word, uint32_t* __restrict__ counters, uint32_t* __restrict__ unit_max,
     uint32_t* __restrict__ unit_hist, uint32_t* __restrict__ cand_cnt)
 {
-    __shared__ uint32_t aid[kMaxAppend][kTablesPerBlock];  // ids of the appended keys (bit p <-> plane p)
-    __shared__ double qd[kMaxGroup][kHeadDim];
-    __shared__ double qnorm[kMaxGroup];
-    __shared__ double sig[kMaxGroup][kTablesPerBlock][kMaxP][2];
-    __shared__ double nib[kMaxGroup][kTablesPerBlock][2][16];
+    __shared__ uint32_t aid[kMaxAppend][kMaxTablesPerBlock];  // ids of the appended keys (bit p <-> plane p)
+    extern __shared__ __align__(16) char st_dyn[];
+    uint16_t* wsm = reinterpret_cast<uint16_t*>(st_dyn);  // [tpb * P][kWRow] bf16 hyperplane rows
+    double* qd = reinterpret_cast<double*>(st_dyn + tpb * P * kWRow * 2);  // [G][kHeadDim]
+    double* qnorm = qd + G * kHeadDim;               // [G]: 2 / (tau ||q_h||)
+    double* sig = qnorm + G;                         // [G][tpb][kMaxP][2]
+    double* nib = sig + G * tpb * kMaxP * 2;         // [G][tpb][2][16]
+    auto SIG = [&](int h, int lt, int p, int s) -> double& { return sig[((h * tpb + lt) * kMaxP + p) * 2 + s]; };
+    auto NIB = [&](int h, int lt, int hi, int v) -> double& { return nib[((h * tpb + lt) * 2 + hi) * 16 + v]; };
 
     const int64_t u = blockIdx.x;  // the unit's query rows are u G .. u G + G - 1 of [B][Hq]
-    const int l0 = blockIdx.y * kTablesPerBlock;
-    const int nt = min(kTablesPerBlock, L - l0);
+    const int l0 = blockIdx.y * tpb;
+    const int nt = min(tpb, L - l0);
     const int NB = 1 << P;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
@@ -74,23 +78,19 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     for (int i = 0; i < (int)(sizeof(qv) / sizeof(qv[0])); ++i)
         if (tid + i * kThreads < npieces) qv[i] = __ldg(qu4 + tid + i * kThreads);
 
-    const int rows = G * nt * P;
-    const int half = tid & 1;
-    int r = tid >> 1;
-    uint4 wv[kHalf / 8];
-    auto load_w = [&](int row) {
-        const int lt = (row / P) % nt, p = row % P;
-        const uint4* w = reinterpret_cast<const uint4*>(W + ((int64_t)(l0 + lt) * P + p) * kHeadDim + half * kHalf);
-#pragma unroll
-        for (int c = 0; c < kHalf / 8; ++c) wv[c] = __ldg(w + c);
-    };
-    if (r < rows) load_w(r);
+    // This CTA's hyperplane rows (nt tables x P planes, contiguous in W),
+    // staged once in shared memory with rows padded to 272 bytes so that a
+    // warp's 16-byte reads of 16 rows x 2 halves fall on distinct banks.
+    const int wrows = nt * P;
+    const uint4* wsrc = reinterpret_cast<const uint4*>(W + (int64_t)l0 * P * kHeadDim);
+    for (int e = tid; e < wrows * (kHeadDim / 8); e += kThreads)
+        *reinterpret_cast<uint4*>(wsm + (e >> 4) * kWRow + (e & 15) * 8) = __ldg(wsrc + e);
 
 #pragma unroll
     for (int i = 0; i < (int)(sizeof(qv) / sizeof(qv[0])); ++i) {
         const int piece = tid + i * kThreads;
         if (piece < npieces) {
-            double* dst = &qd[0][0] + piece * kPer16;  // qd rows are contiguous
+            double* dst = qd + piece * kPer16;  // qd rows are contiguous
             const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -105,48 +105,58 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         }
     }
     __syncthreads();
+    // Per head, the factor taking <W_{l,p}, q_h> to the sigmoid argument
+    // 2 z / tau with z = <W_{l,p}, q_h> / ||q_h|| (0 for a zero query).
     for (int h = warp; h < G; h += kThreads / 32) {
         double s = 0.0;
-        for (int j = lane; j < kHeadDim; j += 32) s += qd[h][j] * qd[h][j];
+        for (int j = lane; j < kHeadDim; j += 32) s += qd[h * kHeadDim + j] * qd[h * kHeadDim + j];
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
-        if (lane == 0) qnorm[h] = sqrt(s);
+        if (lane == 0) qnorm[h] = (s > 0.0 && tau > 0.0) ? 2.0 / (tau * sqrt(s)) : 0.0;
     }
     __syncthreads();
 
-    // Every pair runs the same number of rounds so the shuffle sees both halves.
-    for (; r < (rows + kThreads / 2 - 1) / (kThreads / 2) * (kThreads / 2); r += kThreads / 2) {
+    // Rows ordered (head, table, plane); thread pair (2r, 2r + 1) takes the two
+    // channel halves of row r, and every pair runs the same number of rounds
+    // so the shuffle sees both halves.
+    const int rows = G * wrows;
+    const int half = tid & 1;
+    for (int r = tid >> 1; r < (rows + kThreads / 2 - 1) / (kThreads / 2) * (kThreads / 2); r += kThreads / 2) {
         const bool live = r < rows;
-        const int h = live ? r / (nt * P) : 0;
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        const int h = live ? r / wrows : 0, wr = live ? r - h * wrows : 0;
+        double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
         if (live) {
-            const double* qh = qd[h] + half * kHalf;
+            const double* qh = qd + h * kHeadDim + half * kHalf;
+            const uint16_t* wh = wsm + wr * kWRow + half * kHalf;
 #pragma unroll
             for (int c = 0; c < kHalf / 8; ++c) {
-                const uint32_t words[4] = {wv[c].x, wv[c].y, wv[c].z, wv[c].w};
+                const uint4 wq = *reinterpret_cast<const uint4*>(wh + c * 8);
+                const uint32_t words[4] = {wq.x, wq.y, wq.z, wq.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 f = bf16x2_to_f32x2(words[i]);
-                    acc[i] = fma((double)f.x, qh[c * 8 + 2 * i], acc[i]);
-                    acc[i] = fma((double)f.y, qh[c * 8 + 2 * i + 1], acc[i]);
+                    acc[2 * i] = fma((double)f.x, qh[c * 8 + 2 * i], acc[2 * i]);
+                    acc[2 * i + 1] = fma((double)f.y, qh[c * 8 + 2 * i + 1], acc[2 * i + 1]);
                 }
             }
         }
-        double y = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        double y = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         y += __shfl_xor_sync(kFullMask, y, 1);
         if (live && half == 0) {
-            const int lt = (r / P) % nt, p = r % P;
+            const int lt = wr / P, p = wr - lt * P;
             if (tau == 0.0) {
                 // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
-                sig[h][lt][p][1] = y > 0.0 ? 1.0 : 0.0;
-                sig[h][lt][p][0] = y > 0.0 ? 0.0 : 1.0;
+                SIG(h, lt, p, 1) = y > 0.0 ? 1.0 : 0.0;
+                SIG(h, lt, p, 0) = y > 0.0 ? 0.0 : 1.0;
             } else {
-                const double z = qnorm[h] > 0.0 ? y / qnorm[h] : 0.0;
-                const double x = 2.0 * z / tau;
-                sig[h][lt][p][1] = 1.0 / (1.0 + exp(-x));  // sign +1: bit set
-                sig[h][lt][p][0] = 1.0 / (1.0 + exp(x));   // sign -1: bit clear
+                // sigmoid(+-x) from one exponential: e = exp(-|x|),
+                // sigmoid(|x|) = 1 / (1 + e), sigmoid(-|x|) = e / (1 + e).
+                const double x = y * qnorm[h];
+                const double e = exp(-fabs(x));
+                const double big = 1.0 / (1.0 + e), small = e * big;
+                SIG(h, lt, p, 1) = x >= 0.0 ? big : small;  // sign +1: bit set
+                SIG(h, lt, p, 0) = x >= 0.0 ? small : big;  // sign -1: bit clear
             }
         }
-        if (r + kThreads / 2 < rows) load_w(r + kThreads / 2);
     }
     __syncthreads();
 
@@ -156,8 +166,8 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         const int h = e / (nt * 32), lt = (e / 32) % nt, hi = (e / 16) & 1, v = e & 15;
         double prod = 1.0;
         const int p0 = hi ? 4 : 0, p1 = hi ? P : plo;
-        for (int p = p0; p < p1; ++p) prod *= sig[h][lt][p][(v >> (p - p0)) & 1];
-        nib[h][lt][hi][v] = prod;
+        for (int p = p0; p < p1; ++p) prod *= SIG(h, lt, p, (v >> (p - p0)) & 1);
+        NIB(h, lt, hi, v) = prod;
     }
     __syncthreads();
 
@@ -173,15 +183,43 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     }
     const int nblk = (L + 31) / 32;
     float* tu = tables + u * nblk * (int64_t)NB * 64;
-    for (int e = tid; e < nt * NB; e += kThreads) {
-        const int lt = e % nt, bucket = e / nt;
-        double acc = 0.0;
-        for (int h = 0; h < G; ++h)
-            acc += nib[h][lt][0][bucket & 15] * nib[h][lt][1][bucket >> 4];
-        const int l = l0 + lt;
-        float* row = tu + ((int64_t)(l >> 5) * NB + bucket) * 64;
-        row[l & 31] = (float)acc;
-        row[(l & 31) + 32] = (float)acc;
+    // One bucket of all nt tables per thread: the row's nt adjacent columns
+    // (and their copies 32 columns on) go out as whole vector stores.  tpb
+    // divides 32 and l0 is a multiple of it, so the CTA's tables sit in one
+    // 32-table block and its columns start on an nt-float boundary.
+    for (int bucket = tid; bucket < NB; bucket += kThreads) {
+        float vals[kMaxTablesPerBlock];
+#pragma unroll
+        for (int lt = 0; lt < kMaxTablesPerBlock; ++lt) {
+            double acc = 0.0;
+            if (lt < nt)
+                for (int h = 0; h < G; ++h) acc += NIB(h, lt, 0, bucket & 15) * NIB(h, lt, 1, bucket >> 4);
+            vals[lt] = (float)acc;
+        }
+        float* row = tu + ((int64_t)(l0 >> 5) * NB + bucket) * 64 + (l0 & 31);
+        if (nt == 8) {
+            const float4 a = make_float4(vals[0], vals[1], vals[2], vals[3]);
+            const float4 b = make_float4(vals[4], vals[5], vals[6], vals[7]);
+            *reinterpret_cast<float4*>(row) = a;
+            *reinterpret_cast<float4*>(row + 4) = b;
+            *reinterpret_cast<float4*>(row + 32) = a;
+            *reinterpret_cast<float4*>(row + 36) = b;
+        } else if (nt == 4) {
+            const float4 a = make_float4(vals[0], vals[1], vals[2], vals[3]);
+            *reinterpret_cast<float4*>(row) = a;
+            *reinterpret_cast<float4*>(row + 32) = a;
+        } else if (nt == 2) {
+            const float2 a = make_float2(vals[0], vals[1]);
+            *reinterpret_cast<float2*>(row) = a;
+            *reinterpret_cast<float2*>(row + 32) = a;
+        } else {
+#pragma unroll
+            for (int lt = 0; lt < kMaxTablesPerBlock; ++lt)
+                if (lt < nt) {
+                    row[lt] = vals[lt];
+                    row[lt + 32] = vals[lt];
+                }
+        }
     }
     if (blockIdx.y == 0) {
         const int npad = 32 * nblk - L;
@@ -204,13 +242,12 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         const int nk = (int)(app.end - app.begin);
         const int Lr = 32 * nblk, pieces = Lr / 16;
         uint8_t* idu = app.ids + ukv * Ncap * Lr;
-        for (int e = tid; e < nk * kTablesPerBlock; e += kThreads) aid[e / kTablesPerBlock][e % kTablesPerBlock] = 0u;
+        for (int e = tid; e < nk * kMaxTablesPerBlock; e += kThreads) aid[e / kMaxTablesPerBlock][e % kMaxTablesPerBlock] = 0u;
         __syncthreads();
-        for (int row = warp; row < nk * nt * P; row += kThreads / 32) {
-            const int key = row / (nt * P), lt = (row / P) % nt, p = row % P;
+        for (int key = 0; key < nk; ++key) {
+            // The key row once per warp (four channels per lane); the CTA's
+            // hyperplane rows from shared memory.
             const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
-            const uint2 wq = *reinterpret_cast<const uint2*>(W + ((int64_t)(l0 + lt) * P + p) * kHeadDim + 4 * lane);
-            const float2 w01 = bf16x2_to_f32x2(wq.x), w23 = bf16x2_to_f32x2(wq.y);
             float4 kf;
             if (app.kv_dtype == 1) {
                 const uint2 kq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.K) + off);
@@ -219,9 +256,13 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
             } else {
                 kf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.K) + off);
             }
-            float y = fmaf(w23.y, kf.w, fmaf(w23.x, kf.z, fmaf(w01.y, kf.y, w01.x * kf.x)));
-            for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(kFullMask, y, o);
-            if (lane == 0 && y > 0.0f) atomicOr(&aid[key][lt], 1u << p);
+            for (int wr = warp; wr < wrows; wr += kThreads / 32) {
+                const uint2 wq = *reinterpret_cast<const uint2*>(wsm + wr * kWRow + 4 * lane);
+                const float2 w01 = bf16x2_to_f32x2(wq.x), w23 = bf16x2_to_f32x2(wq.y);
+                float y = fmaf(w23.y, kf.w, fmaf(w23.x, kf.z, fmaf(w01.y, kf.y, w01.x * kf.x)));
+                for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(kFullMask, y, o);
+                if (lane == 0 && y > 0.0f) atomicOr(&aid[key][wr / P], 1u << (wr % P));
+            }
         }
         __syncthreads();
         // Byte of table l in key n's rotated row: block l / 32, slot (l - n) mod 32.
@@ -261,14 +302,46 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                uint32_t* counters, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt,
                                cudaStream_t stream)
 {
-    dim3 grid((unsigned)s.U, (unsigned)((s.L + kTablesPerBlock - 1) / kTablesPerBlock));
+    // Tables per CTA: the fewest (2, 4, 8) whose grid fits in one wave of
+    // resident CTAs, so many units or tables do not queue in waves.
+    const int qi = q_dtype == 1 ? 1 : 0;
+    auto kern = qi ? (void*)soft_tables_kernel<uint16_t> : (void*)soft_tables_kernel<float>;
+    // Resident CTAs per SM by (q dtype, G, log2 tpb - 1), looked up once per process and device.
+    static thread_local int cached_dev = -1;
+    static thread_local int per_sm_cache[2][kMaxGroup + 1][3];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != cached_dev) {
+        for (auto& a : per_sm_cache)
+            for (auto& b : a)
+                for (int& c : b) c = -1;
+        for (void* kf : {(void*)soft_tables_kernel<uint16_t>, (void*)soft_tables_kernel<float>}) {
+            const int max_smem = (int)sizeof(double) * kMaxGroup * (kHeadDim + 1 + kMaxTablesPerBlock * (kMaxP * 2 + 32)) +
+                                 kMaxTablesPerBlock * kMaxP * kWRow * 2;
+            cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+            if (e != cudaSuccess) return e;
+        }
+        cached_dev = dev;
+    }
+    int tpb = 2, smem = 0;
+    for (int li = 0;; ++li, tpb *= 2) {
+        smem = (int)sizeof(double) * s.G * (kHeadDim + 1 + tpb * (kMaxP * 2 + 32)) + tpb * s.P * kWRow * 2;
+        int& per_sm = per_sm_cache[qi][s.G][li];
+        if (per_sm < 0) {
+            cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+            if (e != cudaSuccess) return e;
+        }
+        const int64_t ctas = s.U * ((s.L + tpb - 1) / tpb);
+        if (tpb == kMaxTablesPerBlock || ctas <= (int64_t)per_sm * device_num_sms()) break;
+    }
+    dim3 grid((unsigned)s.U, (unsigned)((s.L + tpb - 1) / tpb));
     if (q_dtype == 1)
-        return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), 0, stream,
-                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables,
+        return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), (size_t)smem, stream,
+                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tpb, tau, app, s.Ncap, s.share, tables,
                           err_word, counters, unit_max, unit_hist, cand_cnt);
-    return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), 0, stream, static_cast<const float*>(q), W,
-                      s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables, err_word, counters, unit_max, unit_hist,
-                      cand_cnt);
+    return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), (size_t)smem, stream, static_cast<const float*>(q),
+                      W, s.G, s.L, s.P, tpb, tau, app, s.Ncap, s.share, tables, err_word, counters, unit_max,
+                      unit_hist, cand_cnt);
 }
 
 }  // namespace socket_attn
