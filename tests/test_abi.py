@@ -35,7 +35,9 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for want in ("socket_hash_keys", "socket_decode", "socket_decode_workspace_size", "socket_last_error"):
+    for want in ("socket_hash_keys", "socket_hash_check", "socket_decode", "socket_decode_workspace_size",
+                 "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_decode_append",
+                 "socket_last_error"):
         assert want in names
 
 
