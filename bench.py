@@ -483,6 +483,17 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         append[name]["decode_kernels_us"] = {n: 1e3 * statistics.fmean(ev_a[t][i].elapsed_time(ev_a[t][i + 1])
                                                                        for t in range(wa.appends))
                                              for i, n in enumerate(names)}
+    # Prefill of this workload (L * P = 480 hyperplanes: two tensor-core passes).
+    h0.record()
+    for _ in range(3):
+        sk.socket_hash_keys(ia["K"], ia["V"], ia["W"], ids_a, vn_a, 0, wa.N)
+    h1.record()
+    torch.cuda.synchronize()
+    pre_ms = h0.elapsed_time(h1) / 3
+    pre_keys = wa.B * wa.Hkv * wa.N
+    pre_bytes = pre_keys * (2 * wa.d * wa.elem_bytes + sk.socket_ids_row_bytes(wa.L) + 4)
+    append["prefill"] = {"keys": pre_keys, "ms": pre_ms, "algorithmic_bytes": pre_bytes,
+                         "gbs": pre_bytes / (pre_ms * 1e-3) / 1e9}
     sk.socket_hash_check()
     assert sk.read_device_error(ws_a) == 0
     del ia, ids_a, vn_a, ws_a, idx_a, out_a

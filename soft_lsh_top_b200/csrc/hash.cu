@@ -262,8 +262,10 @@ __global__ __launch_bounds__(kMThreads) void hash_mma_kernel(const uint16_t* __r
 
 
 // ---------------------------------------------------------------------------
-// bfloat16 keys on the fifth-generation tensor cores (tcgen05), for L*P <= 256
-// hyperplanes.  The projections of a 128-key tile on every hyperplane are one
+// bfloat16 keys on the fifth-generation tensor cores (tcgen05), in passes over
+// whole 32-table blocks of at most 256 hyperplanes (one pass when L*P <= 256;
+// a pass writes the 16-byte pieces of its own blocks, the first also the
+// value norms).  The projections of a 128-key tile on every hyperplane are one
 // UMMA product per 16 channels, y [128 keys x Np planes] = K_tile * W^T
 // (bf16 in, fp32 accumulate in tensor memory), with Np = L*P rounded up to a
 // multiple of 16 (the extra hyperplane rows are zero-filled by the copy and
@@ -373,7 +375,10 @@ struct HashUArgs {
     uint8_t* ids;
     float* vnorm;
     int64_t Ncap, n_begin, n_end;
-    int L, P, Np;
+    int L, P, Np;      // tables of this pass, planes per table, hyperplane rows rounded up to 16
+    int blk0;          // first 32-table block of this pass
+    int pieces_full;   // 16-byte pieces of a key's whole id row
+    int norms;         // this pass also loads V and writes the value norms
     int tiles_per_unit;
     int64_t tiles;
 };
@@ -433,7 +438,7 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
             for (int64_t t = blockIdx.x; t < a.tiles; t += gridDim.x, ++i) {
                 const int s = i % kUStages, g = i & 1;
                 if (!mbar_wait_bounded(&empty[s], ((i / kUStages) & 1) ^ 1, kUMaxPolls) ||
-                    !mbar_wait_bounded(&vempty[g], ((i >> 1) & 1) ^ 1, kUMaxPolls)) {
+                    (a.norms && !mbar_wait_bounded(&vempty[g], ((i >> 1) & 1) ^ 1, kUMaxPolls))) {
                     ok = false;
                     break;
                 }
@@ -442,16 +447,19 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
                 mbar_arrive_expect_tx(&full[s], kUTileBytes);
                 tma_load_3d(sK + s * kUTileBytes, &tmK, 0, n0, u, &full[s]);
                 tma_load_3d(sK + s * kUTileBytes + kUBoxBytes, &tmK, 64, n0, u, &full[s]);
-                mbar_arrive_expect_tx(&vfull[g], kUTileBytes);
-                tma_load_3d(sV + g * kUTileBytes, &tmV, 0, n0, u, &vfull[g]);
-                tma_load_3d(sV + g * kUTileBytes + kUBoxBytes, &tmV, 64, n0, u, &vfull[g]);
+                if (a.norms) {
+                    mbar_arrive_expect_tx(&vfull[g], kUTileBytes);
+                    tma_load_3d(sV + g * kUTileBytes, &tmV, 0, n0, u, &vfull[g]);
+                    tma_load_3d(sV + g * kUTileBytes + kUBoxBytes, &tmV, 64, n0, u, &vfull[g]);
+                }
             }
             if (!ok) atomicOr(&g_hash_err, 1u);
             // The last copies of every stage and buffer have landed before the CTA exits.
             mbar_wait_bounded(&wbar, 0, kUMaxPolls);
             for (int j = max(0, i - kUStages); j < i; ++j)
                 mbar_wait_bounded(&full[j % kUStages], (j / kUStages) & 1, kUMaxPolls);
-            for (int j = max(0, i - 2); j < i; ++j) mbar_wait_bounded(&vfull[j & 1], (j >> 1) & 1, kUMaxPolls);
+            if (a.norms)
+                for (int j = max(0, i - 2); j < i; ++j) mbar_wait_bounded(&vfull[j & 1], (j >> 1) & 1, kUMaxPolls);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -504,7 +512,7 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
             const int64_t u = t / a.tiles_per_unit;
             const int64_t n = a.n_begin + (t % a.tiles_per_unit) * kUKeys + r;
             const bool live = n < a.n_end;
-            const bool ok = mbar_wait_bounded(&vfull[grp], j & 1, kUMaxPolls) &&
+            const bool ok = (!a.norms || mbar_wait_bounded(&vfull[grp], j & 1, kUMaxPolls)) &&
                             mbar_wait_bounded(&tfull[grp], j & 1, kUMaxPolls);
             if (!__all_sync(kFullMask, ok)) {
                 if (lane == 0) atomicOr(&g_hash_err, 1u);
@@ -531,7 +539,7 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[grp]);
 
-            if (live) {
+            if (a.norms && live) {
                 // Value norm: squares summed in float64 (exact squares), rounded once.
                 double s0 = 0.0, s1 = 0.0;
 #pragma unroll
@@ -550,13 +558,17 @@ __global__ __launch_bounds__(kUThreads, 1) void hash_umma_kernel(const __grid_co
                 }
                 a.vnorm[u * a.Ncap + n] = (float)sqrt(s0 + s1);
             }
-            fence_proxy_async_shared();  // these reads precede the next tensor copy into the buffer
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&vempty[grp]);
+            if (a.norms) {
+                fence_proxy_async_shared();  // these reads precede the next tensor copy into the buffer
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vempty[grp]);
+            }
             if (!live) continue;
 
-            // Rotated id row: slot s of block c holds table 32c + (s + n) mod 32.
-            uint8_t* dst = a.ids + u * a.Ncap * Lr + (n >> 5) * pieces * 512 + (n & 31) * 16;
+            // Rotated id row: slot s of block c holds table 32c + (s + n) mod 32;
+            // this pass writes the pieces of its own blocks.
+            uint8_t* dst = a.ids + u * a.Ncap * (a.pieces_full * 16) +
+                           ((n >> 5) * a.pieces_full + 2 * a.blk0) * 512 + (n & 31) * 16;
             const int rot = (int)(n & 31);
             if (a.P == 8) {
                 // One byte per hyperplane group: the sign words are the ids in
@@ -661,10 +673,13 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
                              float* vnorm, cudaStream_t stream)
 {
     const int64_t nkeys = n_end - n_begin;
-    const int planes = L * P;
     // SOCKET_HASH_NO_TCGEN05 in the environment selects the warp-level MMA kernel instead.
     static const bool tcgen05_on = getenv("SOCKET_HASH_NO_TCGEN05") == nullptr;
-    if (kv_dtype == 1 && planes <= kUMaxPlanes && tcgen05_on) {
+    if (kv_dtype == 1 && tcgen05_on) {
+        // Passes over whole 32-table blocks of at most 256 hyperplanes each
+        // (one pass when L * P <= 256); the first also writes the value norms.
+        const int tpp = 32 * max(1, kUMaxPlanes / (32 * P));
+        const int npass = (L + tpp - 1) / tpp;  // <= 4
         HashUArgs a;
         a.V = static_cast<const uint16_t*>(V);
         a.ids = ids;
@@ -672,21 +687,34 @@ cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t
         a.Ncap = Ncap;
         a.n_begin = n_begin;
         a.n_end = n_end;
-        a.L = L;
         a.P = P;
-        a.Np = (planes + 15) / 16 * 16;
+        a.pieces_full = 2 * ((L + 31) / 32);
         a.tiles_per_unit = (int)((nkeys + kUKeys - 1) / kUKeys);
         a.tiles = B * Hkv * a.tiles_per_unit;
-        CUtensorMap tmK, tmV, tmW;
-        if (encode_rows(&tmK, K, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys) &&
-            encode_rows(&tmV, V, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys) &&
-            encode_rows(&tmW, W, (uint64_t)planes, 1, (uint32_t)a.Np)) {
-            const int smem = 1024 + a.Np * 256 + (kUStages + 2) * (int)kUTileBytes + 2 * kUKeys * kUSgnStride * 4;
-            cudaError_t e = cudaFuncSetAttribute(hash_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        CUtensorMap tmK, tmV, tmW[4];
+        bool ok = npass <= 4 && encode_rows(&tmK, K, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys) &&
+                  encode_rows(&tmV, V, (uint64_t)Ncap, (uint64_t)(B * Hkv), kUKeys);
+        for (int ps = 0; ok && ps < npass; ++ps) {
+            const int lp = min(tpp, L - ps * tpp);
+            ok = encode_rows(&tmW[ps], W + (int64_t)ps * tpp * P * kHeadDim, (uint64_t)(lp * P), 1,
+                             (uint32_t)((lp * P + 15) / 16 * 16));
+        }
+        if (ok) {
+            const int max_smem = 1024 + kUMaxPlanes * 256 + (kUStages + 2) * (int)kUTileBytes + 2 * kUKeys * kUSgnStride * 4;
+            cudaError_t e = cudaFuncSetAttribute(hash_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
             if (e != cudaSuccess) return e;
             const int grid = (int)min64(device_num_sms(), a.tiles);
-            hash_umma_kernel<<<grid, kUThreads, smem, stream>>>(tmK, tmV, tmW, a);
-            return cudaGetLastError();
+            for (int ps = 0; ps < npass; ++ps) {
+                a.blk0 = ps * tpp / 32;
+                a.L = min(tpp, L - ps * tpp);
+                a.Np = (a.L * P + 15) / 16 * 16;
+                a.norms = ps == 0;
+                const int smem = 1024 + a.Np * 256 + (kUStages + 2) * (int)kUTileBytes + 2 * kUKeys * kUSgnStride * 4;
+                hash_umma_kernel<<<grid, kUThreads, smem, stream>>>(tmK, tmV, tmW[ps], a);
+                e = cudaGetLastError();
+                if (e != cudaSuccess) return e;
+            }
+            return cudaSuccess;
         }
     }
     if (kv_dtype == 1) {
