@@ -34,6 +34,9 @@ MUTANTS = {
     "attention_unnormalised_weights": ("double w = exp(logit[i] - mx) / total;", "double w = exp(logit[i] - mx);"),
     "attention_values_from_keys": ("out[(int64_t)h * d + j] += w * load_elem(V,", "out[(int64_t)h * d + j] += w * load_elem(K,"),
     "decode_every_head_uses_head0": ("oracle_soft_assign((const char*)q + (size_t)h * d", "oracle_soft_assign((const char*)q + (size_t)0 * d"),
+    "hard_query_sign_flipped": ("if (y > 0.0) hb |= 1 << p;", "if (y < 0.0) hb |= 1 << p;"),
+    "hard_bit_order_reversed": ("if (y > 0.0) hb |= 1 << p;", "if (y > 0.0) hb |= 1 << (P - 1 - p);"),
+    "hard_mass_off_the_bucket": ("prob[(int64_t)l * nb + b] = b == hb ? 1.0 : 0.0;", "prob[(int64_t)l * nb + b] = b == hb ? 0.0 : 1.0;"),
 }
 
 
@@ -60,3 +63,26 @@ def test_mutant_is_caught(name, tmp_path):
 
 def test_unmutated_passes_every_pin():
     assert _failures(oracle.load()) == []
+
+
+def test_per_head_pin_catches_heads_on_the_wrong_kv_unit(monkeypatch):
+    """The per-head decode is a composition in Python; plant the plausible
+    mistake there (units repeated as a tile, so head g of unit u reads another
+    unit's keys) and check its pin notices."""
+    import numpy as np
+
+    import oracle_pins
+
+    def mutant(q, W, L, P, tau, ids, vnorm_f32, K, V, n, k, want_scores=True, lib=None):
+        qs = np.asarray(q)
+        U, G, d = qs.shape
+        rep = lambda a: np.tile(np.asarray(a), (G,) + (1,) * (np.asarray(a).ndim - 1))
+        idx, out, sc = oracle.decode(qs.reshape(U * G, 1, d), W, L, P, tau, rep(ids), rep(vnorm_f32), rep(K),
+                                     rep(V), n, k, want_scores=want_scores, lib=lib)
+        return idx.reshape(U, G, k), out.reshape(U, G, d), (sc.reshape(U, G, n) if sc is not None else None)
+
+    lib = oracle.load()
+    oracle_pins.pin_per_head_selection(lib)
+    monkeypatch.setattr(oracle, "decode_per_head", mutant)
+    with pytest.raises(AssertionError):
+        oracle_pins.pin_per_head_selection(lib)
