@@ -310,7 +310,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// 3-D tensor copy global -> shared (no multicast), completion on `bar`.
+// 3-D tensor copy global -> this CTA's shared memory, completion on `bar`.
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar)
 {
     asm volatile(
