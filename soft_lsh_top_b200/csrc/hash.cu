@@ -9,8 +9,10 @@
 // table, and the value-vector norms are cached.
 //
 // id_l(k) = sum_p [<W_{l,p}, k> > 0] 2^p with the projections in float32:
-// for bfloat16 keys on the tensor cores (hash_mma_kernel), for float32 keys
-// with one fused multiply-add per element in channel order (hash_kernel).
+// for bfloat16 keys on the fifth-generation tensor cores (hash_umma_kernel;
+// the warp-level hash_mma_kernel when SOCKET_HASH_NO_TCGEN05 is set), for
+// float32 keys with one fused multiply-add per element in channel order
+// (hash_kernel).
 // vnorm = sqrt(sum v^2) summed in float64, rounded to float32.
 #include <cuda.h>
 #include <stdlib.h>
