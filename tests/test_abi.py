@@ -219,3 +219,11 @@ def test_rotated_id_rows(L):
         for s in range(Lr):
             assert row[s] == (ids[0, table_of[n, s], n] if table_of[n, s] >= 0 else 0)
     assert padding_bytes(L, ncap).sum() == ncap * (Lr - L)
+
+
+def test_python_append_rejects_no_new_keys():
+    import torch
+    import soft_lsh_top_b200 as s
+    z = torch.zeros(1)
+    with pytest.raises(ValueError, match="n_new"):
+        s.socket_decode_append(z, z, z, z, z, z, 8, 0.5, 4, 0, z, z, z)
