@@ -306,15 +306,16 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
     // resident CTAs, so many units or tables do not queue in waves.
     const int qi = q_dtype == 1 ? 1 : 0;
     auto kern = qi ? (void*)soft_tables_kernel<uint16_t> : (void*)soft_tables_kernel<float>;
-    // Resident CTAs per SM by (q dtype, G, log2 tpb - 1), looked up once per process and device.
+    // Resident CTAs per SM by (q dtype, G, P, log2 tpb - 1), looked up once per thread and device.
     static thread_local int cached_dev = -1;
-    static thread_local int per_sm_cache[2][kMaxGroup + 1][3];
+    static thread_local int per_sm_cache[2][kMaxGroup + 1][kMaxP + 1][3];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev != cached_dev) {
         for (auto& a : per_sm_cache)
             for (auto& b : a)
-                for (int& c : b) c = -1;
+                for (auto& c : b)
+                    for (int& e : c) e = -1;
         for (void* kf : {(void*)soft_tables_kernel<uint16_t>, (void*)soft_tables_kernel<float>}) {
             const int max_smem = (int)sizeof(double) * kMaxGroup * (kHeadDim + 1 + kMaxTablesPerBlock * (kMaxP * 2 + 32)) +
                                  kMaxTablesPerBlock * kMaxP * kWRow * 2;
@@ -326,7 +327,7 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
     int tpb = 2, smem = 0;
     for (int li = 0;; ++li, tpb *= 2) {
         smem = (int)sizeof(double) * s.G * (kHeadDim + 1 + tpb * (kMaxP * 2 + 32)) + tpb * s.P * kWRow * 2;
-        int& per_sm = per_sm_cache[qi][s.G][li];
+        int& per_sm = per_sm_cache[qi][s.G][s.P][li];
         if (per_sm < 0) {
             cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
             if (e != cudaSuccess) return e;
