@@ -573,8 +573,9 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         hash_tflops = hash_flops / (hash_ms * 1e-3) / 1e12
         prefill = {
             "what": "socket_hash_keys over the whole layer (all units, N keys each); not in the decode step",
-            "kernel": ("hash_umma_kernel" if w.L * w.P <= 256 else "hash_mma_kernel") if w.dtype == "bf16"
-                      else "hash_kernel",
+            "kernel": "hash_umma_kernel" if w.dtype == "bf16" else "hash_kernel",
+            # tcgen05 passes over whole 32-table blocks of at most 256 hyperplanes
+            "passes": -(-w.L // (32 * max(1, 256 // (32 * w.P)))) if w.dtype == "bf16" else 1,
             "keys": keys, "ms": hash_ms, "keys_per_s": world * keys / (hash_ms * 1e-3),
             "algorithmic_bytes": hash_bytes, "gbs": hash_gbs, "hbm_frac": hash_gbs / peak,
             "flops": hash_flops, "tflops": hash_tflops,

@@ -246,7 +246,10 @@ int socket_decode_per_head(const void* q, int q_dtype, const uint16_t* W,
  * routine.  Every call on a device shares the same array, which keeps the
  * previous call's contents; the decode clears what must start at zero (its
  * counters and error word) itself.  Calls that overlap on the GPU (other
- * streams, other host threads) race on the array: serialise them.
+ * streams, other host threads) race on the array: serialise them.  The
+ * looked-up address is kept for the life of the process: do not call this
+ * entry point again on a device after cudaDeviceReset() in the same process
+ * (the array may then live elsewhere).
  */
 #define SOCKET_STATIC_WORKSPACE_BYTES (64u << 20)
 int socket_decode_static(const void* q, int q_dtype, const uint16_t* W,

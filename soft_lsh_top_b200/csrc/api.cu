@@ -4,7 +4,9 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "internal.h"
 #include "socket_attn.h"
@@ -119,6 +121,44 @@ size_t workspace_size(bool per_head, int64_t B, int64_t Hq, int64_t Hkv, int64_t
 
 }  // namespace
 
+cudaError_t set_smem_limit_once(const void* func, int bytes)
+{
+    struct Entry {
+        const void* func;
+        int dev, bytes;
+    };
+    static std::mutex lock;
+    static std::vector<Entry> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> guard(lock);
+    for (const Entry& x : done)
+        if (x.func == func && x.dev == dev && x.bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    // Every decode kernel asks for the largest shared-memory carveout, so
+    // consecutive kernels of a step never need an SM's L1/shared split changed.
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    done.push_back({func, dev, bytes});
+    return cudaSuccess;
+}
+
+int device_num_sms()
+{
+    constexpr int kMaxDevices = 128;
+    static int sms[kMaxDevices];  // 0: not looked up yet
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+    if (sms[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        sms[dev] = n > 0 ? n : 1;
+    }
+    return sms[dev];
+}
+
 bool pdl_enabled()
 {
     static const bool on = getenv("SOCKET_NO_PDL") == nullptr;
@@ -139,14 +179,16 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 4);
     w.counters = off;
     off = align256(off + 4 * (size_t)s.U);
-    w.unit_max = off;
+    w.topk_done = off;
     off = align256(off + 4 * (size_t)s.U);
     w.unit_hist = off;
     off = align256(off + 4 * (size_t)s.U * kScoreHistBins);
     w.cand_cnt = off;
     off = align256(off + 4 * (size_t)s.U);
     w.cand = off;
-    off = align256(off + 8 * (size_t)s.U * kTopkCandidates);
+    off = align256(off + 8 * (size_t)s.U * topk_candidate_capacity(s.Ncap));
+    w.bitmap = off;
+    off = align256(off + 4 * (size_t)s.U * (s.Ncap / 32));
     w.tables = off;
     off = align256(off + 4 * (size_t)s.U * ((s.L + 31) / 32) * s.NB * 64);
     w.scores = off;
@@ -199,7 +241,8 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     uint32_t* counters = reinterpret_cast<uint32_t*>(base + w.counters);
     float* tables = reinterpret_cast<float*>(base + w.tables);
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(base + w.scores);
-    uint32_t* unit_max = reinterpret_cast<uint32_t*>(base + w.unit_max);
+    uint32_t* topk_done = reinterpret_cast<uint32_t*>(base + w.topk_done);
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(base + w.bitmap);
     uint32_t* unit_hist = reinterpret_cast<uint32_t*>(base + w.unit_hist);
     uint32_t* cand_cnt = reinterpret_cast<uint32_t*>(base + w.cand_cnt);
     uint2* cand = reinterpret_cast<uint2*>(base + w.cand);
@@ -217,17 +260,18 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
         app.begin = N - n_new;
         app.end = N;
     }
-    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, app, tables, err_word, counters, unit_max, unit_hist,
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, app, tables, err_word, counters, topk_done, unit_hist,
                                         cand_cnt, cs),
                      "soft-table kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(1, cs), "step event record")) != SOCKET_OK) return st;
     const int64_t fresh_chunk = n_new > 0 ? (N - n_new) / 32 : Ncap / 32;
-    st = cuda_status(launch_score(tables, ids, vnorm, s, fresh_chunk, scores, unit_max, unit_hist, err_word, cs),
+    st = cuda_status(launch_score(tables, ids, vnorm, s, fresh_chunk, scores, unit_hist, err_word, cs),
                      "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_topk(scores, unit_max, unit_hist, cand_cnt, cand, s, idx_out, cs), "top-k kernel launch");
+    st = cuda_status(launch_topk(scores, unit_hist, cand_cnt, cand, bitmap, topk_done, s, idx_out, cs),
+                     "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
     st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,

@@ -660,7 +660,7 @@ cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32
 {
     const int rpc = attention_rows_per_cta(s.k, s.nsplit, kWChunk);
     auto kern = attention_warp_kernel<G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWSmemBytes);
+    cudaError_t e = set_smem_limit_once((const void*)kern, kWSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
@@ -677,7 +677,7 @@ cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, c
     constexpr int smem = 2 * 2 * Rows<KT>::kChunk * Rows<KT>::kRowBytes;
     const int rpc = attention_rows_per_cta(s.k, s.nsplit, Rows<KT>::kChunk);
     auto kern = attention_kernel<KT, G>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = set_smem_limit_once((const void*)kern, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream, q, q_dtype,
                    static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.share, s.Ncap, s.k, s.nsplit, rpc,

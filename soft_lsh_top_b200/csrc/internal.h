@@ -24,17 +24,20 @@ struct DecodeShape {
 constexpr int kScoreHistBins = 4096;
 constexpr int kScoreHistShift = 19;
 // Top-k candidate capacity per unit (keys in the threshold bin of the
-// histogram); above it the top-k kernel takes its multi-pass path.
-constexpr int kTopkCandidates = 4096;
+// histogram, at most Ncap); above it the top-k kernel selects over all of
+// the unit's scores instead.
+constexpr int kTopkCandidates = 16384;
+int topk_candidate_capacity(int64_t Ncap);
 
 // Workspace regions (byte offsets from the workspace base, 256-aligned).
 struct DecodeWorkspace {
     size_t err;        // uint32 device error word (offset 0)
     size_t counters;   // uint32 [U] merge counters
-    size_t unit_max;   // uint32 [U] bit pattern of each unit's largest score
+    size_t topk_done;  // uint32 [U] top-k tickets
     size_t unit_hist;  // uint32 [U][kScoreHistBins] score histogram
     size_t cand_cnt;   // uint32 [U] top-k candidate counters
-    size_t cand;       // uint2 [U][kTopkCandidates] top-k candidates (index, bit pattern)
+    size_t cand;       // uint2 [U][cap] top-k candidates (index, bit pattern), cap = topk_candidate_capacity
+    size_t bitmap;     // uint32 [U][Ncap / 32] top-k selection bitmap
     size_t tables;     // float [U][ceil(L/32)][NB][64], column j = table 32c + j mod 32
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
@@ -49,7 +52,12 @@ int attention_chunk_rows(int kv_dtype);
 // Attention CTAs per unit for these sizes (<= ceil(k / 16)).
 int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num_sms);
 int attention_rows_per_cta(int k, int nsplit, int chunk);
+// Multiprocessors of the current device (looked up once per device).
 int device_num_sms();
+// Raises `func`'s dynamic shared-memory limit to `bytes` unless an earlier
+// call already did so on the current device (one runtime call per kernel and
+// device, not per launch).
+cudaError_t set_smem_limit_once(const void* func, int bytes);
 
 // --- kernels (each returns cudaGetLastError() after its launch) -------------
 cudaError_t launch_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv,
@@ -68,24 +76,25 @@ struct AppendHash {
     int64_t begin = 0, end = 0;  // empty: nothing hashed
 };
 
-// Also zeroes the error word, the merge counters, the per-unit max scores,
-// the score histograms and the candidate counters, and hashes `app`'s keys.
+// Also zeroes the error word, the merge counters, the top-k tickets, the
+// score histograms and the candidate counters, and hashes `app`'s keys.
 cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, const DecodeShape& s,
                                double tau, const AppendHash& app, float* tables, uint32_t* err_word,
-                               uint32_t* counters, uint32_t* unit_max, uint32_t* unit_hist, uint32_t* cand_cnt,
+                               uint32_t* counters, uint32_t* topk_done, uint32_t* unit_hist, uint32_t* cand_cnt,
                                cudaStream_t stream);
 
 // fresh_chunk: first 32-key chunk of a unit whose ids the preceding soft-table
 // kernel writes in this step (none: a value >= Ncap / 32); such chunks are
 // not fetched before that kernel has completed.
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         int64_t fresh_chunk, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
-                         uint32_t* err_word, cudaStream_t stream);
+                         int64_t fresh_chunk, float* scores, uint32_t* unit_hist, uint32_t* err_word,
+                         cudaStream_t stream);
 // Bytes of one key's rotated id row (32 per started block of 32 tables).
 int ids_row_bytes(int L);
 
-cudaError_t launch_topk(const float* scores, const uint32_t* unit_max, const uint32_t* unit_hist,
-                        uint32_t* cand_cnt, uint2* cand, const DecodeShape& s, int32_t* idx_out, cudaStream_t stream);
+cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
+                        uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
+                        cudaStream_t stream);
 
 cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
                              const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,

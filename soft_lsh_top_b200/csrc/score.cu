@@ -78,19 +78,11 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int i)
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-__device__ __forceinline__ float ldg_stream_f32(const float* p)
-{
-    float v;
-    asm("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
-    return v;
-}
-
 struct ScoreArgs {
     const float* tables;  // [U][nblk][NB][64] expanded soft tables
     const uint8_t* ids;   // [U / share][Ncap][32 nblk] rotated id rows
     const float* vnorm;   // [U / share][Ncap]
     float* scores;        // [U][Ncap]
-    uint32_t* unit_max;
     uint32_t* unit_hist;
     uint32_t* err_word;
     int share;            // units per kv unit (CTAs per group)
@@ -118,7 +110,6 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     constexpr uint32_t kRingBytes = NS * kStageBytes;
     constexpr uint32_t kHistBytes = LAST ? kHistBins * 4u : 0u;
     extern __shared__ __align__(1024) char smem[];
-    __shared__ uint32_t red[kWarps];
     __shared__ __align__(8) uint64_t bar[kSlots];
     __shared__ __align__(8) uint64_t ring_bar[kWarps][NS];
 
@@ -188,7 +179,6 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         }
     };
 
-    uint32_t mx = 0;
     // Ids and norms stream through L2 once; the scores stay there for top-k.
     const uint64_t pol_stream = l2_policy_evict_first(), pol_keep = l2_policy_evict_last();
     uint32_t seq = 0;      // batches this warp has taken from its ring so far
@@ -309,11 +299,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                 if (c < cend && n < N) {
                     const float sc = LAST ? acc[j] * vn[j] : acc[j];
                     st_global_hint(su + n, sc, pol_keep);
-                    if (LAST) {
-                        const uint32_t bits = __float_as_uint(sc);
-                        mx = max(mx, bits);
-                        atomicAdd(shist + min(bits >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
-                    }
+                    if (LAST)
+                        atomicAdd(shist + min(__float_as_uint(sc) >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
                 }
             }
         }
@@ -325,15 +312,8 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         seq += nbatch;
 
         if (LAST) {
-            // The unit's largest live score and its score histogram.
-            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFullMask, mx, o));
-            if (lane == 0) red[warp] = mx;
+            // The unit's score histogram.
             __syncthreads();
-            if (tid == 0) {
-                uint32_t m = 0;
-                for (int w = 0; w < kWarps; ++w) m = max(m, red[w]);
-                atomicMax(a.unit_max + u, m);
-            }
             uint32_t* gh = a.unit_hist + u * kHistBins;
             for (int bn = tid; bn < kHistBins; bn += kThreads) {
                 const uint32_t c = shist[bn];
@@ -342,7 +322,6 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                     shist[bn] = 0;
                 }
             }
-            mx = 0;
         }
         if (k + kSlots < nseg) {
             __syncthreads();  // every warp is done with this slot's regions
@@ -357,7 +336,7 @@ template <int NBLK, int KEYS, int NS, bool FIRST, bool LAST>
 cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
 {
     auto kern = score_kernel<NBLK, KEYS, NS, FIRST, LAST>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = set_smem_limit_once((const void*)kern, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, args);
     if (e != cudaSuccess) return e;
@@ -366,26 +345,17 @@ cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
 
 }  // namespace
 
-int device_num_sms()
-{
-    int dev = 0, n = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 1;
-}
-
 int ids_row_bytes(int L) { return 32 * ((L + 31) / 32); }
 
 cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* vnorm, const DecodeShape& s,
-                         int64_t fresh_chunk, float* scores, uint32_t* unit_max, uint32_t* unit_hist,
-                         uint32_t* err_word, cudaStream_t stream)
+                         int64_t fresh_chunk, float* scores, uint32_t* unit_hist, uint32_t* err_word,
+                         cudaStream_t stream)
 {
     ScoreArgs a;
     a.tables = tables;
     a.ids = ids;
     a.vnorm = vnorm;
     a.scores = scores;
-    a.unit_max = unit_max;
     a.unit_hist = unit_hist;
     a.err_word = err_word;
     a.nblk = (s.L + 31) / 32;

@@ -74,8 +74,8 @@ def test_hash_in_ranges_matches_oracle(case):
     """The cache hashed piecewise -- a long range from an unaligned start, single
     appended keys, a range inside one 32-key chunk, the rest -- equals the
     oracle's hash of every key (tensor-core tiles that start anywhere and end
-    ragged; the last case has more hyperplanes than one tensor-core tile and
-    takes the warp-level kernel)."""
+    ragged; the last case has more hyperplanes than one tensor-core
+    accumulator holds and runs in two passes over 32-table blocks)."""
     w = SMALL[case]
     inp = wl.make_inputs(w, DEV)
     ids, vnorm = sk.alloc_cache_index(inp["K"].shape[0], w.Hkv, w.ncap, w.L, DEV)
@@ -200,6 +200,20 @@ def test_all_ties_candidate_path():
     for b in range(w.B):
         for h in range(w.Hkv):
             assert torch.equal(idx[b, h], want)
+
+
+def test_all_ties_above_candidate_capacity():
+    """All scores equal with more keys than the candidate list holds: the
+    last top-k CTA of each unit selects over all of the unit's scores and
+    compacts from them -- still keys 0..k-1."""
+    w = wl.Workload(name="ties_wide", B=1, Hq=2, Hkv=1, N=40000, L=4, P=8, tau=0.3, k=1000, seed=7012)
+    inp = wl.make_inputs(w, DEV)
+    inp["q"].zero_()
+    inp["V"].fill_(1.0)
+    ids, vnorm = gpu_hash(inp, w)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm)
+    assert torch.equal(idx[0, 0], torch.arange(w.k, dtype=torch.int32, device=DEV))
+    torch.testing.assert_close(out, torch.ones_like(out), atol=1e-6, rtol=0)
 
 
 def test_decode_in_a_cuda_graph_matches_direct_calls():

@@ -2,15 +2,15 @@
 
 It serves callers that cannot call cudaMalloc and get no scratch from anyone
 (for example code embedded in a serving runtime that has reserved the GPU's
-memory for its own pool).  It must give the same results as socket_decode
-with a caller workspace, on consecutive calls that share its fixed device
-scratch, and refuse sizes that do not fit that scratch.
+memory for its own pool).  It runs the same kernels as socket_decode on the
+same inputs, only with its scratch in a fixed device array, so its results
+must equal socket_decode's bit for bit, on consecutive calls that share that
+scratch; it must not allocate device memory; and it must refuse sizes that
+do not fit the scratch.
 
 This file is collected last on purpose: if it fails, a run that stops at the
 first failure has already run every other test.
 """
-import ctypes
-
 import pytest
 import torch
 
@@ -34,6 +34,10 @@ def test_static_decode_rejects_sizes_beyond_its_scratch():
     assert "static scratch" in lib.socket_last_error().decode()
 
 
+def _bits(t):
+    return t.view(torch.int32) if t.dtype == torch.float32 else t
+
+
 @pytest.mark.gpu
 def test_static_decode_matches_workspace_decode_on_consecutive_calls():
     dev = torch.device("cuda:0")
@@ -44,18 +48,39 @@ def test_static_decode_matches_workspace_decode_on_consecutive_calls():
     ws, _, _ = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, dev)
     queries = [inp["q"], torch.randn(inp["q"].shape, generator=torch.Generator(dev).manual_seed(5),
                                      device=dev).to(inp["q"].dtype)]
-    for q in queries:  # two calls in a row; the second sees the first call's leftover scratch
+    results = []
+    for q in queries:
         ref_idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=dev)
         ref_out = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device=dev)
         ref_sc = torch.empty(w.B, w.Hkv, w.ncap, dtype=torch.float32, device=dev)
         sk.socket_decode(q, inp["W"], ids, vnorm, inp["K"], inp["V"], w.N, w.tau, w.k, ws, ref_idx, ref_out,
                          scores_out=ref_sc)
-        idx = torch.full_like(ref_idx, -1)
-        out = torch.full_like(ref_out, float("nan"))
-        sc = torch.full_like(ref_sc, float("nan"))
+        out_bufs = (torch.full_like(ref_idx, -1), torch.full_like(ref_out, float("nan")),
+                    torch.full_like(ref_sc, float("nan")))
+        results.append(((ref_idx, ref_out, ref_sc), out_bufs))
+    torch.cuda.synchronize()
+
+    # The first call on the device looks up the scratch's address (and may
+    # load the module that holds it); measure memory from after that call on.
+    _, (idx0, out0, sc0) = results[0]
+    sk.socket_decode_static(queries[0], inp["W"], ids, vnorm, inp["K"], inp["V"], w.N, w.tau, w.k, idx0, out0,
+                            scores_out=sc0)
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    torch_before = torch.cuda.memory_allocated(dev)
+    for q, (_, (idx, out, sc)) in zip(queries, results):
+        # two calls in a row; the second sees the first call's leftover scratch
+        idx.fill_(-1)
+        out.fill_(float("nan"))
+        sc.fill_(float("nan"))
         sk.socket_decode_static(q, inp["W"], ids, vnorm, inp["K"], inp["V"], w.N, w.tau, w.k, idx, out,
                                 scores_out=sc)
-        torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info(dev)
+    assert free_after == free_before, (free_before, free_after)
+    assert torch.cuda.memory_allocated(dev) == torch_before
+    for (ref_idx, ref_out, ref_sc), (idx, out, sc) in results:
+        # the same kernels on the same inputs: bit-identical results
         assert torch.equal(idx, ref_idx)
-        torch.testing.assert_close(sc[..., : w.N], ref_sc[..., : w.N], rtol=1e-5, atol=0)
-        torch.testing.assert_close(out, ref_out, rtol=0, atol=2e-3)
+        assert torch.equal(_bits(sc[..., : w.N]), _bits(ref_sc[..., : w.N]))
+        assert torch.equal(_bits(out), _bits(ref_out))
