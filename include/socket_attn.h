@@ -280,6 +280,19 @@ const char* socket_last_error(void);
 #define SOCKET_DECODE_KERNELS 4
 int socket_set_step_events(void* const* events, int n);
 
+/*
+ * socket_set_wait_limit -- failure-path diagnostic.  Sets how many times a
+ * decode kernel (scoring, attention) polls for data it has requested before
+ * it gives up, sets its bit in the workspace error word
+ * (SOCKET_DEVERR_TABLE_TIMEOUT, SOCKET_DEVERR_GATHER_TIMEOUT), lets the
+ * copies it has already issued land, and returns without its results.
+ * Default 4194304 polls (~ a second or more); 0 makes every such wait give
+ * up at once, which is how tests drive the give-up path without a fault;
+ * 0xffffffff restores the default.  Process-wide; affects calls made after
+ * it.  Returns the previous limit.  No counterpart in the method.
+ */
+uint32_t socket_set_wait_limit(uint32_t polls);
+
 /* socket_version -- ABI version of this library (major * 100 + minor). */
 int socket_version(void);
 

@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
     "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check", "socket_decode_append",
-    "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events", "library_path", "load_library",
+    "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events",
+    "socket_set_wait_limit", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
 
@@ -82,6 +83,8 @@ def load_library(path: str | None = None):
     lib.socket_last_error.restype = ctypes.c_char_p
     lib.socket_set_step_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _int]
     lib.socket_set_step_events.restype = _int
+    lib.socket_set_wait_limit.argtypes = [ctypes.c_uint32]
+    lib.socket_set_wait_limit.restype = ctypes.c_uint32
     lib.socket_ids_row_bytes.argtypes = [_int]
     lib.socket_ids_row_bytes.restype = _int
     lib.socket_version.argtypes = []
@@ -306,6 +309,13 @@ def socket_set_step_events(events) -> None:
     n = len(events)
     arr = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(int(e.cuda_event)) for e in events])
     _raise(lib.socket_set_step_events(arr, n))
+
+
+def socket_set_wait_limit(polls: int) -> int:
+    """Polls before a decode kernel's wait for requested data gives up (0: at
+    once, for tests of the failure path; 0xffffffff: the default).  Returns
+    the previous limit."""
+    return int(load_library().socket_set_wait_limit(polls & 0xffffffff))
 
 
 # ----------------------------------------------------------------------------

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -159,6 +160,13 @@ int device_num_sms()
     return sms[dev];
 }
 
+namespace {
+constexpr uint32_t kDefaultWaitPolls = 1u << 22;
+std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
+}  // namespace
+
+uint32_t wait_poll_limit() { return g_wait_polls.load(std::memory_order_relaxed); }
+
 bool pdl_enabled()
 {
     static const bool on = getenv("SOCKET_NO_PDL") == nullptr;
@@ -188,7 +196,7 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     w.cand = off;
     off = align256(off + 8 * (size_t)s.U * topk_candidate_capacity(s.Ncap));
     w.bitmap = off;
-    off = align256(off + 4 * (size_t)s.U * (s.Ncap / 32));
+    off = align256(off + 4 * (size_t)s.U * (size_t)topk_bitmap_stride(s.Ncap));
     w.tables = off;
     off = align256(off + 4 * (size_t)s.U * ((s.L + 31) / 32) * s.NB * 64);
     w.scores = off;
@@ -302,6 +310,11 @@ int socket_set_step_events(void* const* events, int n)
 }
 
 const char* socket_last_error(void) { return g_last_error.c_str(); }
+
+uint32_t socket_set_wait_limit(uint32_t polls)
+{
+    return g_wait_polls.exchange(polls == 0xffffffffu ? kDefaultWaitPolls : polls);
+}
 
 int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv, int64_t Ncap,
                      int64_t n_begin, int64_t n_end, int64_t d, const uint16_t* W, int L, int P, uint8_t* ids,

@@ -142,7 +142,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     const void* __restrict__ q, int q_dtype, const KT* __restrict__ K, const KT* __restrict__ V,
     const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
-    uint32_t* __restrict__ err_word, float* __restrict__ out)
+    uint32_t* __restrict__ err_word, float* __restrict__ out, uint32_t max_polls)
 {
     constexpr int kChunk = Rows<KT>::kChunk;
     constexpr int kRowBytes = Rows<KT>::kRowBytes;
@@ -221,7 +221,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
         const int nrows = min(kChunk, r_end - (r_begin + c * kChunk));
         const char* ks = smem + st * kStageBytes;
         const char* vs = ks + kChunk * kRowBytes;
-        if (!mbar_wait_bounded(&bar[st], (uint32_t)((c >> 1) & 1), kMaxPolls)) {
+        if (!mbar_wait_bounded(&bar[st], (uint32_t)((c >> 1) & 1), max_polls)) {
             if (tid == 0) atomicOr(err_word, SOCKET_DEVERR_GATHER_TIMEOUT);
             // let copies in flight land before exiting
             mbar_wait_bounded(&bar[st], (uint32_t)((c >> 1) & 1), kMaxPolls);
@@ -440,7 +440,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
     const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
     float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
-    uint32_t* __restrict__ err_word, float* __restrict__ out)
+    uint32_t* __restrict__ err_word, float* __restrict__ out, uint32_t max_polls)
 {
     static_assert(G <= 8, "heads are the M rows 0..7 of the 16-row tile");
     extern __shared__ __align__(128) char smem[];
@@ -534,7 +534,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     for (int j = 0; j < cw; ++j) {
         const int st = j & 1;
         const int32_t next_row = row_index(j + 2);  // in flight while chunk j is used
-        const bool got = mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), kMaxPolls);
+        const bool got = mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), max_polls);
         if (__any_sync(kFullMask, !got)) {
             if (lane == 0) atomicOr(err_word, SOCKET_DEVERR_GATHER_TIMEOUT);
             mbar_wait_bounded(&bar[warp][st], (uint32_t)((j >> 1) & 1), kMaxPolls);
@@ -664,7 +664,8 @@ cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                   idx, s.share, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out);
+                   idx, s.share, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out,
+                   wait_poll_limit());
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -681,7 +682,7 @@ cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, c
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream, q, q_dtype,
                    static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.share, s.Ncap, s.k, s.nsplit, rpc,
-                   part_o, part_ml, counters, err_word, out);
+                   part_o, part_ml, counters, err_word, out, wait_poll_limit());
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

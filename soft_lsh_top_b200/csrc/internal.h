@@ -26,8 +26,11 @@ constexpr int kScoreHistShift = 19;
 // Top-k candidate capacity per unit (keys in the threshold bin of the
 // histogram, at most Ncap); above it the top-k kernel selects over all of
 // the unit's scores instead.
-constexpr int kTopkCandidates = 16384;
+constexpr int kTopkCandidates = 8192;
 int topk_candidate_capacity(int64_t Ncap);
+// Words per unit row of the top-k selection bitmap (Ncap / 32 rounded up to
+// a multiple of 4, so every row starts on a 16-byte boundary).
+int64_t topk_bitmap_stride(int64_t Ncap);
 
 // Workspace regions (byte offsets from the workspace base, 256-aligned).
 struct DecodeWorkspace {
@@ -37,7 +40,7 @@ struct DecodeWorkspace {
     size_t unit_hist;  // uint32 [U][kScoreHistBins] score histogram
     size_t cand_cnt;   // uint32 [U] top-k candidate counters
     size_t cand;       // uint2 [U][cap] top-k candidates (index, bit pattern), cap = topk_candidate_capacity
-    size_t bitmap;     // uint32 [U][Ncap / 32] top-k selection bitmap
+    size_t bitmap;     // uint32 [U][topk_bitmap_stride(Ncap)] top-k selection bitmap
     size_t tables;     // float [U][ceil(L/32)][NB][64], column j = table 32c + j mod 32
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
@@ -103,6 +106,11 @@ cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const vo
 // Waits for `stream`, then reads and clears the hash kernels' device error
 // bits; returns a cudaError_t value.
 int hash_device_error(cudaStream_t stream, uint32_t* bits);
+
+// Polls after which a decode kernel's wait for data gives up (the
+// socket_set_wait_limit diagnostic; waits that drain copies already issued
+// keep their own, long limit).
+uint32_t wait_poll_limit();
 
 // Sets the calling thread's socket_last_error() message; returns `status`.
 int record_error(int status, const char* message);

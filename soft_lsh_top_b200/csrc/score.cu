@@ -51,13 +51,19 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr uint32_t kRegionBytes = 1u << 16;  // [256 buckets][64 columns] floats
-constexpr int kRegions = 2;
+constexpr int kMaxRegions = 2;
 constexpr int kHistBins = kScoreHistBins;  // unit histogram of score bit patterns >> kHistShift
 constexpr int kHistShift = kScoreHistShift;
 // The regions sit at 64 KB-aligned shared addresses inside the dynamic
 // allocation; the histogram and the copy rings use the space around them.
 constexpr int kSmemBytes = 226 * 1024;
 constexpr uint32_t kMaxPolls = 1u << 22;
+#ifndef SCORE_R1
+#define SCORE_R1 2
+#endif
+#ifndef SCORE_NS1
+#define SCORE_NS1 2
+#endif
 
 __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
@@ -93,17 +99,20 @@ struct ScoreArgs {
     int64_t Ncap, N;
     int64_t chunks_per_unit, total_chunks, chunks_per_cta;  // over kv units; per group of CTAs
     int64_t fresh_chunk;  // chunks from here on get ids in this step: not fetched before the wait
+    uint32_t max_polls;   // polls before a wait for data gives up (draining waits use kMaxPolls)
 };
 
-// NBLK: 32-table blocks scored by this launch (1 or 2); KEYS: 32-key chunks
-// per warp per batch; NS: batches in a warp's copy ring; FIRST / LAST:
-// whether this launch starts / finishes the sum (launches in between pass
-// partial sums through the score buffer).
-template <int NBLK, int KEYS, int NS, bool FIRST, bool LAST>
+// NBLK: 32-table blocks scored by this launch (1 or 2); REGIONS: 64 KB table
+// regions in shared memory (REGIONS / NBLK units staged at once); KEYS:
+// 32-key chunks per warp per batch; NS: batches in a warp's copy ring;
+// FIRST / LAST: whether this launch starts / finishes the sum (launches in
+// between pass partial sums through the score buffer).
+template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST>
 __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 {
+    static_assert(REGIONS >= NBLK && REGIONS <= kMaxRegions, "a unit's blocks fit the regions");
     constexpr int V = 2 * NBLK;                            // 16-byte id pieces per key
-    constexpr int kSlots = kRegions / NBLK;                // units staged at once
+    constexpr int kSlots = REGIONS / NBLK;                 // units staged at once
     constexpr uint32_t kChunkIds = 1024u * NBLK;           // id bytes of a chunk in this launch
     constexpr uint32_t kChunkBytes = kChunkIds + (LAST ? 128u : 0u);  // + the chunk's norms
     constexpr uint32_t kStageBytes = KEYS * kChunkBytes;
@@ -120,7 +129,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 
     // The histogram and the warps' copy rings fill the space below the two
     // table regions, then the space above them.
-    uint32_t lo = sbase, hi = region0 + kRegions * kRegionBytes;
+    uint32_t lo = sbase, hi = region0 + REGIONS * kRegionBytes;
     const uint32_t lo_end = region0, hi_end = sbase + kSmemBytes;
     auto place = [&](uint32_t bytes) -> uint32_t {
         if (lo + bytes <= lo_end) { lo += bytes; return lo - bytes; }
@@ -231,20 +240,27 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         // this step (keys hashed on append).
         const int nfirst = min(NS, nbatch);
         const bool early = k > 0 || nfirst == 0 || chunk_at(nfirst * KEYS - 1) < a.fresh_chunk;
-        if (lane == 0 && !failed && early)
-            for (int b = 0; b < nfirst; ++b) issue(b);
+        int issued = 0;  // batches of this segment copied so far (warp-uniform)
+        if (!failed && early) {
+            if (lane == 0)
+                for (int b = 0; b < nfirst; ++b) issue(b);
+            issued = nfirst;
+        }
         if (k == 0) {
             // The soft tables (and, after the first launch, the partial sums)
             // come from the previous kernel on the stream.
             pdl_wait();
-            if (lane == 0 && !failed && !early)
-                for (int b = 0; b < nfirst; ++b) issue(b);
+            if (!failed && !early) {
+                if (lane == 0)
+                    for (int b = 0; b < nfirst; ++b) issue(b);
+                issued = nfirst;
+            }
             if (tid == 0)
                 for (int kk = 0; kk < min(kSlots, nseg); ++kk) issue_tables(kk);
         }
         // Waits give up after a bounded number of polls; a warp gives up as a
         // whole so it never splits around __syncwarp.
-        const bool tables_ok = mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
+        const bool tables_ok = mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), a.max_polls);
         if (__any_sync(kFullMask, !tables_ok)) {
             if (lane == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
             mbar_wait_bounded(&bar[slot], (uint32_t)((k / kSlots) & 1), kMaxPolls);
@@ -254,7 +270,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         int b = 0;
         for (; b < nbatch && !failed; ++b) {
             const uint32_t st = (seq + b) % NS;
-            const bool ids_ok = mbar_wait_bounded(&ring_bar[warp][st], ((seq + b) / NS) & 1u, kMaxPolls);
+            const bool ids_ok = mbar_wait_bounded(&ring_bar[warp][st], ((seq + b) / NS) & 1u, a.max_polls);
             if (__any_sync(kFullMask, !ids_ok)) {
                 if (lane == 0) atomicOr(a.err_word, SOCKET_DEVERR_TABLE_TIMEOUT);
                 failed = true;
@@ -272,7 +288,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
             // Every lane's reads of this stage precede the next copy into it.
             fence_proxy_async_shared();
             __syncwarp();
-            if (lane == 0 && b + NS < nbatch) issue(b + NS);
+            if (b + NS < nbatch) {
+                if (lane == 0) issue(b + NS);
+                issued = b + NS + 1;
+            }
             float acc[KEYS];
 #pragma unroll
             for (int j = 0; j < KEYS; ++j)
@@ -306,7 +325,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         }
         if (failed) {
             // Let this warp's copies in flight land before anything moves on.
-            for (int bb = b; bb < min(nbatch, b + NS); ++bb)
+            for (int bb = b; bb < issued; ++bb)
                 mbar_wait_bounded(&ring_bar[warp][(seq + bb) % NS], ((seq + bb) / NS) & 1u, kMaxPolls);
         }
         seq += nbatch;
@@ -332,10 +351,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     }
 }
 
-template <int NBLK, int KEYS, int NS, bool FIRST, bool LAST>
+template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST>
 cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
 {
-    auto kern = score_kernel<NBLK, KEYS, NS, FIRST, LAST>;
+    auto kern = score_kernel<NBLK, REGIONS, KEYS, NS, FIRST, LAST>;
     cudaError_t e = set_smem_limit_once((const void*)kern, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, args);
@@ -364,6 +383,7 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     a.N = s.N;
     a.share = s.share;
     a.fresh_chunk = fresh_chunk;
+    a.max_polls = wait_poll_limit();
     a.chunks_per_unit = (s.N + 31) / 32;
     a.total_chunks = (s.U / s.share) * a.chunks_per_unit;
     // At least one chunk per warp per CTA; at most one CTA per SM; groups of
@@ -374,21 +394,21 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     a.chunks_per_cta = (a.total_chunks + groups - 1) / groups;
     // Blocks two at a time (two 64 KB regions); partial sums pass through
     // the score buffer between launches when L > 64.
-    for (int b0 = 0; b0 < a.nblk; b0 += kRegions) {
-        const int nb = min(kRegions, a.nblk - b0);
+    for (int b0 = 0; b0 < a.nblk; b0 += kMaxRegions) {
+        const int nb = min(kMaxRegions, a.nblk - b0);
         a.blk0 = b0;
         a.first = b0 == 0;
         a.last = b0 + nb == a.nblk;
         cudaError_t e;
         if (nb == 1)
-            e = a.first ? launch_one<1, 2, 2, true, true>(a, grid, stream)
-                        : launch_one<1, 2, 2, false, true>(a, grid, stream);
+            e = a.first ? launch_one<1, SCORE_R1, 2, SCORE_NS1, true, true>(a, grid, stream)
+                        : launch_one<1, SCORE_R1, 2, SCORE_NS1, false, true>(a, grid, stream);
         else if (a.first)
-            e = a.last ? launch_one<2, 1, 2, true, true>(a, grid, stream)
-                       : launch_one<2, 1, 2, true, false>(a, grid, stream);
+            e = a.last ? launch_one<2, 2, 1, 2, true, true>(a, grid, stream)
+                       : launch_one<2, 2, 1, 2, true, false>(a, grid, stream);
         else
-            e = a.last ? launch_one<2, 1, 2, false, true>(a, grid, stream)
-                       : launch_one<2, 1, 2, false, false>(a, grid, stream);
+            e = a.last ? launch_one<2, 2, 1, 2, false, true>(a, grid, stream)
+                       : launch_one<2, 2, 1, 2, false, false>(a, grid, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

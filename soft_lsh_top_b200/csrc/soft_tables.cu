@@ -25,6 +25,17 @@ constexpr int kRows = kTpb * kMaxP;        // hyperplane rows per CTA
 constexpr int kWRow = kHeadDim + 8;        // padded bf16 hyperplane row in shared memory (272 bytes)
 constexpr int kHeadsPerPass = 4;           // heads whose dot products share one read of a hyperplane row
 
+// bfloat16 bits (low 16) -> float64, exact.  Normal values are rebuilt with
+// integer operations (sign, exponent rebiased by 1023 - 127, the 7 mantissa
+// bits at the top of the fp64 mantissa); zero, subnormals, infinities and NaN
+// take the hardware widening.
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t b)
+{
+    const uint32_t mag = b & 0x7fffu, e = mag >> 7;
+    if (e == 0u || e == 0xffu) return (double)__uint_as_float(b << 16);
+    return __hiloint2double((int)(((b & 0x8000u) << 16) | ((mag << 13) + (896u << 20))), 0);
+}
+
 // Dynamic shared memory of a CTA for group size G.
 __host__ __device__ constexpr int smem_bytes(int G)
 {
@@ -141,9 +152,8 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
                 const uint32_t words[4] = {w8.x, w8.y, w8.z, w8.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float2 f = bf16x2_to_f32x2(words[i]);
-                    wd[8 * s + 2 * i] = (double)f.x;
-                    wd[8 * s + 2 * i + 1] = (double)f.y;
+                    wd[8 * s + 2 * i] = bf16_bits_to_f64(words[i] & 0xffffu);
+                    wd[8 * s + 2 * i + 1] = bf16_bits_to_f64(words[i] >> 16);
                 }
             }
         }
@@ -195,8 +205,9 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
 
         // Nibble tables: lo over planes 0..min(P,4)-1, hi over planes 4..P-1.
         const int plo = min(P, 4);
-        for (int e = tid; e < G * nt * 32; e += kThreads) {
-            const int h = e / (nt * 32), t = (e >> 5) % nt, hi = (e >> 4) & 1, v = e & 15;
+        for (int e = tid; e < G * kTpb * 32; e += kThreads) {
+            const int h = e >> 8, t = (e >> 5) & (kTpb - 1), hi = (e >> 4) & 1, v = e & 15;
+            if (t >= nt) continue;
             double prod = 1.0;
             const int p0 = hi ? 4 : 0, p1 = hi ? P : plo;
             for (int pp = p0; pp < p1; ++pp) prod *= SIG(h, t, pp, (v >> (pp - p0)) & 1);
@@ -225,7 +236,11 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         for (int t = 0; t < kTpb; ++t) {
             double acc = 0.0;
             if (t < nt)
-                for (int h = 0; h < G; ++h) acc = fma(NIB(h, t, 0, bucket & 15), NIB(h, t, 1, bucket >> 4), acc);
+                for (int h0 = 0; h0 < G; h0 += 4)
+#pragma unroll
+                    for (int hh = 0; hh < 4; ++hh)
+                        if (h0 + hh < G)
+                            acc = fma(NIB(h0 + hh, t, 0, bucket & 15), NIB(h0 + hh, t, 1, bucket >> 4), acc);
             vals[t] = (float)acc;
         }
         float* row = tu + ((int64_t)(l0 >> 5) * NB + bucket) * 64 + (l0 & 31);

@@ -38,14 +38,17 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kSliceKeys = 32768;                      // keys per CTA
-constexpr int kLoads = 8;                              // 16-byte score loads per thread in flight
-constexpr int kRounds = kSliceKeys / (4 * kThreads * kLoads);
+constexpr int kLoadsPerThread = kSliceKeys / (4 * kThreads);  // 16-byte score loads per thread
+constexpr int kInFlight = 6;                           // of them in flight at a time
 constexpr int kBins = 2048;                            // radix bins of the digit passes
 constexpr int kWordsPerThread = 8;                     // bitmap words per thread and tile of the compaction
+constexpr int kTileWords = kThreads * kWordsPerThread;  // bitmap words per tile (131072 keys)
 
 struct Shared {
     uint32_t warp_sums[kWarps];
     uint32_t digit, krem, last;
+    uint32_t count;  // keys in the bin found by the last digit; candidates of this CTA during the read
+    uint32_t base;   // offset of this CTA's candidates in the unit list
     __align__(16) uint32_t hist[kBins];
 };
 
@@ -111,6 +114,10 @@ __device__ __forceinline__ void radix_digit(Shared& sh, int n, Get get, int shif
 {
     const int tid = threadIdx.x;
     for (int b = tid; b < kBins; b += kThreads) sh.hist[b] = 0;
+    if (tid == 0) {  // kept if no bin holds the krem-th value (inconsistent input)
+        sh.digit = 0;
+        sh.krem = krem;
+    }
     __syncthreads();
     for (int i = tid; i < n; i += kThreads) {
         const uint32_t x = get(i);
@@ -126,6 +133,8 @@ __device__ __forceinline__ void radix_digit(Shared& sh, int n, Get get, int shif
         c[q] = sh.hist[bins[q]];
     }
     find_bin<kPer>(c, krem, sh, [&](int q) { return (uint32_t)bins[q]; });
+    __syncthreads();
+    if (threadIdx.x == 0) sh.count = sh.hist[sh.digit];
     __syncthreads();
     prefix |= sh.digit << shift;
     mask |= dmask << shift;
@@ -188,28 +197,45 @@ struct TopkArgs {
     const uint32_t* unit_hist; // [U][kScoreHistBins]
     uint32_t* cand_cnt;        // [U] candidates appended (zeroed before the step)
     uint2* cand;               // [U][cap] (index, bit pattern)
-    uint32_t* bitmap;          // [U][Ncap / 32]
+    uint32_t* bitmap;          // [U][bm_stride] (Ncap / 32 words used)
     uint32_t* done;            // [U] tickets of finished CTAs (zeroed before the step)
     int32_t* idx_out;          // [U][k]
-    int64_t Ncap;
+    int64_t Ncap, bm_stride;
     int N, k, C, cap;
 };
 
 // Grid: U * C CTAs of kThreads; CTA r of unit u reads keys [r S, min(N, (r+1) S)).
+// Dynamic shared memory: the CTA's candidates (then the unit's) and one tile
+// of the selection bitmap.
 __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
 {
     __shared__ Shared sh;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    extern __shared__ __align__(16) char topk_dyn[];
+    uint2* scand = reinterpret_cast<uint2*>(topk_dyn);                               // [a.cap]
+    uint32_t* sbits = reinterpret_cast<uint32_t*>(topk_dyn + sizeof(uint2) * a.cap);  // [kTileWords]
+    const int tid = threadIdx.x, lane = tid & 31;
     const int64_t u = blockIdx.x / a.C;
     const int r = blockIdx.x % a.C;
     const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + u * a.Ncap);
-    uint32_t* bm = a.bitmap + u * (a.Ncap / 32);
+    uint32_t* bm = a.bitmap + u * a.bm_stride;  // 16-byte aligned rows
     const int lo = r * kSliceKeys, hi = min(a.N, lo + kSliceKeys);
 
     // The grid fits in one wave, so the attention kernel's CTAs may be placed
     // now; they wait for this grid to finish before they read anything.
     pdl_launch_dependents();
     pdl_wait();  // scores and histograms come from the previous kernel on the stream
+
+    // Load g of this thread covers keys lo + 2048 g + 4 tid .. + 3 (lanes
+    // 8m .. 8m + 7 of a warp: the 32 keys of one bitmap word).  The first
+    // kInFlight loads are issued before the histogram is read.
+    auto key_of = [&](int g) { return lo + g * 4 * kThreads + 4 * tid; };
+    auto load = [&](int g) {
+        const int n0 = key_of(g);
+        return n0 < hi ? __ldcg(reinterpret_cast<const uint4*>(su + n0)) : make_uint4(0, 0, 0, 0);
+    };
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int g = 0; g < kInFlight; ++g) v[g] = load(g);
 
     // ---- the unit histogram: bin d0 of the k-th largest score.
     {
@@ -218,73 +244,78 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         const uint4* hp = reinterpret_cast<const uint4*>(a.unit_hist + u * kScoreHistBins + (b0 - (kPer - 1)));
         uint32_t c[kPer];
 #pragma unroll
-        for (int v = 0; v < kPer / 4; ++v) {
-            const uint4 w = __ldcg(hp + (kPer / 4 - 1 - v));
-            c[4 * v] = w.w;
-            c[4 * v + 1] = w.z;
-            c[4 * v + 2] = w.y;
-            c[4 * v + 3] = w.x;
+        for (int q = 0; q < kPer / 4; ++q) {
+            const uint4 w = __ldcg(hp + (kPer / 4 - 1 - q));
+            c[4 * q] = w.w;
+            c[4 * q + 1] = w.z;
+            c[4 * q + 2] = w.y;
+            c[4 * q + 3] = w.x;
         }
         if (tid == 0) {
             sh.digit = 0;
             sh.krem = (uint32_t)a.k;
+            sh.count = 0;
         }
         __syncthreads();
         find_bin<kPer>(c, (uint32_t)a.k, sh, [&](int q) { return (uint32_t)(b0 - q); });
         __syncthreads();
     }
     const uint32_t d0 = sh.digit, krem0 = sh.krem;
+    const uint32_t ncand = __ldcg(a.unit_hist + u * kScoreHistBins + d0);  // keys of the unit in bin d0
+    const bool fits = ncand <= (uint32_t)a.cap;
 
-    // ---- one read of the slice: bitmap words and candidates.  In load i of
-    // a round thread t holds keys base + 2048 i + 4 t .. + 3, so lanes
-    // 8m .. 8m + 7 of a warp hold the 32 keys of one bitmap word.
-    for (int round = 0; round < kRounds; ++round) {
-        const int base = lo + round * kLoads * 4 * kThreads;
-        if (base >= hi) break;
-        uint4 v[kLoads];
+    // ---- one read of the slice: bitmap words, and the candidates into
+    // shared memory (one shared atomic per warp and load that has any).
 #pragma unroll
-        for (int i = 0; i < kLoads; ++i) {
-            const int n0 = base + i * 4 * kThreads + 4 * tid;
-            v[i] = n0 < hi ? __ldcg(reinterpret_cast<const uint4*>(su + n0)) : make_uint4(0, 0, 0, 0);
+    for (int g = 0; g < kLoadsPerThread; ++g) {
+        const uint4 x = v[g % kInFlight];
+        if (g + kInFlight < kLoadsPerThread) v[g % kInFlight] = load(g + kInFlight);
+        const int n0 = key_of(g);
+        const uint32_t vals[4] = {x.x, x.y, x.z, x.w};
+        uint32_t nib = 0, cmask = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t top = vals[e] >> kScoreHistShift;
+            const bool live = n0 + e < hi;
+            nib |= (uint32_t)(live && top >= d0) << e;
+            cmask |= (uint32_t)(live && top == d0) << e;
         }
+        uint32_t word = nib << ((lane & 7) * 4);
+        word |= __shfl_xor_sync(kFullMask, word, 1);
+        word |= __shfl_xor_sync(kFullMask, word, 2);
+        word |= __shfl_xor_sync(kFullMask, word, 4);
+        if ((lane & 7) == 0 && n0 < hi) bm[n0 >> 5] = word;
+        const uint32_t cnt = fits ? __popc(cmask) : 0u;
+        if (__any_sync(kFullMask, cnt != 0)) {
+            uint32_t incl = cnt;
 #pragma unroll
-        for (int i = 0; i < kLoads; ++i) {
-            const int n0 = base + i * 4 * kThreads + 4 * tid;
-            const uint32_t vals[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-            uint32_t nib = 0, cmask = 0;
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(kFullMask, incl, o);
+                if (lane >= o) incl += y;
+            }
+            uint32_t slot = 0;
+            if (lane == 31) slot = atomicAdd(&sh.count, incl);
+            slot = __shfl_sync(kFullMask, slot, 31) + incl - cnt;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const uint32_t top = vals[e] >> kScoreHistShift;
-                const bool live = n0 + e < hi;
-                nib |= (uint32_t)(live && top >= d0) << e;
-                cmask |= (uint32_t)(live && top == d0) << e;
-            }
-            uint32_t word = nib << ((lane & 7) * 4);
-            word |= __shfl_xor_sync(kFullMask, word, 1);
-            word |= __shfl_xor_sync(kFullMask, word, 2);
-            word |= __shfl_xor_sync(kFullMask, word, 4);
-            if ((lane & 7) == 0 && n0 < hi) bm[n0 >> 5] = word;
-            // Candidates: one atomic per warp and load round that has any.
-            const uint32_t cnt = __popc(cmask);
-            if (__any_sync(kFullMask, cnt != 0)) {
-                uint32_t incl = cnt;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t y = __shfl_up_sync(kFullMask, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                uint32_t slot = 0;
-                if (lane == 31) slot = atomicAdd(a.cand_cnt + u, incl);
-                slot = __shfl_sync(kFullMask, slot, 31) + incl - cnt;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    if (cmask >> e & 1u) {
-                        if (slot < (uint32_t)a.cap) a.cand[u * a.cap + slot] = make_uint2((uint32_t)(n0 + e), vals[e]);
-                        ++slot;
-                    }
+                if (cmask >> e & 1u) {
+                    // slot < ncand <= cap: the slice's candidates are a subset of the unit's
+                    if (slot < (uint32_t)a.cap) scand[slot] = make_uint2((uint32_t)(n0 + e), vals[e]);
+                    ++slot;
                 }
             }
         }
+    }
+    __syncthreads();
+    // The CTA's candidates -> the unit list (one global atomic per CTA).
+    {
+        const uint32_t nl = min(sh.count, (uint32_t)a.cap);
+        if (tid == 0 && nl) sh.base = atomicAdd(a.cand_cnt + u, nl);
+        __syncthreads();
+        const uint32_t base = sh.base;
+        uint2* cu = a.cand + u * a.cap;
+        for (uint32_t i = tid; i < nl; i += kThreads)
+            if (base + i < (uint32_t)a.cap) cu[base + i] = scand[i];
     }
 
     // ---- the unit's last CTA to get here selects.
@@ -296,10 +327,9 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     __threadfence();
 
     int32_t* out = a.idx_out + u * (int64_t)a.k;
-    const uint32_t ncand = __ldcg(a.unit_hist + u * kScoreHistBins + d0);  // == candidates appended
-    if (ncand > (uint32_t)a.cap) {
-        // The threshold bin holds more keys than the list: three digits over
-        // all of the unit's scores, then a compaction pass over them.
+    if (!fits) {
+        // The threshold bin holds more keys than the candidate list: three
+        // digits over all of the unit's scores, then a compaction pass.
         uint32_t prefix = 0, mask = 0, krem = (uint32_t)a.k;
         auto get = [&](int i) { return __ldcg(su + i); };
         radix_digit(sh, a.N, get, 20, 0x7ffu, true, prefix, mask, krem);
@@ -310,59 +340,79 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         return;
     }
 
-    // ---- the krem0-th largest among the candidates: digits 18-8 and 7-0.
-    const uint2* cu = a.cand + u * a.cap;
+    // The first bitmap tile is fetched while the candidates are ranked.
+    const int words = (a.N + 31) / 32;
+    uint4 tw[kWordsPerThread / 4];
+    auto load_tile = [&](int w0) {
+#pragma unroll
+        for (int q = 0; q < kWordsPerThread / 4; ++q) {
+            // Rows are padded to whole 16-byte groups; words past the last key are dropped.
+            const int wi = w0 + tid * kWordsPerThread + 4 * q;
+            uint4 x = wi < words ? __ldcg(reinterpret_cast<const uint4*>(bm + wi)) : make_uint4(0, 0, 0, 0);
+            if (wi + 1 >= words) x.y = 0u;
+            if (wi + 2 >= words) x.z = 0u;
+            if (wi + 3 >= words) x.w = 0u;
+            tw[q] = x;
+        }
+    };
+    load_tile(0);
+
+    // ---- the unit's candidates in shared memory; the krem0-th largest among
+    // them: digits 18-8 and 7-0.
     const int nc = (int)ncand;
-    uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
     {
-        auto get = [&](int i) { return __ldcg(&cu[i].y); };
-        radix_digit(sh, nc, get, 8, 0x7ffu, true, prefix, mask, need);
-        radix_digit(sh, nc, get, 0, 0xffu, true, prefix, mask, need);
+        const uint2* cu = a.cand + u * a.cap;
+        for (int i = tid; i < nc; i += kThreads) scand[i] = __ldcg(cu + i);
+        __syncthreads();
     }
-    const uint32_t t = prefix;
-    // Ties at t: if more than `need`, keep the `need` lowest indices, i.e.
-    // those at or below the need-th smallest tie index ti.
-    uint32_t ties = 0;
-    for (int i = tid; i < nc; i += kThreads) ties += __ldcg(&cu[i].y) == t;
-    uint32_t ties_total;
-    block_exclusive_scan(ties, sh.warp_sums, ties_total);
+    uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
+    auto bits_of = [&](int i) { return scand[i].y; };
+    radix_digit(sh, nc, bits_of, 8, 0x7ffu, true, prefix, mask, need);
+    radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
+    const uint32_t t = prefix, ties_total = sh.count;  // keys equal to t
+    // Ties at t beyond `need`: keep the `need` lowest indices, i.e. those at
+    // or below the need-th smallest tie index ti (digits 30-20, 19-9, 8-0 of
+    // the ties' indices, ascending; non-ties map to 2^32 - 1 and never match).
     uint32_t ti = 0xffffffffu;
     if (ties_total > need) {
-        uint32_t ik = need;
-        // Indices below 2^31: digits 30-20, 19-9, 8-0 of the ties' indices, ascending.
-        auto get = [&](int i) {
-            const uint2 e = __ldcg(&cu[i]);
-            return e.y == t ? e.x : 0xffffffffu;  // non-ties never match the prefix once bit 31 is fixed
+        auto idx_of_tie = [&](int i) {
+            const uint2 e = scand[i];
+            return e.y == t ? e.x : 0xffffffffu;
         };
-        uint32_t p31 = 0, m31 = 0x80000000u;
-        radix_digit(sh, nc, [&](int i) { return get(i); }, 20, 0x7ffu, false, p31, m31, ik);
-        radix_digit(sh, nc, [&](int i) { return get(i); }, 9, 0x7ffu, false, p31, m31, ik);
-        radix_digit(sh, nc, [&](int i) { return get(i); }, 0, 0x1ffu, false, p31, m31, ik);
-        ti = p31;
+        uint32_t ip = 0, im = 0x80000000u, ik = need;
+        radix_digit(sh, nc, idx_of_tie, 20, 0x7ffu, false, ip, im, ik);
+        radix_digit(sh, nc, idx_of_tie, 9, 0x7ffu, false, ip, im, ik);
+        radix_digit(sh, nc, idx_of_tie, 0, 0x1ffu, false, ip, im, ik);
+        ti = ip;
     }
-    // Clear the bits of the candidates that are not selected.
-    for (int i = tid; i < nc; i += kThreads) {
-        const uint2 e = __ldcg(&cu[i]);
-        const bool keep = e.y > t || (e.y == t && e.x <= ti);
-        if (!keep) atomicAnd(bm + (e.x >> 5), ~(1u << (e.x & 31)));
-    }
-    __threadfence();
-    __syncthreads();
 
-    // ---- selected keys in index order from the bitmap: tiles of
-    // kThreads x 8 words, each thread a run of consecutive words.
-    const int words = (a.N + 31) / 32;
+    // ---- selected keys in index order, tile by tile of the bitmap: the
+    // tile's words in shared memory, the candidates that are not selected
+    // cleared there, then each thread's run of consecutive words written out
+    // from one block-wide scan of their population counts.
     uint32_t out_base = 0;
-    for (int w0 = 0; w0 < words; w0 += kThreads * kWordsPerThread) {
-        const int wt = w0 + tid * kWordsPerThread;
+    for (int w0 = 0; w0 < words; w0 += kTileWords) {
+#pragma unroll
+        for (int q = 0; q < kWordsPerThread / 4; ++q)
+            *reinterpret_cast<uint4*>(sbits + tid * kWordsPerThread + 4 * q) = tw[q];
+        __syncthreads();
+        if (w0 + kTileWords < words) load_tile(w0 + kTileWords);
+        const uint32_t klo = 32u * (uint32_t)w0, khi = klo + 32u * kTileWords;
+        for (int i = tid; i < nc; i += kThreads) {
+            const uint2 e = scand[i];
+            const bool keep = e.y > t || (e.y == t && e.x <= ti);
+            if (!keep && e.x >= klo && e.x < khi) atomicAnd(sbits + ((e.x - klo) >> 5), ~(1u << (e.x & 31)));
+        }
+        __syncthreads();
         uint32_t wv[kWordsPerThread];
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread; ++q) wv[q] = wt + q < words ? __ldcg(bm + wt + q) : 0u;
+        for (int q = 0; q < kWordsPerThread; ++q) wv[q] = sbits[tid * kWordsPerThread + q];
         uint32_t cnt = 0;
 #pragma unroll
         for (int q = 0; q < kWordsPerThread; ++q) cnt += __popc(wv[q]);
         uint32_t total;
         uint32_t pos = out_base + block_exclusive_scan(cnt, sh.warp_sums, total);
+        const int wt = w0 + tid * kWordsPerThread;
 #pragma unroll
         for (int q = 0; q < kWordsPerThread; ++q) {
             uint32_t x = wv[q];
@@ -384,6 +434,12 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
 
 int topk_candidate_capacity(int64_t Ncap) { return (int)min64(Ncap, (int64_t)kTopkCandidates); }
 
+int64_t topk_bitmap_stride(int64_t Ncap) { return (Ncap / 32 + 3) / 4 * 4; }
+
+namespace {
+int topk_smem_bytes(int cap) { return (int)sizeof(uint2) * cap + 4 * kTileWords; }
+}  // namespace
+
 cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
                         uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
                         cudaStream_t stream)
@@ -397,13 +453,15 @@ cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t
     a.done = done;
     a.idx_out = idx_out;
     a.Ncap = s.Ncap;
+    a.bm_stride = topk_bitmap_stride(s.Ncap);
     a.N = (int)s.N;
     a.k = s.k;
     a.C = (int)((s.N + kSliceKeys - 1) / kSliceKeys);
     a.cap = topk_candidate_capacity(s.Ncap);
-    cudaError_t e = set_smem_limit_once((const void*)topk_kernel, 0);
+    cudaError_t e = set_smem_limit_once((const void*)topk_kernel, topk_smem_bytes(kTopkCandidates));
     if (e != cudaSuccess) return e;
-    return launch_pdl(topk_kernel, dim3((unsigned)(s.U * a.C)), dim3(kThreads), 0, stream, a);
+    return launch_pdl(topk_kernel, dim3((unsigned)(s.U * a.C)), dim3(kThreads), (size_t)topk_smem_bytes(a.cap),
+                      stream, a);
 }
 
 }  // namespace socket_attn

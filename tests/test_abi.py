@@ -51,6 +51,15 @@ def test_version(lib):
     assert lib.socket_version() == 200
 
 
+def test_wait_limit_diagnostic_round_trips(lib):
+    """socket_set_wait_limit returns the previous limit; 0xffffffff restores
+    the default (host state only, nothing launched)."""
+    default = lib.socket_set_wait_limit(7)
+    assert default == 1 << 22
+    assert lib.socket_set_wait_limit(0xFFFFFFFF) == 7
+    assert lib.socket_set_wait_limit(0xFFFFFFFF) == default
+
+
 # Fake, aligned, never-dereferenced device addresses: every call below fails
 # validation before it could touch them.
 P16 = 0x10000
