@@ -28,7 +28,7 @@
 // A region starts at a 64 KB-aligned shared address, so one byte-permute of
 // the packed id word (id into byte 1, lane column in byte 0) gives the row
 // address and the round's column is the load's immediate offset: a lookup is
-// one PRMT, one LDS and one FADD.  Each warp streams its batches (KEYS
+// one PRMT, one LDS and half a packed two-key FADD.  Each warp streams its batches (KEYS
 // consecutive 32-key chunks of id pieces and norms, one bulk copy each) into
 // its own ring of shared-memory stages on mbarriers, and reads them back with
 // conflict-free 16-byte loads; ids and norms stream through L2 with an
@@ -58,18 +58,26 @@ constexpr int kHistShift = kScoreHistShift;
 // allocation; the histogram and the copy rings use the space around them.
 constexpr int kSmemBytes = 226 * 1024;
 constexpr uint32_t kMaxPolls = 1u << 22;
-#ifndef SCORE_R1
-#define SCORE_R1 2
-#endif
-#ifndef SCORE_NS1
-#define SCORE_NS1 2
-#endif
+
 
 __device__ __forceinline__ float lds_f32(uint32_t addr)
 {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
+}
+
+// (a, b) += (x, y) as one packed float32x2 add (round to nearest), the same
+// two float32 additions as a += x and b += y.
+__device__ __forceinline__ void add_f32x2(float& a, float& b, float x, float y)
+{
+    asm("{.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%0, %1};\n\t"
+        "mov.b64 rb, {%2, %3};\n\t"
+        "add.rn.f32x2 ra, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, ra;}"
+        : "+f"(a), "+f"(b)
+        : "f"(x), "f"(y));
 }
 
 __device__ __forceinline__ uint4 lds_u4(uint32_t addr)
@@ -302,12 +310,18 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     const int q = bl * 32 + r;  // id byte within this launch's part of the row
+                    // byte 1 <- the id (row), bytes 0, 2, 3 <- region and lane column
+                    auto row = [&](int j) {
+                        return __byte_perm(base, word_of(v[j][q >> 4], (q >> 2) & 3), 0x3240u | ((q & 3) << 4));
+                    };
+                    if constexpr (KEYS % 2 == 0) {
+                        // two keys' sums advance in one packed float32x2 add
 #pragma unroll
-                    for (int j = 0; j < KEYS; ++j) {
-                        // byte 1 <- the id (row), bytes 0, 2, 3 <- region and lane column
-                        const uint32_t row =
-                            __byte_perm(base, word_of(v[j][q >> 4], (q >> 2) & 3), 0x3240u | ((q & 3) << 4));
-                        acc[j] += lds_f32(row + 4u * r);
+                        for (int j = 0; j < KEYS; j += 2)
+                            add_f32x2(acc[j], acc[j + 1], lds_f32(row(j) + 4u * r), lds_f32(row(j + 1) + 4u * r));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < KEYS; ++j) acc[j] += lds_f32(row(j) + 4u * r);
                     }
                 }
             }
@@ -401,8 +415,8 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
         a.last = b0 + nb == a.nblk;
         cudaError_t e;
         if (nb == 1)
-            e = a.first ? launch_one<1, SCORE_R1, 2, SCORE_NS1, true, true>(a, grid, stream)
-                        : launch_one<1, SCORE_R1, 2, SCORE_NS1, false, true>(a, grid, stream);
+            e = a.first ? launch_one<1, 2, 2, 2, true, true>(a, grid, stream)
+                        : launch_one<1, 2, 2, 2, false, true>(a, grid, stream);
         else if (a.first)
             e = a.last ? launch_one<2, 2, 1, 2, true, true>(a, grid, stream)
                        : launch_one<2, 2, 1, 2, true, false>(a, grid, stream);
