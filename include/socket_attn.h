@@ -260,6 +260,96 @@ int socket_decode_static(const void* q, int q_dtype, const uint16_t* W,
                          int32_t* idx_out, float* out, float* scores_out, void* stream);
 
 /*
+ * Sequence-sharded decode -- one sequence's cache split by position over S
+ * shards (e.g. S GPUs, one rank each), with the same selection and output
+ * as socket_decode over the whole cache.  The method's pages claim scaling
+ * to contexts of millions of tokens ([ES] "Significado y Afirmaciones";
+ * [DE] "Bedeutung und Behauptungen") but describe no multi-device scheme;
+ * this one rests on a fact of the selection: a key of the global top-k is in
+ * its own shard's top-k (fewer than k keys of that shard beat it; ties go to
+ * the lower index everywhere), so each shard selects locally, the shards
+ * exchange k (score, global index) pairs per kv head, re-select, attend over
+ * the selected keys they hold, and merge their softmax states.  Per step:
+ *   1. socket_shard_select on every shard;
+ *   2. gather the pairs of all shards in shard order (an all-gather);
+ *   3. socket_shard_merge on every shard (the same global selection
+ *      everywhere, plus each shard's own rows);
+ *   4. socket_shard_attend on every shard;
+ *   5. gather the partial outputs and states, socket_shard_combine.
+ * Shard s holds global keys [n_offset_s, n_offset_s + N_s), the shards in
+ * increasing order of n_offset with no gaps or overlaps; every shard uses the
+ * same W, q, L, P, tau and k.  Global indices stay below 2^31.
+ *
+ * socket_shard_select -- steps a2-a4 on this shard's keys (its own cache
+ * arrays, laid out as for socket_decode with N = N_s keys):
+ *   cand_score, cand_index  device out, [B][Hkv][k] float32 / int32: the
+ *             shard's min(k, N_s) selected keys in increasing index order,
+ *             (score, n_offset + local index); slots past min(k, N_s) hold
+ *             (-1, -1).
+ *   workspace  as for socket_decode: socket_decode_workspace_size with this
+ *             shard's Ncap and k' = min(k, N_s).
+ * Preconditions as for socket_decode with N = N_s >= 1;
+ * 0 <= n_offset, n_offset + N_s < 2^31.
+ */
+int socket_shard_select(const void* q, int q_dtype, const uint16_t* W,
+                        const uint8_t* ids, const float* vnorm,
+                        int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d,
+                        int L, int P, double tau, int k, int64_t n_offset,
+                        void* workspace, size_t workspace_bytes,
+                        float* cand_score, int32_t* cand_index, void* stream);
+
+/*
+ * socket_shard_merge -- step a4 across shards: from the S shards' pairs,
+ * cand_score / cand_index [S][B][Hkv][k] (shard order), the k with the
+ * largest scores, ties to the lower index, in increasing index order:
+ *   idx_out      device out, [B][Hkv][k] int32 global indices (as
+ *                socket_decode's idx_out; -1 past the number of pairs when
+ *                the shards hold fewer than k keys together).
+ *   local_idx    device out, [B][Hkv][k] int32: the selected keys in
+ *                [n_offset, n_offset + n_local) (the calling shard's),
+ *                as local indices, increasing.
+ *   local_count  device out, [B][Hkv] int32: how many of them.
+ * Arrays 4-byte aligned.  S >= 1, S * k <= 2^30.
+ */
+int socket_shard_merge(const float* cand_score, const int32_t* cand_index, int S,
+                       int64_t B, int64_t Hkv, int k, int64_t n_offset, int64_t n_local,
+                       int32_t* idx_out, int32_t* local_idx, int32_t* local_count, void* stream);
+
+/*
+ * socket_shard_attend_workspace_size -- bytes of device scratch that
+ * socket_shard_attend needs for these sizes (256-byte aligned), or 0 if the
+ * sizes are invalid.
+ */
+size_t socket_shard_attend_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int k);
+
+/*
+ * socket_shard_attend -- step a5 on this shard's share of the selection:
+ * for each query row, softmax attention (scale 1/sqrt(d)) over the
+ * local_count[b][h] keys local_idx[b][h][0 ..) of its kv head, in the
+ * shard's own K and V ([B][Hkv][Ncap][d]):
+ *   out  device out, [B][Hq][d] float32, normalised over those keys (0 for a
+ *        kv head with none);
+ *   ml   device out, [B][Hq][2] float32: the largest logit m and the sum l
+ *        of exp(logit - m) over those keys (l = 0 when there are none).
+ * The workspace (socket_shard_attend_workspace_size) is cleared by the call
+ * itself.  Alignment as for socket_decode; ml 8-byte aligned.
+ */
+int socket_shard_attend(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
+                        int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int k,
+                        const int32_t* local_idx, const int32_t* local_count,
+                        void* workspace, size_t workspace_bytes, float* out, float* ml, void* stream);
+
+/*
+ * socket_shard_combine -- the log-sum-exp merge of the S shards' partial
+ * results, outs [S][B][Hq][d] and mls [S][B][Hq][2] (shard order): per query
+ * row, out = sum_s w_s o_s / sum_s w_s with w_s = exp(m_s - M) l_s over the
+ * shards with l_s > 0, M their largest m_s.  out [B][Hq][d] float32.
+ * outs and out 16-byte aligned, mls 8-byte.  d == 128.
+ */
+int socket_shard_combine(const float* outs, const float* mls, int S, int64_t B, int64_t Hq, int64_t d,
+                         float* out, void* stream);
+
+/*
  * socket_last_error -- message for the last non-OK status returned on the
  * calling host thread ("" if none).  The pointer stays valid until the next
  * call on that thread.

@@ -22,7 +22,8 @@ __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
     "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check", "socket_decode_append",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events",
-    "socket_set_wait_limit", "library_path", "load_library",
+    "socket_set_wait_limit", "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
+    "socket_shard_attend_workspace_size", "socket_shard_combine", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
 
@@ -83,6 +84,18 @@ def load_library(path: str | None = None):
     lib.socket_last_error.restype = ctypes.c_char_p
     lib.socket_set_step_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), _int]
     lib.socket_set_step_events.restype = _int
+    lib.socket_shard_select.argtypes = [_vp, _int, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int,
+                                        _dbl, _int, _i64, _vp, _sz, _vp, _vp, _vp]
+    lib.socket_shard_select.restype = _int
+    lib.socket_shard_merge.argtypes = [_vp, _vp, _int, _i64, _i64, _int, _i64, _i64, _vp, _vp, _vp, _vp]
+    lib.socket_shard_merge.restype = _int
+    lib.socket_shard_attend_workspace_size.argtypes = [_i64, _i64, _i64, _i64, _i64, _int]
+    lib.socket_shard_attend_workspace_size.restype = _sz
+    lib.socket_shard_attend.argtypes = [_vp, _int, _vp, _vp, _int, _i64, _i64, _i64, _i64, _i64, _int, _vp, _vp,
+                                        _vp, _sz, _vp, _vp, _vp]
+    lib.socket_shard_attend.restype = _int
+    lib.socket_shard_combine.argtypes = [_vp, _vp, _int, _i64, _i64, _i64, _vp, _vp]
+    lib.socket_shard_combine.restype = _int
     lib.socket_set_wait_limit.argtypes = [ctypes.c_uint32]
     lib.socket_set_wait_limit.restype = ctypes.c_uint32
     lib.socket_ids_row_bytes.argtypes = [_int]
@@ -309,6 +322,105 @@ def socket_set_step_events(events) -> None:
     n = len(events)
     arr = (ctypes.c_void_p * max(n, 1))(*[ctypes.c_void_p(int(e.cuda_event)) for e in events])
     _raise(lib.socket_set_step_events(arr, n))
+
+
+def _check_workspace(workspace: torch.Tensor, dev):
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1 or not workspace.is_cuda or workspace.device != dev:
+        raise ValueError("workspace must be a 1-D uint8 CUDA tensor on the inputs' device")
+
+
+def socket_shard_select(q: torch.Tensor, W: torch.Tensor, ids: torch.Tensor, vnorm: torch.Tensor, N: int,
+                        tau: float, k: int, n_offset: int, workspace: torch.Tensor, cand_score: torch.Tensor,
+                        cand_index: torch.Tensor, stream=None) -> None:
+    """This shard's own top-k as (score, global index) pairs (see the header).
+
+    q: [B, Hq, 128]; W: [L, P, 128] bfloat16; ids, vnorm: this shard's cache
+    index ([B, Hkv, ...] as for socket_decode, N keys); workspace of
+    >= socket_decode_workspace_size(..., min(k, N)) bytes; cand_score: [B, Hkv, k]
+    float32; cand_index: [B, Hkv, k] int32."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    L, P, _ = W.shape
+    Hkv, Ncap = vnorm.shape[1], vnorm.shape[2]
+    dev = q.device
+    _check(q, "q", (B, Hq, d), device=dev)
+    _check(W, "W", (L, P, d), dtype=torch.bfloat16, device=dev)
+    _check(ids, "ids", ids_shape(B, Hkv, Ncap, L), dtype=torch.uint8, device=dev)
+    _check(vnorm, "vnorm", (B, Hkv, Ncap), dtype=torch.float32, device=dev)
+    _check(cand_score, "cand_score", (B, Hkv, k), dtype=torch.float32, device=dev)
+    _check(cand_index, "cand_index", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check_workspace(workspace, dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_shard_select(q.data_ptr(), _code(q), W.data_ptr(), ids.data_ptr(), vnorm.data_ptr(), B, Hq,
+                                       Hkv, Ncap, int(N), d, L, P, float(tau), int(k), int(n_offset),
+                                       workspace.data_ptr(), workspace.numel(), cand_score.data_ptr(),
+                                       cand_index.data_ptr(), _stream_handle(stream)))
+
+
+def socket_shard_merge(cand_score: torch.Tensor, cand_index: torch.Tensor, n_offset: int, n_local: int,
+                       idx_out: torch.Tensor, local_idx: torch.Tensor, local_count: torch.Tensor,
+                       stream=None) -> None:
+    """The global top-k from all shards' pairs, cand_score / cand_index
+    [S, B, Hkv, k] in shard order: idx_out [B, Hkv, k] int32 (global),
+    local_idx [B, Hkv, k] int32 and local_count [B, Hkv] int32 (this shard's
+    keys [n_offset, n_offset + n_local) among them, as local indices)."""
+    lib = load_library()
+    S, B, Hkv, k = cand_score.shape
+    dev = cand_score.device
+    _check(cand_score, "cand_score", (S, B, Hkv, k), dtype=torch.float32, device=dev)
+    _check(cand_index, "cand_index", (S, B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(idx_out, "idx_out", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(local_idx, "local_idx", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(local_count, "local_count", (B, Hkv), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_shard_merge(cand_score.data_ptr(), cand_index.data_ptr(), S, B, Hkv, k, int(n_offset),
+                                      int(n_local), idx_out.data_ptr(), local_idx.data_ptr(), local_count.data_ptr(),
+                                      _stream_handle(stream)))
+
+
+def socket_shard_attend_workspace_size(B: int, Hq: int, Hkv: int, Ncap: int, k: int) -> int:
+    n = int(load_library().socket_shard_attend_workspace_size(B, Hq, Hkv, Ncap, HEAD_DIM, k))
+    if n == 0:
+        raise ValueError("invalid sizes for socket_shard_attend")
+    return n
+
+
+def socket_shard_attend(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, k: int, local_idx: torch.Tensor,
+                        local_count: torch.Tensor, workspace: torch.Tensor, out: torch.Tensor, ml: torch.Tensor,
+                        stream=None) -> None:
+    """Attention over this shard's share of the selection: out [B, Hq, 128]
+    float32 (normalised over those keys) and ml [B, Hq, 2] float32 (largest
+    logit, sum of weights)."""
+    lib = load_library()
+    B, Hq, d = q.shape
+    _, Hkv, Ncap, _ = K.shape
+    dev = q.device
+    _check(q, "q", (B, Hq, d), device=dev)
+    _check(K, "K", (B, Hkv, Ncap, d), device=dev)
+    _check(V, "V", (B, Hkv, Ncap, d), dtype=K.dtype, device=dev)
+    _check(local_idx, "local_idx", (B, Hkv, k), dtype=torch.int32, device=dev)
+    _check(local_count, "local_count", (B, Hkv), dtype=torch.int32, device=dev)
+    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
+    _check(ml, "ml", (B, Hq, 2), dtype=torch.float32, device=dev)
+    _check_workspace(workspace, dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_shard_attend(q.data_ptr(), _code(q), K.data_ptr(), V.data_ptr(), _code(K), B, Hq, Hkv, Ncap,
+                                       d, int(k), local_idx.data_ptr(), local_count.data_ptr(), workspace.data_ptr(),
+                                       workspace.numel(), out.data_ptr(), ml.data_ptr(), _stream_handle(stream)))
+
+
+def socket_shard_combine(outs: torch.Tensor, mls: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Log-sum-exp merge of the shards' partial results outs [S, B, Hq, 128]
+    and mls [S, B, Hq, 2] into out [B, Hq, 128] float32."""
+    lib = load_library()
+    S, B, Hq, d = outs.shape
+    dev = outs.device
+    _check(outs, "outs", (S, B, Hq, d), dtype=torch.float32, device=dev)
+    _check(mls, "mls", (S, B, Hq, 2), dtype=torch.float32, device=dev)
+    _check(out, "out", (B, Hq, d), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _raise(lib.socket_shard_combine(outs.data_ptr(), mls.data_ptr(), S, B, Hq, d, out.data_ptr(),
+                                        _stream_handle(stream)))
 
 
 def socket_set_wait_limit(polls: int) -> int:

@@ -120,6 +120,34 @@ size_t workspace_size(bool per_head, int64_t B, int64_t Hq, int64_t Hkv, int64_t
     return decode_workspace_layout(s).total;
 }
 
+// Scratch of socket_shard_attend: error word, merge counters, split partials.
+struct AttendWorkspace {
+    size_t counters, part_o, part_ml, total;
+};
+AttendWorkspace attend_layout(const DecodeShape& s)
+{
+    AttendWorkspace w;
+    size_t off = align256(4);  // error word at 0
+    w.counters = off;
+    off = align256(off + 4 * (size_t)s.U);
+    w.part_o = off;
+    off = align256(off + 4 * (size_t)s.U * s.G * s.nsplit * s.d);
+    w.part_ml = off;
+    off = align256(off + 8 * (size_t)s.U * s.G * s.nsplit);
+    w.total = off;
+    return w;
+}
+
+// Shape of an attention-only call (no hashing parameters involved).  k is
+// the row capacity of the selection lists, which may exceed this shard's keys.
+int fill_attend_shape(DecodeShape& s, int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int k)
+{
+    if (k < 1) return fail(SOCKET_EINVAL, "k=%d must be >= 1", k);
+    const int st = fill_shape(s, B, Hq, Hkv, Ncap, Ncap, d, 1, 1, (int)(k < Ncap ? k : Ncap));
+    s.k = k;
+    return st;
+}
+
 }  // namespace
 
 cudaError_t set_smem_limit_once(const void* func, int bytes)
@@ -205,6 +233,8 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 4 * (size_t)s.U * s.G * s.nsplit * s.d);
     w.part_ml = off;
     off = align256(off + 8 * (size_t)s.U * s.G * s.nsplit);
+    w.sel_idx = off;
+    off = align256(off + 4 * (size_t)s.U * s.k);
     w.total = off;
     return w;
 }
@@ -282,8 +312,8 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
                      "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
-    st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, s, part_o, part_ml, counters, err_word,
-                                      out, cs),
+    st = cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, idx_out, nullptr, s, part_o, part_ml, counters,
+                                      err_word, out, nullptr, cs),
                      "attention kernel launch");
     if (st != SOCKET_OK) return st;
     return cuda_status(mark_step(4, cs), "step event record");
@@ -389,6 +419,140 @@ int socket_decode_per_head(const void* q, int q_dtype, const uint16_t* W, const 
 {
     return decode(true, q, q_dtype, W, ids, vnorm, K, V, kv_dtype, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, workspace,
                   workspace_bytes, idx_out, out, scores_out, static_cast<cudaStream_t>(stream));
+}
+
+
+int socket_shard_select(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
+                        int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t N, int64_t d, int L, int P,
+                        double tau, int k, int64_t n_offset, void* workspace, size_t workspace_bytes,
+                        float* cand_score, int32_t* cand_index, void* stream)
+{
+    g_last_error.clear();
+    if (k < 1) return fail(SOCKET_EINVAL, "k=%d must be >= 1", k);
+    if (N < 1) return fail(SOCKET_EINVAL, "a shard holds at least one key (N=%lld)", (long long)N);
+    const int k_eff = (int)(N < k ? N : k);
+    DecodeShape s;
+    int st = fill_shape(s, B, Hq, Hkv, Ncap, N, d, L, P, k_eff);
+    if (st != SOCKET_OK) return st;
+    if (!valid_dtype(q_dtype)) return fail(SOCKET_EINVAL, "q_dtype=%d unknown", q_dtype);
+    if (!(tau >= 0.0) || !isfinite(tau)) return fail(SOCKET_EINVAL, "tau=%g must be finite and >= 0", tau);
+    if (n_offset < 0 || n_offset + N > (int64_t(1) << 31) - 1)
+        return fail(SOCKET_EINVAL, "n_offset=%lld: global indices must stay below 2^31", (long long)n_offset);
+    if (!q || !W || !ids || !vnorm || !workspace || !cand_score || !cand_index)
+        return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(W, 16) || !aligned(ids, 16) || !aligned(vnorm, 16) || !aligned(cand_score, 4) ||
+        !aligned(cand_index, 4))
+        return fail(SOCKET_EINVAL, "q, W, ids, vnorm must be 16-byte aligned, cand_score and cand_index 4-byte");
+    if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
+    const size_t need = workspace_size(false, B, Hq, Hkv, Ncap, d, L, P, k_eff);
+    if (workspace_bytes < need)
+        return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    s.nsplit = 0;  // no attention here
+    const DecodeWorkspace w = decode_workspace_layout(s);
+    char* base = static_cast<char*>(workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    uint32_t* err_word = reinterpret_cast<uint32_t*>(base + w.err);
+    float* scores = reinterpret_cast<float*>(base + w.scores);
+    int32_t* sel = reinterpret_cast<int32_t*>(base + w.sel_idx);
+    AppendHash none;
+    st = cuda_status(launch_soft_tables(q, q_dtype, W, s, tau, none, reinterpret_cast<float*>(base + w.tables), err_word,
+                                        reinterpret_cast<uint32_t*>(base + w.counters),
+                                        reinterpret_cast<uint32_t*>(base + w.topk_done),
+                                        reinterpret_cast<uint32_t*>(base + w.unit_hist),
+                                        reinterpret_cast<uint32_t*>(base + w.cand_cnt), cs),
+                     "soft-table kernel launch");
+    if (st != SOCKET_OK) return st;
+    st = cuda_status(launch_score(reinterpret_cast<float*>(base + w.tables), ids, vnorm, s, Ncap / 32, scores,
+                                  reinterpret_cast<uint32_t*>(base + w.unit_hist), err_word, cs),
+                     "score kernel launch");
+    if (st != SOCKET_OK) return st;
+    st = cuda_status(launch_topk(scores, reinterpret_cast<uint32_t*>(base + w.unit_hist),
+                                 reinterpret_cast<uint32_t*>(base + w.cand_cnt), reinterpret_cast<uint2*>(base + w.cand),
+                                 reinterpret_cast<uint32_t*>(base + w.bitmap),
+                                 reinterpret_cast<uint32_t*>(base + w.topk_done), s, sel, cs),
+                     "top-k kernel launch");
+    if (st != SOCKET_OK) return st;
+    return cuda_status(launch_shard_pairs(scores, sel, s, k_eff, k, n_offset, cand_score, cand_index, cs),
+                       "shard pair kernel launch");
+}
+
+int socket_shard_merge(const float* cand_score, const int32_t* cand_index, int S, int64_t B, int64_t Hkv, int k,
+                       int64_t n_offset, int64_t n_local, int32_t* idx_out, int32_t* local_idx, int32_t* local_count,
+                       void* stream)
+{
+    g_last_error.clear();
+    if (S < 1 || k < 1 || B < 1 || Hkv < 1) return fail(SOCKET_EINVAL, "S, k, B, Hkv must be >= 1");
+    if (B * Hkv > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hkv=%lld above 65535", (long long)(B * Hkv));
+    if ((int64_t)S * k > (int64_t(1) << 30)) return fail(SOCKET_EUNSUPPORTED, "S*k above 2^30");
+    if (n_offset < 0 || n_local < 0) return fail(SOCKET_EINVAL, "n_offset and n_local must be >= 0");
+    if (!cand_score || !cand_index || !idx_out || !local_idx || !local_count)
+        return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(cand_score, 4) || !aligned(cand_index, 4) || !aligned(idx_out, 4) || !aligned(local_idx, 4) ||
+        !aligned(local_count, 4))
+        return fail(SOCKET_EINVAL, "arrays must be 4-byte aligned");
+    return cuda_status(launch_shard_merge(cand_score, cand_index, S, B * Hkv, k, n_offset, n_local, idx_out, local_idx,
+                                          local_count, static_cast<cudaStream_t>(stream)),
+                       "shard merge kernel launch");
+}
+
+size_t socket_shard_attend_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int k)
+{
+    DecodeShape s;
+    const std::string saved = g_last_error;
+    if (fill_attend_shape(s, B, Hq, Hkv, Ncap, d, k) != SOCKET_OK) {
+        g_last_error = saved;
+        return 0;
+    }
+    s.nsplit = (k + 15) / 16;  // attention splits never exceed ceil(k / 16)
+    return attend_layout(s).total;
+}
+
+int socket_shard_attend(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype, int64_t B,
+                        int64_t Hq, int64_t Hkv, int64_t Ncap, int64_t d, int k, const int32_t* local_idx,
+                        const int32_t* local_count, void* workspace, size_t workspace_bytes, float* out, float* ml,
+                        void* stream)
+{
+    g_last_error.clear();
+    DecodeShape s;
+    int st = fill_attend_shape(s, B, Hq, Hkv, Ncap, d, k);
+    if (st != SOCKET_OK) return st;
+    if (!valid_dtype(q_dtype) || !valid_dtype(kv_dtype))
+        return fail(SOCKET_EINVAL, "q_dtype=%d / kv_dtype=%d unknown", q_dtype, kv_dtype);
+    if (!q || !K || !V || !local_idx || !local_count || !workspace || !out || !ml)
+        return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) || !aligned(ml, 8) ||
+        !aligned(local_idx, 4) || !aligned(local_count, 4))
+        return fail(SOCKET_EINVAL, "q, K, V, out must be 16-byte aligned, ml 8-byte, local_idx and local_count 4-byte");
+    if (!aligned(workspace, 256)) return fail(SOCKET_EWORKSPACE, "workspace must be 256-byte aligned");
+    const size_t need = socket_shard_attend_workspace_size(B, Hq, Hkv, Ncap, d, k);
+    if (workspace_bytes < need)
+        return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+    s.nsplit = attention_splits(kv_dtype, q_dtype, s.G, s.U, k, device_num_sms());
+    const AttendWorkspace w = attend_layout(s);
+    char* base = static_cast<char*>(workspace);
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // The error word and the merge counters start at zero.
+    if ((st = cuda_status(cudaMemsetAsync(base, 0, w.part_o, cs), "workspace clear")) != SOCKET_OK) return st;
+    return cuda_status(launch_attention(q, q_dtype, K, V, kv_dtype, local_idx, local_count, s,
+                                        reinterpret_cast<float*>(base + w.part_o),
+                                        reinterpret_cast<float2*>(base + w.part_ml),
+                                        reinterpret_cast<uint32_t*>(base + w.counters),
+                                        reinterpret_cast<uint32_t*>(base), out, reinterpret_cast<float2*>(ml), cs),
+                       "attention kernel launch");
+}
+
+int socket_shard_combine(const float* outs, const float* mls, int S, int64_t B, int64_t Hq, int64_t d, float* out,
+                         void* stream)
+{
+    g_last_error.clear();
+    if (d != SOCKET_HEAD_DIM) return fail(SOCKET_EUNSUPPORTED, "head dim d=%lld unsupported (only 128)", (long long)d);
+    if (S < 1 || B < 1 || Hq < 1) return fail(SOCKET_EINVAL, "S, B, Hq must be >= 1");
+    if (!outs || !mls || !out) return fail(SOCKET_EINVAL, "null pointer argument");
+    if (!aligned(outs, 16) || !aligned(out, 16) || !aligned(mls, 8))
+        return fail(SOCKET_EINVAL, "outs and out must be 16-byte aligned, mls 8-byte");
+    return cuda_status(launch_shard_combine(outs, reinterpret_cast<const float2*>(mls), S, B * Hq, out,
+                                            static_cast<cudaStream_t>(stream)),
+                       "shard combine kernel launch");
 }
 
 }  // extern "C"

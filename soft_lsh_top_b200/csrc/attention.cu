@@ -62,7 +62,8 @@ template <int G, int NT>
 __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
                                            const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                            uint32_t* __restrict__ counters, float* __restrict__ out,
-                                           float (*red)[G], float* wsm, uint32_t& s_last)
+                                           float2* __restrict__ ml_out, float (*red)[G], float* wsm,
+                                           uint32_t& s_last)
 {
     static_assert(kHeadDim % NT == 0 && NT % 32 == 0, "NT threads cover the head dimension evenly");
     constexpr int kCols = kHeadDim / NT;  // output columns per thread: tid, tid + NT, ...
@@ -96,7 +97,7 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
             __syncthreads();
             if (tid < cnt) {
                 const float2 t = __ldcg(&part_ml[base + s0 + tid]);
-                const float w = expf(t.x - M);
+                const float w = t.x == -INFINITY ? 0.0f : expf(t.x - M);  // empty splits weigh nothing
                 wsm[tid] = w;
                 lsum += t.y * w;
             }
@@ -123,8 +124,10 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
         float L = 0.0f;
 #pragma unroll
         for (int w = 0; w < NT / 32; ++w) L += red[w][0];
+        // No rows at all (an empty share of a sharded selection): zero output.
 #pragma unroll
-        for (int j = 0; j < kCols; ++j) out[(qrow0 + h) * kHeadDim + tid + j * NT] = acc[j] / L;
+        for (int j = 0; j < kCols; ++j) out[(qrow0 + h) * kHeadDim + tid + j * NT] = L > 0.0f ? acc[j] / L : 0.0f;
+        if (ml_out && tid == 0) ml_out[qrow0 + h] = make_float2(M, L);
     }
     if (tid == 0) counters[u] = 0u;
 }
@@ -140,9 +143,9 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
 template <typename KT, int G>
 __global__ __launch_bounds__(kThreads) void attention_kernel(
     const void* __restrict__ q, int q_dtype, const KT* __restrict__ K, const KT* __restrict__ V,
-    const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
-    float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
-    uint32_t* __restrict__ err_word, float* __restrict__ out, uint32_t max_polls)
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ counts, int share, int64_t Ncap, int k,
+    int nsplit, int rpc, float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
+    uint32_t* __restrict__ err_word, float* __restrict__ out, float2* __restrict__ ml_out, uint32_t max_polls)
 {
     constexpr int kChunk = Rows<KT>::kChunk;
     constexpr int kRowBytes = Rows<KT>::kRowBytes;
@@ -162,8 +165,6 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     const int split = blockIdx.x % nsplit;
     const int64_t ukv = u / share;  // the unit's key/value rows
     const int r_begin = split * rpc;
-    const int r_end = min(k, r_begin + rpc);
-    const int nchunks = (r_end - r_begin + kChunk - 1) / kChunk;
 
     const int64_t qrow0 = u * G;  // the unit's query rows of [B][Hq]
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
@@ -182,6 +183,11 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     }
     __syncthreads();
     pdl_wait();  // the selected indices come from the previous kernel on the stream
+    // Rows of the unit: k, or its own count when the selection is a share of a
+    // sharded one (counts, clamped to [0, k]).
+    const int rows = counts ? max(0, min(k, __ldcg(counts + u))) : k;
+    const int r_end = min(rows, r_begin + rpc);
+    const int nchunks = r_end > r_begin ? (r_end - r_begin + kChunk - 1) / kChunk : 0;
 
     // Gather chunk c into stage st: thread i < rows copies one key row and one value row.
     auto issue = [&](int c, int st) {
@@ -200,7 +206,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
         }
         if (tid == 0) mbar_arrive_expect_tx(&bar[st], (uint32_t)nr * 2u * kRowBytes);
     };
-    issue(0, 0);
+    if (nchunks > 0) issue(0, 0);
     if (nchunks > 1) issue(1, 1);
 
     float qreg[G][4];
@@ -321,7 +327,7 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
     for (int h = 0; h < G; ++h) part_o[((pbase + h * nsplit) + split) * kHeadDim + tid] = o[h];
     if (tid < G) part_ml[pbase + tid * nsplit + split] = make_float2(m_run[tid], l_run[tid]);
 
-    merge_unit<G, kThreads>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, red, wsm, s_last);
+    merge_unit<G, kThreads>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, ml_out, red, wsm, s_last);
 }
 
 // ---------------------------------------------------------------------------
@@ -376,7 +382,7 @@ template <int G>
 __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
                                                  const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                                  uint32_t* __restrict__ counters, float* __restrict__ out,
-                                                 uint32_t& s_last)
+                                                 float2* __restrict__ ml_out, uint32_t& s_last)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __threadfence();
@@ -428,9 +434,11 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(kFullMask, lsum, o);
-        const float inv = 1.0f / lsum;
+        // No rows at all (an empty share of a sharded selection): zero output.
+        const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
         reinterpret_cast<float4*>(out + (qrow0 + h) * kHeadDim)[lane] =
             make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        if (ml_out && lane == 0) ml_out[qrow0 + h] = make_float2(M, lsum);
     }
     if (tid == 0) counters[u] = 0u;
 }
@@ -438,9 +446,9 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
 template <int G>
 __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
-    const int32_t* __restrict__ idx, int share, int64_t Ncap, int k, int nsplit, int rpc,
-    float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
-    uint32_t* __restrict__ err_word, float* __restrict__ out, uint32_t max_polls)
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ counts, int share, int64_t Ncap, int k,
+    int nsplit, int rpc, float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
+    uint32_t* __restrict__ err_word, float* __restrict__ out, float2* __restrict__ ml_out, uint32_t max_polls)
 {
     static_assert(G <= 8, "heads are the M rows 0..7 of the 16-row tile");
     extern __shared__ __align__(128) char smem[];
@@ -453,9 +461,6 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const int split = blockIdx.x % nsplit;
     const int64_t ukv = u / share;  // the unit's key/value rows
     const int r_begin = split * rpc;
-    const int r_end = min(k, r_begin + rpc);
-    const int nch = (r_end - r_begin + kWChunk - 1) / kWChunk;        // chunks of this CTA
-    const int cw = nch > warp ? (nch - warp + kWWarps - 1) / kWWarps : 0;  // chunks of this warp
     const int64_t qrow0 = u * G;  // the unit's query rows of [B][Hq]
     char* wsm_base = smem + warp * kWStages * kWStageBytes;
     const uint32_t wbase = smem_addr(wsm_base);
@@ -486,6 +491,12 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     // placed now; it waits for this grid to finish before it reads anything.
     pdl_launch_dependents();
     pdl_wait();  // the selected indices come from the previous kernel on the stream
+    // Rows of the unit: k, or its own count when the selection is a share of a
+    // sharded one (counts, clamped to [0, k]).
+    const int rows = counts ? max(0, min(k, __ldcg(counts + u))) : k;
+    const int r_end = min(rows, r_begin + rpc);
+    const int nch = r_end > r_begin ? (r_end - r_begin + kWChunk - 1) / kWChunk : 0;  // chunks of this CTA
+    const int cw = nch > warp ? (nch - warp + kWWarps - 1) / kWWarps : 0;               // chunks of this warp
 
     // Row index of this lane's row (lane % 16) of chunk j, or -1 past the end.
     auto row_index = [&](int j) -> int32_t {
@@ -650,13 +661,13 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
             }
         }
     }
-    merge_unit_warps<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, s_last);
+    merge_unit_warps<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, ml_out, s_last);
 }
 
 template <int G>
-cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32_t* idx, const DecodeShape& s,
-                        float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word, float* out,
-                        cudaStream_t stream)
+cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32_t* idx, const int32_t* counts,
+                        const DecodeShape& s, float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word,
+                        float* out, float2* ml_out, cudaStream_t stream)
 {
     const int rpc = attention_rows_per_cta(s.k, s.nsplit, kWChunk);
     auto kern = attention_warp_kernel<G>;
@@ -664,16 +675,16 @@ cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
                    static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), static_cast<const uint16_t*>(V),
-                   idx, s.share, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out,
-                   wait_poll_limit());
+                   idx, counts, s.share, s.Ncap, s.k, s.nsplit, rpc, part_o, part_ml, counters, err_word, out,
+                   ml_out, wait_poll_limit());
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <typename KT, int G>
 cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, const int32_t* idx,
-                     const DecodeShape& s, float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word,
-                     float* out, cudaStream_t stream)
+                     const int32_t* counts, const DecodeShape& s, float* part_o, float2* part_ml, uint32_t* counters,
+                     uint32_t* err_word, float* out, float2* ml_out, cudaStream_t stream)
 {
     constexpr int smem = 2 * 2 * Rows<KT>::kChunk * Rows<KT>::kRowBytes;
     const int rpc = attention_rows_per_cta(s.k, s.nsplit, Rows<KT>::kChunk);
@@ -681,19 +692,20 @@ cudaError_t launch_g(const void* q, int q_dtype, const void* K, const void* V, c
     cudaError_t e = set_smem_limit_once((const void*)kern, smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kThreads), smem, stream, q, q_dtype,
-                   static_cast<const KT*>(K), static_cast<const KT*>(V), idx, s.share, s.Ncap, s.k, s.nsplit, rpc,
-                   part_o, part_ml, counters, err_word, out, wait_poll_limit());
+                   static_cast<const KT*>(K), static_cast<const KT*>(V), idx, counts, s.share, s.Ncap, s.k, s.nsplit,
+                   rpc, part_o, part_ml, counters, err_word, out, ml_out, wait_poll_limit());
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
 template <typename KT>
 cudaError_t launch_kt(const void* q, int q_dtype, const void* K, const void* V, const int32_t* idx,
-                      const DecodeShape& s, float* part_o, float2* part_ml, uint32_t* counters, uint32_t* err_word,
-                      float* out, cudaStream_t stream)
+                      const int32_t* counts, const DecodeShape& s, float* part_o, float2* part_ml, uint32_t* counters,
+                      uint32_t* err_word, float* out, float2* ml_out, cudaStream_t stream)
 {
 #define SOCKET_G_CASE(g) \
-    case g: return launch_g<KT, g>(q, q_dtype, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
+    case g:              \
+        return launch_g<KT, g>(q, q_dtype, K, V, idx, counts, s, part_o, part_ml, counters, err_word, out, ml_out, stream);
     switch (s.G) {
         SOCKET_G_CASE(1) SOCKET_G_CASE(2) SOCKET_G_CASE(3) SOCKET_G_CASE(4)
         SOCKET_G_CASE(5) SOCKET_G_CASE(6) SOCKET_G_CASE(7) SOCKET_G_CASE(8)
@@ -729,12 +741,13 @@ int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num
 }
 
 cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
-                             const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
-                             uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream)
+                             const int32_t* idx, const int32_t* counts, const DecodeShape& s, float* part_o,
+                             float2* part_ml, uint32_t* counters, uint32_t* err_word, float* out, float2* ml_out,
+                             cudaStream_t stream)
 {
     if (warp_path(kv_dtype, q_dtype, s.G)) {
 #define SOCKET_MMA_CASE(g) \
-    case g: return launch_warp<g>(q, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
+    case g: return launch_warp<g>(q, K, V, idx, counts, s, part_o, part_ml, counters, err_word, out, ml_out, stream);
         switch (s.G) {
             SOCKET_MMA_CASE(1) SOCKET_MMA_CASE(2) SOCKET_MMA_CASE(3) SOCKET_MMA_CASE(4)
             SOCKET_MMA_CASE(5) SOCKET_MMA_CASE(6) SOCKET_MMA_CASE(7) SOCKET_MMA_CASE(8)
@@ -743,8 +756,9 @@ cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const vo
 #undef SOCKET_MMA_CASE
     }
     if (kv_dtype == 1)
-        return launch_kt<uint16_t>(q, q_dtype, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
-    return launch_kt<float>(q, q_dtype, K, V, idx, s, part_o, part_ml, counters, err_word, out, stream);
+        return launch_kt<uint16_t>(q, q_dtype, K, V, idx, counts, s, part_o, part_ml, counters, err_word, out, ml_out,
+                                   stream);
+    return launch_kt<float>(q, q_dtype, K, V, idx, counts, s, part_o, part_ml, counters, err_word, out, ml_out, stream);
 }
 
 }  // namespace socket_attn

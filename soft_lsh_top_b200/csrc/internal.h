@@ -45,6 +45,7 @@ struct DecodeWorkspace {
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
     size_t part_ml;    // float2 [U][G][nsplit]
+    size_t sel_idx;    // int32 [U][k] a shard's own selection (local indices)
     size_t total;
 };
 
@@ -99,9 +100,24 @@ cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t
                         uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
                         cudaStream_t stream);
 
+// counts (nullable): rows of each unit's selection to use (the first
+// counts[u] of its k slots; all k when null).  ml_out (nullable): per query
+// row the largest logit and the sum of exp(logit - largest) over those rows
+// (the log-sum-exp state a merge across shards needs); out is normalised by
+// that sum (zero for a unit with no rows).
 cudaError_t launch_attention(const void* q, int q_dtype, const void* K, const void* V, int kv_dtype,
-                             const int32_t* idx, const DecodeShape& s, float* part_o, float2* part_ml,
-                             uint32_t* counters, uint32_t* err_word, float* out, cudaStream_t stream);
+                             const int32_t* idx, const int32_t* counts, const DecodeShape& s, float* part_o,
+                             float2* part_ml, uint32_t* counters, uint32_t* err_word, float* out, float2* ml_out,
+                             cudaStream_t stream);
+
+// --- sequence-sharded decode (shard.cu) -------------------------------------
+cudaError_t launch_shard_pairs(const float* scores, const int32_t* sel, const DecodeShape& s, int k_eff, int k,
+                               int64_t n_offset, float* cand_score, int32_t* cand_index, cudaStream_t stream);
+cudaError_t launch_shard_merge(const float* cand_score, const int32_t* cand_index, int S, int64_t U, int k,
+                               int64_t n_offset, int64_t n_local, int32_t* idx_out, int32_t* local_idx,
+                               int32_t* local_count, cudaStream_t stream);
+cudaError_t launch_shard_combine(const float* outs, const float2* mls, int S, int64_t rows, float* out,
+                                 cudaStream_t stream);
 
 // Waits for `stream`, then reads and clears the hash kernels' device error
 // bits; returns a cudaError_t value.

@@ -37,7 +37,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ("socket_hash_keys", "socket_hash_check", "socket_decode", "socket_decode_workspace_size",
                  "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_decode_append",
-                 "socket_last_error"):
+                 "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
+                 "socket_shard_attend_workspace_size", "socket_shard_combine", "socket_last_error"):
         assert want in names
 
 
@@ -236,3 +237,21 @@ def test_python_append_rejects_no_new_keys():
     z = torch.zeros(1)
     with pytest.raises(ValueError, match="n_new"):
         s.socket_decode_append(z, z, z, z, z, z, 8, 0.5, 4, 0, z, z, z)
+
+
+def test_sharded_calls_reject_bad_arguments_on_the_host(lib):
+    """The sequence-sharded entry points validate before any launch (the
+    pointers are never dereferenced)."""
+    f = P16
+    # a shard holds at least one key
+    assert lib.socket_shard_select(f, 1, f, f, f, 1, 4, 1, 64, 0, 128, 8, 8, 0.5, 8, 0, f, 1 << 30, f, f, None) == EINVAL
+    # global indices must stay below 2^31
+    assert lib.socket_shard_select(f, 1, f, f, f, 1, 4, 1, 64, 64, 128, 8, 8, 0.5, 8, (1 << 31) - 10, f, 1 << 30, f, f,
+                                   None) == EINVAL
+    assert lib.socket_shard_merge(f, f, 0, 1, 1, 8, 0, 64, f, f, f, None) == EINVAL
+    assert lib.socket_shard_merge(f, f, 2, 1, 1, 8, -1, 64, f, f, f, None) == EINVAL
+    assert lib.socket_shard_attend_workspace_size(1, 4, 1, 64, 128, 0) == 0
+    assert lib.socket_shard_attend_workspace_size(1, 4, 1, 64, 128, 8) > 0
+    assert lib.socket_shard_attend(f, 1, f, f, 1, 1, 4, 1, 64, 128, 8, f, f, f, 16, f, f, None) == EWS
+    assert lib.socket_shard_combine(f, f, 2, 1, 4, 64, f, None) == EUNSUP
+    assert lib.socket_shard_combine(f, f, 0, 1, 4, 128, f, None) == EINVAL
