@@ -18,12 +18,13 @@ namespace socket_attn {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTpb = 8;                    // tables per CTA
+constexpr int kTpb = 4;                    // tables per CTA
 constexpr int kMaxGroup = 16;
 constexpr int kMaxP = 8;
-constexpr int kRows = kTpb * kMaxP;        // hyperplane rows per CTA
-constexpr int kWRow = kHeadDim + 8;        // padded bf16 hyperplane row in shared memory (272 bytes)
-constexpr int kHeadsPerPass = 4;           // heads whose dot products share one read of a hyperplane row
+constexpr int kTpr = 8;                    // threads per hyperplane row (16 channels each)
+constexpr int kChan = kHeadDim / kTpr;     // 16
+constexpr int kQSeg = kChan + 2;           // padded fp64 segment of a query row (bank spread)
+constexpr int kHeadsPerPass = 4;           // heads whose dot products share one read of a row
 
 // bfloat16 bits (low 16) -> float64, exact.  Normal values are rebuilt with
 // integer operations (sign, exponent rebiased by 1023 - 127, the 7 mantissa
@@ -39,27 +40,27 @@ __device__ __forceinline__ double bf16_bits_to_f64(uint32_t b)
 // Dynamic shared memory of a CTA for group size G.
 __host__ __device__ constexpr int smem_bytes(int G)
 {
-    return kRows * kWRow * 2                      // hyperplane rows (bf16)
-           + G * kHeadDim * 8                     // query rows (fp64)
+    return G * kTpr * kQSeg * 8                   // query rows (fp64), one padded segment per channel slice
            + G * 8                                // per-head factor 2 / (tau ||q_h||)
            + G * kTpb * kMaxP * 2 * 8             // per-plane sigmoid pairs
            + G * kTpb * 2 * 16 * 8;               // nibble tables
 }
 
-// Grid: (U, 4 * ceil(L / 32)); CTA y covers tables 8y .. 8y + 7 (the ones
-// >= L are written as zero columns).  Block: kThreads.
-//   1. the CTA's hyperplane rows are staged in shared memory and the unit's G
-//      query rows widened to float64, with their norms;
-//   2. four threads per hyperplane row (channel octets 4s + quarter) form
-//      <W_{l,p}, q_h> for four heads per pass, so each element of W is
-//      widened once per four heads; the quarters are added by shuffles and
-//      each of the four threads turns one head's projection into the two
-//      per-plane factors sigmoid(+-2z/tau), both from one exponential;
+// Grid: (U, 8 * ceil(L / 32)); CTA y covers tables 4y .. 4y + 3 (the ones
+// >= L are written as zero columns).  Block: kThreads.  Many small CTAs keep
+// every step's dependent chain short and enough warps resident to hide it.
+//   1. the unit's G query rows are widened to float64 in shared memory, with
+//      their norms; each thread holds 16 channels of one hyperplane row
+//      (eight threads per row, 32 B each, read straight from W), widened once;
+//   2. the eight threads of a row form <W_{l,p}, q_h> for four heads per pass
+//      (partial sums added by shuffles), and thread j of the row turns head
+//      j's projection into the two per-plane factors sigmoid(+-2z/tau), both
+//      from one exponential;
 //   3. the per-plane factors of planes 0-3 and 4-7 are multiplied into two
 //      16-entry nibble tables per (head, table);
-//   4. thread b forms entry b of the CTA's eight tables,
+//   4. thread b forms entry b of the CTA's four tables,
 //      T_l(b) = sum_h lo_h(b & 15) hi_h(b >> 4), rounds it once to float32
-//      and writes the eight adjacent columns (and their copies 32 columns on)
+//      and writes the four adjacent columns (and their copies 32 columns on)
 //      of row b of the expanded layout the scoring kernel copies into shared
 //      memory: per 32-table block c a [bucket][64] row whose column j holds
 //      table 32c + j mod 32.
@@ -72,11 +73,11 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
 {
     __shared__ uint32_t aid[kMaxAppend][kTpb];  // ids of the appended keys (bit p <-> plane p)
     extern __shared__ __align__(16) char st_dyn[];
-    uint16_t* wsm = reinterpret_cast<uint16_t*>(st_dyn);                      // [kRows][kWRow]
-    double* qd = reinterpret_cast<double*>(st_dyn + kRows * kWRow * 2);        // [G][kHeadDim]
-    double* qscale = qd + G * kHeadDim;                                        // [G]
-    double* sig = qscale + G;                                                  // [G][kTpb][kMaxP][2]
-    double* nib = sig + G * kTpb * kMaxP * 2;                                  // [G][kTpb][2][16]
+    double* qd = reinterpret_cast<double*>(st_dyn);  // [G][kTpr][kQSeg]
+    double* qscale = qd + G * kTpr * kQSeg;          // [G]
+    double* sig = qscale + G;                        // [G][kTpb][kMaxP][2]
+    double* nib = sig + G * kTpb * kMaxP * 2;        // [G][kTpb][2][16]
+    auto QD = [&](int h, int c) -> double& { return qd[(h * kTpr + (c >> 4)) * kQSeg + (c & 15)]; };
     auto SIG = [&](int h, int lt, int p, int s) -> double& { return sig[((h * kTpb + lt) * kMaxP + p) * 2 + s]; };
     auto NIB = [&](int h, int lt, int hi, int v) -> double& { return nib[((h * kTpb + lt) * 2 + hi) * 16 + v]; };
 
@@ -95,35 +96,36 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     pdl_launch_dependents();
 
     if (nt > 0) {
-        // The unit's G query rows in 16-byte pieces (8 bf16 or 4 fp32 each),
-        // one or two per thread, issued before the hyperplane loads.
+        // This thread's slice of its hyperplane row (loaded before the query
+        // is staged, so both loads are in flight together).
+        const int r = tid / kTpr, part = tid % kTpr;
+        const int wrows = nt * P;
+        const bool live = r < wrows;
+        uint4 w2[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        if (live) {
+            const uint4* wsrc = reinterpret_cast<const uint4*>(W + ((int64_t)l0 * P + r) * kHeadDim + kChan * part);
+            w2[0] = __ldg(wsrc);
+            w2[1] = __ldg(wsrc + 1);
+        }
+        // The unit's G query rows in 16-byte pieces (8 bf16 or 4 fp32 each).
         constexpr int kPer16 = 16 / (int)sizeof(QT);
         const int npieces = G * kHeadDim / kPer16;  // <= 512 for G <= 16
         const uint4* qu4 = reinterpret_cast<const uint4*>(q + u * G * kHeadDim);
         constexpr int kQv = (kMaxGroup * kHeadDim / kPer16 + kThreads - 1) / kThreads;
-        uint4 qv[kQv];
-#pragma unroll
-        for (int i = 0; i < kQv; ++i)
-            if (tid + i * kThreads < npieces) qv[i] = __ldg(qu4 + tid + i * kThreads);
-        // This CTA's hyperplane rows (nt tables x P planes, contiguous in W).
-        const int wrows = nt * P;
-        const uint4* wsrc = reinterpret_cast<const uint4*>(W + (int64_t)l0 * P * kHeadDim);
-        for (int e = tid; e < wrows * (kHeadDim / 8); e += kThreads)
-            *reinterpret_cast<uint4*>(wsm + (e >> 4) * kWRow + (e & 15) * 8) = __ldg(wsrc + e);
 #pragma unroll
         for (int i = 0; i < kQv; ++i) {
             const int piece = tid + i * kThreads;
             if (piece < npieces) {
-                double* dst = qd + piece * kPer16;  // qd rows are contiguous
-                const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+                const uint4 v = __ldg(qu4 + piece);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                const int h = piece * kPer16 / kHeadDim, c0 = piece * kPer16 % kHeadDim;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if constexpr (sizeof(QT) == 2) {
-                        const float2 f = bf16x2_to_f32x2(w4[e]);
-                        dst[2 * e] = (double)f.x;
-                        dst[2 * e + 1] = (double)f.y;
+                        QD(h, c0 + 2 * e) = bf16_bits_to_f64(w4[e] & 0xffffu);
+                        QD(h, c0 + 2 * e + 1) = bf16_bits_to_f64(w4[e] >> 16);
                     } else {
-                        dst[e] = (double)__uint_as_float(w4[e]);
+                        QD(h, c0 + e) = (double)__uint_as_float(w4[e]);
                     }
                 }
             }
@@ -132,60 +134,53 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         // Per head, the factor taking <W_{l,p}, q_h> to the sigmoid argument
         // 2 z / tau with z = <W_{l,p}, q_h> / ||q_h|| (0 for a zero query).
         for (int h = warp; h < G; h += kThreads / 32) {
-            const double* qh = qd + h * kHeadDim + 4 * lane;
-            double s = qh[0] * qh[0] + qh[1] * qh[1] + qh[2] * qh[2] + qh[3] * qh[3];
+            double s = 0.0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const double x = QD(h, 4 * lane + j);
+                s = fma(x, x, s);
+            }
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
             if (lane == 0) qscale[h] = (s > 0.0 && tau > 0.0) ? 2.0 / (tau * sqrt(s)) : 0.0;
         }
-        __syncthreads();
-
-        // Thread (row r, quarter qq) takes channels 8 (4 s + qq) .. + 7, s < 4.
-        const int r = tid >> 2, qq = tid & 3;
-        const bool live = r < wrows;
-        const int lt = live ? r / P : 0, p = live ? r - lt * P : 0;
-        double wd[32];  // this thread's 32 channels of the row, widened once
+        double wd[kChan];  // this thread's 16 channels of the row, widened once
         {
-            const uint16_t* wr = wsm + (live ? r : 0) * kWRow + 8 * qq;
+            const uint32_t words[8] = {w2[0].x, w2[0].y, w2[0].z, w2[0].w, w2[1].x, w2[1].y, w2[1].z, w2[1].w};
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint4 w8 = *reinterpret_cast<const uint4*>(wr + 32 * s);
-                const uint32_t words[4] = {w8.x, w8.y, w8.z, w8.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    wd[8 * s + 2 * i] = bf16_bits_to_f64(words[i] & 0xffffu);
-                    wd[8 * s + 2 * i + 1] = bf16_bits_to_f64(words[i] >> 16);
-                }
+            for (int i = 0; i < 8; ++i) {
+                wd[2 * i] = bf16_bits_to_f64(words[i] & 0xffffu);
+                wd[2 * i + 1] = bf16_bits_to_f64(words[i] >> 16);
             }
         }
+        __syncthreads();
+
+        const int lt = live ? r / P : 0, p = live ? r - lt * P : 0;
         for (int h0 = 0; h0 < G; h0 += kHeadsPerPass) {
             double acc[kHeadsPerPass];
 #pragma unroll
             for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                 double a0 = 0.0, a1 = 0.0;
                 if (h0 + hh < G) {
-                    const double* qh = qd + (h0 + hh) * kHeadDim + 8 * qq;
+                    const double* qh = &QD(h0 + hh, kChan * part);
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-#pragma unroll
-                        for (int i = 0; i < 8; i += 2) {
-                            const double2 qv2 = *reinterpret_cast<const double2*>(qh + 32 * s + i);
-                            a0 = fma(wd[8 * s + i], qv2.x, a0);
-                            a1 = fma(wd[8 * s + i + 1], qv2.y, a1);
-                        }
+                    for (int i = 0; i < kChan; i += 2) {
+                        const double2 qv2 = *reinterpret_cast<const double2*>(qh + i);
+                        a0 = fma(wd[i], qv2.x, a0);
+                        a1 = fma(wd[i + 1], qv2.y, a1);
                     }
                 }
                 acc[hh] = a0 + a1;
             }
-            // Sum the four quarters; every thread of the row then holds the
-            // four heads' projections, and quarter hh finishes head h0 + hh.
+            // Sum the row's eight slices; thread hh of the row finishes head h0 + hh.
 #pragma unroll
             for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                 acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 1);
                 acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 2);
+                acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 4);
             }
-            const double y = qq == 0 ? acc[0] : qq == 1 ? acc[1] : qq == 2 ? acc[2] : acc[3];
-            const int h = h0 + qq;
-            if (live && h < G) {
+            const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
+            const int h = h0 + part;
+            if (live && part < kHeadsPerPass && h < G) {
                 if (tau == 0.0) {
                     // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
                     SIG(h, lt, p, 1) = y > 0.0 ? 1.0 : 0.0;
@@ -206,7 +201,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         // Nibble tables: lo over planes 0..min(P,4)-1, hi over planes 4..P-1.
         const int plo = min(P, 4);
         for (int e = tid; e < G * kTpb * 32; e += kThreads) {
-            const int h = e >> 8, t = (e >> 5) & (kTpb - 1), hi = (e >> 4) & 1, v = e & 15;
+            const int h = e >> 7, t = (e >> 5) & (kTpb - 1), hi = (e >> 4) & 1, v = e & 15;
             if (t >= nt) continue;
             double prod = 1.0;
             const int p0 = hi ? 4 : 0, p1 = hi ? P : plo;
@@ -228,7 +223,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     }
     const int nblk = (L + 31) / 32;
     float* tu = tables + u * nblk * (int64_t)NB * 64;
-    // Entry `bucket` of the CTA's eight tables: eight adjacent columns (and
+    // Entry `bucket` of the CTA's four tables: four adjacent columns (and
     // their copies 32 columns on) of one row, as vector stores.
     for (int bucket = tid; bucket < NB; bucket += kThreads) {
         float vals[kTpb];
@@ -245,11 +240,8 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         }
         float* row = tu + ((int64_t)(l0 >> 5) * NB + bucket) * 64 + (l0 & 31);
         const float4 a = make_float4(vals[0], vals[1], vals[2], vals[3]);
-        const float4 b = make_float4(vals[4], vals[5], vals[6], vals[7]);
         *reinterpret_cast<float4*>(row) = a;
-        *reinterpret_cast<float4*>(row + 4) = b;
         *reinterpret_cast<float4*>(row + 32) = a;
-        *reinterpret_cast<float4*>(row + 36) = b;
     }
 
     // Keys appended in this step (the step 1 hash of those keys, "Pre-cálculo"):
@@ -268,7 +260,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         const int wrows = nt * P;
         for (int key = 0; key < nk && wrows > 0; ++key) {
             // The key row once per warp (four channels per lane); the CTA's
-            // hyperplane rows from shared memory.
+            // hyperplane rows from W (four channels per lane).
             const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
             float4 kf;
             if (app.kv_dtype == 1) {
@@ -279,7 +271,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
                 kf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.K) + off);
             }
             for (int wr = warp; wr < wrows; wr += kThreads / 32) {
-                const uint2 wq = *reinterpret_cast<const uint2*>(wsm + wr * kWRow + 4 * lane);
+                const uint2 wq = __ldg(reinterpret_cast<const uint2*>(W + ((int64_t)l0 * P + wr) * kHeadDim + 4 * lane));
                 const float2 w01 = bf16x2_to_f32x2(wq.x), w23 = bf16x2_to_f32x2(wq.y);
                 float y = fmaf(w23.y, kf.w, fmaf(w23.x, kf.z, fmaf(w01.y, kf.y, w01.x * kf.x)));
                 for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(kFullMask, y, o);
@@ -323,7 +315,7 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                cudaStream_t stream)
 {
     const int smem = smem_bytes(s.G);
-    const dim3 grid((unsigned)s.U, (unsigned)(4 * ((s.L + 31) / 32)));
+    const dim3 grid((unsigned)s.U, (unsigned)(32 / kTpb * ((s.L + 31) / 32)));
     if (q_dtype == 1) {
         cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<uint16_t>, smem_bytes(kMaxGroup));
         if (e != cudaSuccess) return e;
