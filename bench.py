@@ -90,7 +90,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.0005):
         self.period = period_s
         self.samples = []
         self.reasons = 0
@@ -215,16 +215,37 @@ def oracle_decode_timing(w, K, V, q, W, units_kvh, min_seconds=2.0, reps_max=50)
     return el / reps, S, threads, hash_s
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(w, inp):
+    """The oracle's decode on a bounded sample of the workload's units, with
+    OpenMP over those units, and on one unit with one thread."""
+    import oracle
     units = list(range(min(w.Hkv, 8)))
     K = inp["K"][0].cpu()
     V = inp["V"][0].cpu()
-    t, S, threads, hash_s = oracle_decode_timing(w, K, V, inp["q"][0].cpu(), inp["W"].cpu(), units)
+    q, W = inp["q"][0].cpu(), inp["W"].cpu()
+    t, S, threads, hash_s = oracle_decode_timing(w, K, V, q, W, units)
+    t1, S1, _, _ = oracle_decode_timing(w, K, V, q, W, units[:1], min_seconds=1.0)
+    oracle.set_num_threads(oracle.max_threads())
     value = 1.0 / (t * w.U / S)
     return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "single_thread": {"value": 1.0 / (t1 * w.U / S1), "unit": UNIT, "cores": 1,
+                              "sample": f"1 unit at full N={w.N}, {t1 * 1e3:.1f} ms; steps/s scaled by {w.U}"},
             "hash_keys_per_s": S * w.N / hash_s,
             "sample": f"{S} of {w.U} (batch, kv-head) units at full N={w.N}, oracle decode (soft tables, scores, "
-                      f"top-k, attention) in fp64, {t * 1e3:.1f} ms per sample; steps/s scaled by {w.U}/{S}"}
+                      f"top-k, attention) in fp64 with {threads} threads (one per unit), {t * 1e3:.1f} ms per "
+                      f"sample; steps/s scaled by {w.U}/{S}"}
 
 
 def run_reference(args, world: int, rank: int):
@@ -273,6 +294,59 @@ def run_reference(args, world: int, rank: int):
 # ----------------------------------------------------------------------------
 # the CUDA path
 # ----------------------------------------------------------------------------
+
+def time_workload(name: str, dev, steps: int = 100, flush_l2: bool = False):
+    """Decode steps of another workload on this GPU (one layer).  Workloads
+    larger than L2 replay a CUDA graph back to back; the small ones (whose
+    data would stay in L2 between steps) are timed one step at a time with a
+    write of 2 x L2 bytes before each, so every step starts cold."""
+    import soft_lsh_top_b200 as sk
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w, dev)
+    ids, vn = sk.alloc_cache_index(w.B, w.Hkv, w.ncap, w.L, dev)
+    sk.socket_hash_keys(inp["K"], inp["V"], inp["W"], ids, vn, 0, w.N)
+    ws, idx, out = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, dev)
+    step = lambda: sk.socket_decode(inp["q"], inp["W"], ids, vn, inp["K"], inp["V"], w.N, w.tau, w.k, ws, idx, out)
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    peak, _ = hbm_peak()
+    if flush_l2:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        junk = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in evs:
+            junk.fill_(1)
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+        how = "one step at a time, L2 overwritten before each step; median of CUDA-event times around the step"
+        del junk
+    else:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        us = a.elapsed_time(b) / steps * 1e3
+        how = "CUDA graph of one step replayed back to back (inputs larger than L2)"
+        del g
+    assert sk.read_device_error(ws) == 0
+    res = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "L": w.L, "P": w.P, "tau": w.tau, "k": w.k,
+           "kv_dtype": w.dtype, "us_per_step": us, "steps_per_s": 1e6 / us, "bytes_per_step": w.step_bytes(),
+           "step_roofline_frac": w.step_bytes() / (us * 1e-6) / 1e9 / peak, "how": how}
+    del inp, ids, vn, ws, idx, out
+    torch.cuda.empty_cache()
+    return res
+
 
 def run_socket(args, world: int, rank: int, local_rank: int):
     import soft_lsh_top_b200 as sk
@@ -611,11 +685,13 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         result = {
             "metric": METRIC, "value": whole_job_rate(world, K, ms_total), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "data": "synthetic",
+            "dtype": ("bf16 K/V and q, f32 scores, softmax and outputs" if w.dtype == "bf16" else "f32"),
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "L": w.L,
-                       "P": w.P, "tau": w.tau, "k": w.k, "kv_dtype": w.dtype, "parallelism": f"replicas{world}",
-                       "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB per step, {R} rotating layers "
-                             "of independent data", "launch": launch},
+                       "P": w.P, "tau": w.tau, "k": w.k, "kv_dtype": w.dtype},
+            "run": {"parallelism": f"replicas{world}",
+                    "l2": f"inputs larger than L2: {bytes_step / 1e6:.0f} MB per step, {R} rotating layers "
+                          "of independent data", "launch": launch},
             "bytes_per_step": bytes_step,
             "step_hbm_gbs": bytes_step / (ms_step * 1e-3) / 1e9,
             "step_roofline_frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak,
@@ -623,6 +699,10 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "roofline": {"bound": "hbm", "kernel": "score_kernel", "achieved": score_gbs, "peak": peak,
                          "unit": "GB/s", "frac": score_gbs / peak, "traffic": traffic,
                          "algorithmic_bytes_per_launch": score_bytes, "peak_source": peak_src,
+                         "step": {"what": "the whole decode step (4 kernels): ids + norms + 2 k d 2 bytes per kv "
+                                          "head, over ms_per_step", "achieved": bytes_step / (ms_step * 1e-3) / 1e9,
+                                  "frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak, "bytes": bytes_step,
+                                  "target_frac": 0.70},
                          "attention_gbs": attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9},
             "gpu_launches": nk * K,
             "clocks": clocks.summary(),
@@ -635,6 +715,13 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                            "output + indices copied back every step, on a copy stream double-buffered against "
                            "the kernels"},
         }
+        if not args.no_workloads:
+            # The other workloads of the method's long-context range, same GPU.
+            result["workloads"] = {
+                wl.MILLION.name: time_workload(wl.MILLION.name, dev, steps=100),
+                wl.LLAMA_32K.name: time_workload(wl.LLAMA_32K.name, dev, steps=100, flush_l2=True),
+                wl.TINY.name: time_workload(wl.TINY.name, dev, steps=100, flush_l2=True),
+            }
         if world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, layers[0][0])
         print(json.dumps(result), flush=True)
@@ -654,6 +741,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=wl.BATCH8_128K.name, choices=sorted(wl.WORKLOADS))
     ap.add_argument("--layers", type=int, default=3, help="independently drawn layers rotated across steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other workloads' step times")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling captures)")
     ap.add_argument("--no-graph", action="store_true", help="time direct calls instead of CUDA graph replay")
     args = ap.parse_args(argv)

@@ -307,8 +307,9 @@ def test_batch8_128k_sampled_units_and_needles():
 
 def test_batch8_128k_per_head_sampled_units_and_needles():
     """One selection per query head at full size: sampled kv units checked
-    head by head against the oracle, and each head's own needles found by its
-    own selection (no competition from the group's other heads)."""
+    head by head against the oracle, and every head finds all 16 of its own
+    needles (cosine 0.9 to its query; no competition from the group's other
+    heads, unlike the grouped selection)."""
     w = wl.BATCH8_128K
     units = [5, 40]
     inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
@@ -316,8 +317,7 @@ def test_batch8_128k_per_head_sampled_units_and_needles():
     needles, m = inp["needles"], w.needles_per_head
     found = sum(int(torch.isin(needles[b, kvh, g * m:(g + 1) * m].to(torch.int32), idx[b, kvh * w.G + g]).sum())
                 for b in range(w.B) for kvh in range(w.Hkv) for g in range(w.G))
-    recall = found / needles.numel()
-    assert recall >= 0.99, recall
+    assert found == needles.numel(), found / needles.numel()
     substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
     idx, out, sc = gpu_decode(inp, w, ids, vnorm, per_head=True)
     check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, per_head=True)
