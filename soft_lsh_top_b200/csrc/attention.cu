@@ -373,11 +373,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 __device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(pack_bf16(x, 0.0f) << 16); }
 
 // The unit's last CTA merges the splits' partials: head h is merged by warp
-// h % kWWarps with no CTA barrier.  For each head, M = max_s m_s, the weights
-// w_s = exp(m_s - M) live in the lanes (split s in lane s % 32, a tile of 32
-// splits at a time) and reach the others by shuffle, and each lane
-// accumulates four output columns from 16-byte loads of every split's row,
-// in split order: out = sum_s w_s o_s / sum_s w_s l_s.
+// h % kWWarps with no CTA barrier.  Splits are taken 16 at a time, their
+// (m, l) pairs (split s in lane s) and 16-byte loads of their rows issued
+// together; the weights w_s = exp(m_s - M) reach the other lanes by shuffle,
+// and each lane accumulates four output columns in split order, rescaling
+// when a later tile raises the running max M:
+// out = sum_s w_s o_s / sum_s w_s l_s with M = max_s m_s.
 template <int G>
 __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
                                                  const float* __restrict__ part_o, const float2* __restrict__ part_ml,
@@ -391,45 +392,42 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    constexpr int kTile = 16;  // splits whose rows are loaded at once
     for (int h = warp; h < G; h += kWWarps) {
         const int64_t base = pbase + h * nsplit;
-        float M = -INFINITY;
-        for (int s0 = 0; s0 < nsplit; s0 += 32)
-            if (s0 + lane < nsplit) M = fmaxf(M, __ldcg(&part_ml[base + s0 + lane]).x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, o));
+        float M = -INFINITY, lsum = 0.0f;  // lsum: this lane's splits, at the running max M
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        float lsum = 0.0f;
-        for (int s0 = 0; s0 < nsplit; s0 += 32) {
-            const int cnt = min(32, nsplit - s0);
-            float w = 0.0f;
-            if (lane < cnt) {
-                const float2 t = __ldcg(&part_ml[base + s0 + lane]);
-                w = t.x == -INFINITY ? 0.0f : expf(t.x - M);
-                lsum += t.y * w;
-            }
+        for (int s0 = 0; s0 < nsplit; s0 += kTile) {
+            // The tile's (m, l) pairs (split s0 + i in lane i) and rows, all in flight at once.
+            const int cnt = min(kTile, nsplit - s0);
+            const float2 t = lane < cnt ? __ldcg(&part_ml[base + s0 + lane]) : make_float2(-INFINITY, 0.0f);
             const float4* po = reinterpret_cast<const float4*>(part_o + (base + s0) * kHeadDim) + lane;
-            int i = 0;
-            for (; i + 8 <= cnt; i += 8) {
-                float4 v[8];
+            float4 v[kTile];
 #pragma unroll
-                for (int r = 0; r < 8; ++r) v[r] = __ldcg(po + (int64_t)(i + r) * (kHeadDim / 4));
+            for (int r = 0; r < kTile; ++r)
+                v[r] = r < cnt ? __ldcg(po + (int64_t)r * (kHeadDim / 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float mt = t.x;
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const float wr = __shfl_sync(kFullMask, w, i + r);
+            for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(kFullMask, mt, o));
+            const float Mn = fmaxf(M, mt);
+            if (Mn != -INFINITY) {
+                const float sc = M == -INFINITY ? 0.0f : expf(M - Mn);  // rescale the earlier tiles
+                acc.x *= sc;
+                acc.y *= sc;
+                acc.z *= sc;
+                acc.w *= sc;
+                lsum *= sc;
+                const float w = t.x == -INFINITY ? 0.0f : expf(t.x - Mn);
+                lsum += t.y * w;
+#pragma unroll
+                for (int r = 0; r < kTile; ++r) {
+                    const float wr = __shfl_sync(kFullMask, w, r);
                     acc.x += wr * v[r].x;
                     acc.y += wr * v[r].y;
                     acc.z += wr * v[r].z;
                     acc.w += wr * v[r].w;
                 }
-            }
-            for (; i < cnt; ++i) {
-                const float4 v = __ldcg(po + (int64_t)i * (kHeadDim / 4));
-                const float wr = __shfl_sync(kFullMask, w, i);
-                acc.x += wr * v.x;
-                acc.y += wr * v.y;
-                acc.z += wr * v.z;
-                acc.w += wr * v.w;
+                M = Mn;
             }
         }
 #pragma unroll

@@ -40,6 +40,7 @@ using namespace select512;
 constexpr int kSliceKeys = 32768;                      // keys per CTA
 constexpr int kLoadsPerThread = kSliceKeys / (4 * kThreads);  // 16-byte score loads per thread
 constexpr int kInFlight = 6;                           // of them in flight at a time
+constexpr int kRankMax = 96;                           // candidates ranked by counting (nc^2 comparisons)
 constexpr int kWordsPerThread = 8;                     // bitmap words per thread and tile of the compaction
 constexpr int kTileWords = kThreads * kWordsPerThread;  // bitmap words per tile (131072 keys)
 
@@ -67,6 +68,7 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t u = blockIdx.x / a.C;
     const int r = blockIdx.x % a.C;
+    const bool single = a.C == 1;  // one CTA holds the whole unit: bitmap and candidates stay in shared memory
     const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + u * a.Ncap);
     uint32_t* bm = a.bitmap + u * a.bm_stride;  // 16-byte aligned rows
     const int lo = r * kSliceKeys, hi = min(a.N, lo + kSliceKeys);
@@ -119,6 +121,7 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     // shared memory (one shared atomic per warp and load that has any).
 #pragma unroll
     for (int g = 0; g < kLoadsPerThread; ++g) {
+        if (lo + g * 4 * kThreads + 128 * (tid >> 5) >= hi) continue;  // the warp's keys all lie past the slice
         const uint4 x = v[g % kInFlight];
         if (g + kInFlight < kLoadsPerThread) v[g % kInFlight] = load(g + kInFlight);
         const int n0 = key_of(g);
@@ -135,7 +138,10 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         word |= __shfl_xor_sync(kFullMask, word, 1);
         word |= __shfl_xor_sync(kFullMask, word, 2);
         word |= __shfl_xor_sync(kFullMask, word, 4);
-        if ((lane & 7) == 0 && n0 < hi) bm[n0 >> 5] = word;
+        if ((lane & 7) == 0 && n0 < hi) {
+            if (single) sbits[n0 >> 5] = word;
+            else bm[n0 >> 5] = word;
+        }
         const uint32_t cnt = fits ? __popc(cmask) : 0u;
         if (__any_sync(kFullMask, cnt != 0)) {
             uint32_t incl = cnt;
@@ -158,8 +164,8 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         }
     }
     __syncthreads();
-    // The CTA's candidates -> the unit list (one global atomic per CTA).
-    {
+    if (!single) {
+        // The CTA's candidates -> the unit list (one global atomic per CTA).
         const uint32_t nl = min(sh.count, (uint32_t)a.cap);
         if (tid == 0 && nl) sh.base = atomicAdd(a.cand_cnt + u, nl);
         __syncthreads();
@@ -167,15 +173,14 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         uint2* cu = a.cand + u * a.cap;
         for (uint32_t i = tid; i < nl; i += kThreads)
             if (base + i < (uint32_t)a.cap) cu[base + i] = scand[i];
+        // ---- the unit's last CTA to get here selects.
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) sh.last = atomicAdd(a.done + u, 1u) == (uint32_t)(a.C - 1);
+        __syncthreads();
+        if (!sh.last) return;
+        __threadfence();
     }
-
-    // ---- the unit's last CTA to get here selects.
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sh.last = atomicAdd(a.done + u, 1u) == (uint32_t)(a.C - 1);
-    __syncthreads();
-    if (!sh.last) return;
-    __threadfence();
 
     int32_t* out = a.idx_out + u * (int64_t)a.k;
     if (!fits) {
@@ -206,35 +211,76 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
             tw[q] = x;
         }
     };
-    load_tile(0);
-
-    // ---- the unit's candidates in shared memory; the krem0-th largest among
-    // them: digits 18-8 and 7-0.
     const int nc = (int)ncand;
-    {
+    if (!single) {
+        load_tile(0);
+        // ---- the unit's candidates in shared memory.
         const uint2* cu = a.cand + u * a.cap;
         for (int i = tid; i < nc; i += kThreads) scand[i] = __ldcg(cu + i);
         __syncthreads();
     }
-    uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
-    auto bits_of = [&](int i) { return scand[i].y; };
-    radix_digit(sh, nc, bits_of, 8, 0x7ffu, true, prefix, mask, need);
-    radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
-    const uint32_t t = prefix, ties_total = sh.count;  // keys equal to t
-    // Ties at t beyond `need`: keep the `need` lowest indices, i.e. those at
-    // or below the need-th smallest tie index ti (digits 30-20, 19-9, 8-0 of
-    // the ties' indices, ascending; non-ties map to 2^32 - 1 and never match).
-    uint32_t ti = 0xffffffffu;
-    if (ties_total > need) {
-        auto idx_of_tie = [&](int i) {
+    // ---- among the nc candidates (every key of bin d0), keep the krem0 with
+    // the largest scores, ties to the lower index; the decision replaces each
+    // candidate's bit pattern (1 keep, 0 drop).  A few hundred: rank each by
+    // counting those ahead of it (T lanes per candidate, a power of two);
+    // more: two radix digits for the krem0-th pattern t, then the ties at t by
+    // a radix select over their indices.
+    if (nc <= kRankMax) {
+        int T = 1;
+        while (T < 32 && T * 2 * nc <= kThreads) T *= 2;
+        const int sub = lane & (T - 1);
+        uint32_t keep[(kRankMax + kThreads - 1) / kThreads] = {};
+        for (int i0 = 0, it = 0; i0 < nc * T; i0 += kThreads, ++it) {
+            const int i = (i0 + tid) / T;
+            uint32_t ahead = 0;
+            if (i < nc) {
+                const uint2 me = scand[i];
+                int j = sub;
+                for (; j + 3 * T < nc; j += 4 * T) {
+                    const uint2 o0 = scand[j], o1 = scand[j + T], o2 = scand[j + 2 * T], o3 = scand[j + 3 * T];
+                    ahead += (o0.y > me.y || (o0.y == me.y && o0.x < me.x)) +
+                             (o1.y > me.y || (o1.y == me.y && o1.x < me.x)) +
+                             (o2.y > me.y || (o2.y == me.y && o2.x < me.x)) +
+                             (o3.y > me.y || (o3.y == me.y && o3.x < me.x));
+                }
+                for (; j < nc; j += T) {
+                    const uint2 o = scand[j];
+                    ahead += o.y > me.y || (o.y == me.y && o.x < me.x);
+                }
+            }
+            for (int o = 1; o < T; o <<= 1) ahead += __shfl_xor_sync(kFullMask, ahead, o);
+            keep[it] = ahead < krem0;
+        }
+        __syncthreads();  // every rank counted before the patterns are overwritten
+        for (int i0 = 0, it = 0; i0 < nc * T; i0 += kThreads, ++it) {
+            const int i = (i0 + tid) / T;
+            if (i < nc && sub == 0) scand[i].y = keep[it];
+        }
+    } else {
+        uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
+        auto bits_of = [&](int i) { return scand[i].y; };
+        radix_digit(sh, nc, bits_of, 8, 0x7ffu, true, prefix, mask, need);
+        radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
+        const uint32_t t = prefix, ties_total = sh.count;  // keys equal to t
+        // Ties at t beyond `need`: keep the `need` lowest indices, i.e. those at
+        // or below the need-th smallest tie index ti (digits 30-20, 19-9, 8-0 of
+        // the ties' indices, ascending; non-ties map to 2^32 - 1 and never match).
+        uint32_t ti = 0xffffffffu;
+        if (ties_total > need) {
+            auto idx_of_tie = [&](int i) {
+                const uint2 e = scand[i];
+                return e.y == t ? e.x : 0xffffffffu;
+            };
+            uint32_t ip = 0, im = 0x80000000u, ik = need;
+            radix_digit(sh, nc, idx_of_tie, 20, 0x7ffu, false, ip, im, ik);
+            radix_digit(sh, nc, idx_of_tie, 9, 0x7ffu, false, ip, im, ik);
+            radix_digit(sh, nc, idx_of_tie, 0, 0x1ffu, false, ip, im, ik);
+            ti = ip;
+        }
+        for (int i = tid; i < nc; i += kThreads) {
             const uint2 e = scand[i];
-            return e.y == t ? e.x : 0xffffffffu;
-        };
-        uint32_t ip = 0, im = 0x80000000u, ik = need;
-        radix_digit(sh, nc, idx_of_tie, 20, 0x7ffu, false, ip, im, ik);
-        radix_digit(sh, nc, idx_of_tie, 9, 0x7ffu, false, ip, im, ik);
-        radix_digit(sh, nc, idx_of_tie, 0, 0x1ffu, false, ip, im, ik);
-        ti = ip;
+            scand[i].y = e.y > t || (e.y == t && e.x <= ti);
+        }
     }
 
     // ---- selected keys in index order, tile by tile of the bitmap: the
@@ -243,21 +289,23 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     // from one block-wide scan of their population counts.
     uint32_t out_base = 0;
     for (int w0 = 0; w0 < words; w0 += kTileWords) {
+        if (!single) {  // a single CTA's words (one tile at most) are in shared memory already
+            __syncthreads();  // the previous tile's words have been read
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread / 4; ++q)
-            *reinterpret_cast<uint4*>(sbits + tid * kWordsPerThread + 4 * q) = tw[q];
+            for (int q = 0; q < kWordsPerThread / 4; ++q)
+                *reinterpret_cast<uint4*>(sbits + tid * kWordsPerThread + 4 * q) = tw[q];
+        }
         __syncthreads();
-        if (w0 + kTileWords < words) load_tile(w0 + kTileWords);
+        if (!single && w0 + kTileWords < words) load_tile(w0 + kTileWords);
         const uint32_t klo = 32u * (uint32_t)w0, khi = klo + 32u * kTileWords;
         for (int i = tid; i < nc; i += kThreads) {
             const uint2 e = scand[i];
-            const bool keep = e.y > t || (e.y == t && e.x <= ti);
-            if (!keep && e.x >= klo && e.x < khi) atomicAnd(sbits + ((e.x - klo) >> 5), ~(1u << (e.x & 31)));
+            if (!e.y && e.x >= klo && e.x < khi) atomicAnd(sbits + ((e.x - klo) >> 5), ~(1u << (e.x & 31)));
         }
         __syncthreads();
         uint32_t wv[kWordsPerThread];
 #pragma unroll
-        for (int q = 0; q < kWordsPerThread; ++q) wv[q] = sbits[tid * kWordsPerThread + q];
+        for (int q = 0; q < kWordsPerThread; ++q) wv[q] = w0 + tid * kWordsPerThread + q < words ? sbits[tid * kWordsPerThread + q] : 0u;
         uint32_t cnt = 0;
 #pragma unroll
         for (int q = 0; q < kWordsPerThread; ++q) cnt += __popc(wv[q]);
