@@ -181,9 +181,10 @@ int socket_decode(const void* q, int q_dtype, const uint16_t* W,
  *   Arguments as for socket_decode, except that ids and vnorm are also
  *   written (the rows of the n_new keys) and:
  *   n_new      1 <= n_new <= min(64, N).
- * The projections are summed in float32 in another order than the hash
- * kernels', so an id can differ from socket_hash_keys' only where some
- * |<W_{l,p}, k>| is within float32 accumulation error of 0.  The workspace is
+ * The appended keys' projections are formed in float64 (by the kernel that
+ * projects the queries), so an id can differ from socket_hash_keys' (float32
+ * accumulation) only where some |<W_{l,p}, k>| is within float32
+ * accumulation error of 0.  The workspace is
  * socket_decode_workspace_size()'s.
  */
 int socket_decode_append(const void* q, int q_dtype, const uint16_t* W,

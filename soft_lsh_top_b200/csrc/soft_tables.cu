@@ -37,10 +37,24 @@ __device__ __forceinline__ double bf16_bits_to_f64(uint32_t b)
     return __hiloint2double((int)(((b & 0x8000u) << 16) | ((mag << 13) + (896u << 20))), 0);
 }
 
-// Dynamic shared memory of a CTA for group size G.
-__host__ __device__ constexpr int smem_bytes(int G)
+// Four channels of a value row (element offset `off`) as float32.
+__device__ __forceinline__ float4 load_v4(const AppendHash& app, int64_t off)
 {
-    return G * kTpr * kQSeg * 8                   // query rows (fp64), one padded segment per channel slice
+    if (app.kv_dtype == 1) {
+        const uint2 vq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.V) + off);
+        const float2 v01 = bf16x2_to_f32x2(vq.x), v23 = bf16x2_to_f32x2(vq.y);
+        return make_float4(v01.x, v01.y, v23.x, v23.y);
+    }
+    return *reinterpret_cast<const float4*>(static_cast<const float*>(app.V) + off);
+}
+
+constexpr int kKeySlots = 16;              // appended keys projected per pass group (extra rows of qd)
+
+// Dynamic shared memory of a CTA for group size G, with `slots` rows for
+// appended keys.
+__host__ __device__ constexpr int smem_bytes(int G, int slots)
+{
+    return (G + slots) * kTpr * kQSeg * 8         // query rows, then key rows (fp64), padded channel slices
            + G * 8                                // per-head factor 2 / (tau ||q_h||)
            + G * kTpb * kMaxP * 2 * 8             // per-plane sigmoid pairs
            + G * kTpb * 2 * 16 * 8;               // nibble tables
@@ -65,7 +79,7 @@ __host__ __device__ constexpr int smem_bytes(int G)
 //      memory: per 32-table block c a [bucket][64] row whose column j holds
 //      table 32c + j mod 32.
 template <typename QT>
-__global__ __launch_bounds__(kThreads) void soft_tables_kernel(
+__global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L, int P, double tau,
     const AppendHash app, int64_t Ncap, int share, float* __restrict__ tables, uint32_t* __restrict__ err_word,
     uint32_t* __restrict__ counters, uint32_t* __restrict__ topk_done, uint32_t* __restrict__ unit_hist,
@@ -73,13 +87,39 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
 {
     __shared__ uint32_t aid[kMaxAppend][kTpb];  // ids of the appended keys (bit p <-> plane p)
     extern __shared__ __align__(16) char st_dyn[];
-    double* qd = reinterpret_cast<double*>(st_dyn);  // [G][kTpr][kQSeg]
-    double* qscale = qd + G * kTpr * kQSeg;          // [G]
+    // Keys appended in this step are hashed here too (step 1 of the method,
+    // "Pre-cálculo"), by the first unit of each kv unit: their rows take
+    // kKeySlots extra rows of qd and the same dot products as the queries.
+    const bool appending = app.end > app.begin && blockIdx.x % share == 0;
+    const int slots = appending ? kKeySlots : 0;
+    double* qd = reinterpret_cast<double*>(st_dyn);  // [G + slots][kTpr][kQSeg]
+    double* qscale = qd + (G + slots) * kTpr * kQSeg;  // [G]
     double* sig = qscale + G;                        // [G][kTpb][kMaxP][2]
     double* nib = sig + G * kTpb * kMaxP * 2;        // [G][kTpb][2][16]
     auto QD = [&](int h, int c) -> double& { return qd[(h * kTpr + (c >> 4)) * kQSeg + (c & 15)]; };
     auto SIG = [&](int h, int lt, int p, int s) -> double& { return sig[((h * kTpb + lt) * kMaxP + p) * 2 + s]; };
     auto NIB = [&](int h, int lt, int hi, int v) -> double& { return nib[((h * kTpb + lt) * 2 + hi) * 16 + v]; };
+    // Appended keys k0 .. k0 + nk - 1 of the kv unit into rows G .. G + nk - 1
+    // of qd, widened to float64, from 16-byte pieces (8 bf16 or 4 float32).
+    auto stage_keys = [&](int k0, int nk) {
+        const int per = app.kv_dtype == 1 ? 8 : 4;
+        const char* kbase = static_cast<const char*>(app.K) +
+                            ((int64_t)(blockIdx.x / share) * Ncap + app.begin + k0) * kHeadDim * (int64_t)(16 / per);
+        for (int e = threadIdx.x; e < nk * kHeadDim / per; e += kThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(kbase + 16 * (int64_t)e);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            const int key = e * per / kHeadDim, c0 = e * per % kHeadDim;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (per == 8) {
+                    QD(G + key, c0 + 2 * j) = bf16_bits_to_f64(w4[j] & 0xffffu);
+                    QD(G + key, c0 + 2 * j + 1) = bf16_bits_to_f64(w4[j] >> 16);
+                } else {
+                    QD(G + key, c0 + j) = (double)__uint_as_float(w4[j]);
+                }
+            }
+        }
+    };
 
     const int64_t u = blockIdx.x;  // the unit's query rows are u G .. u G + G - 1 of [B][Hq]
     const int l0 = blockIdx.y * kTpb;
@@ -94,6 +134,16 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
     // kernel's writes).
     pdl_wait();
     pdl_launch_dependents();
+    const int nk_all = appending ? (int)(app.end - app.begin) : 0;
+    const int nk0 = min(kKeySlots, nk_all);  // keys projected in the same passes as the queries
+    const int64_t ukv = u / share;
+    // The first unit CTA's warp j fetches appended key j's value row now, for
+    // its norm at the end (the load's latency overlaps the projections).
+    float4 vpre = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (blockIdx.y == 0 && warp < nk_all) vpre = load_v4(app, (ukv * Ncap + app.begin + warp) * kHeadDim + 4 * lane);
+    if (appending) {
+        for (int e = tid; e < kMaxAppend * kTpb; e += kThreads) aid[e / kTpb][e % kTpb] = 0u;
+    }
 
     if (nt > 0) {
         // This thread's slice of its hyperplane row (loaded before the query
@@ -130,6 +180,7 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
                 }
             }
         }
+        stage_keys(0, nk0);
         __syncthreads();
         // Per head, the factor taking <W_{l,p}, q_h> to the sigmoid argument
         // 2 z / tau with z = <W_{l,p}, q_h> / ||q_h|| (0 for a zero query).
@@ -154,13 +205,16 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         }
         __syncthreads();
 
+        // Rows 0 .. G-1 of qd are the queries, rows G .. G + nk0 - 1 the first
+        // appended keys: bit p of a key's id in table l is [<W_{l,p}, k> > 0].
         const int lt = live ? r / P : 0, p = live ? r - lt * P : 0;
-        for (int h0 = 0; h0 < G; h0 += kHeadsPerPass) {
+        const int Ht = G + nk0;
+        for (int h0 = 0; h0 < Ht; h0 += kHeadsPerPass) {
             double acc[kHeadsPerPass];
 #pragma unroll
             for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                 double a0 = 0.0, a1 = 0.0;
-                if (h0 + hh < G) {
+                if (h0 + hh < Ht) {
                     const double* qh = &QD(h0 + hh, kChan * part);
 #pragma unroll
                     for (int i = 0; i < kChan; i += 2) {
@@ -180,7 +234,9 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
             }
             const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
             const int h = h0 + part;
-            if (live && part < kHeadsPerPass && h < G) {
+            if (live && part < kHeadsPerPass && h >= G && h < Ht) {
+                if (y > 0.0) atomicOr(&aid[h - G][lt], 1u << p);
+            } else if (live && part < kHeadsPerPass && h < G) {
                 if (tau == 0.0) {
                     // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
                     SIG(h, lt, p, 1) = y > 0.0 ? 1.0 : 0.0;
@@ -194,6 +250,39 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
                     SIG(h, lt, p, 1) = x >= 0.0 ? big : small;  // sign +1: bit set
                     SIG(h, lt, p, 0) = x >= 0.0 ? small : big;  // sign -1: bit clear
                 }
+            }
+        }
+        // Any further appended keys, kKeySlots at a time, on the same rows.
+        for (int k0 = kKeySlots; k0 < nk_all; k0 += kKeySlots) {
+            const int nk = min(kKeySlots, nk_all - k0);
+            __syncthreads();  // the previous keys' rows have been read
+            stage_keys(k0, nk);
+            __syncthreads();
+            for (int h0 = 0; h0 < nk; h0 += kHeadsPerPass) {
+                double acc[kHeadsPerPass];
+#pragma unroll
+                for (int hh = 0; hh < kHeadsPerPass; ++hh) {
+                    double a0 = 0.0, a1 = 0.0;
+                    if (h0 + hh < nk) {
+                        const double* kh = &QD(G + h0 + hh, kChan * part);
+#pragma unroll
+                        for (int i = 0; i < kChan; i += 2) {
+                            const double2 kv2 = *reinterpret_cast<const double2*>(kh + i);
+                            a0 = fma(wd[i], kv2.x, a0);
+                            a1 = fma(wd[i + 1], kv2.y, a1);
+                        }
+                    }
+                    acc[hh] = a0 + a1;
+                }
+#pragma unroll
+                for (int hh = 0; hh < kHeadsPerPass; ++hh) {
+                    acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 1);
+                    acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 2);
+                    acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 4);
+                }
+                const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
+                if (live && part < kHeadsPerPass && h0 + part < nk && y > 0.0)
+                    atomicOr(&aid[k0 + h0 + part][lt], 1u << p);
             }
         }
         __syncthreads();
@@ -244,41 +333,15 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         *reinterpret_cast<float4*>(row + 32) = a;
     }
 
-    // Keys appended in this step (the step 1 hash of those keys, "Pre-cálculo"):
-    // the id slots of this CTA's eight tables (0 for tables >= L), and for the
-    // first CTA of the unit the norms.  Projections in float32 (one warp per
-    // (key, hyperplane row), four channels per lane, tree sum); norms in
-    // float64.  The first unit of each kv unit does it; the scoring kernel
-    // reads these rows only after this grid has completed.
-    if (app.end > app.begin && u % share == 0) {
-        const int64_t ukv = u / share;
-        const int nk = (int)(app.end - app.begin);
+    // The appended keys' id slots of this CTA's four tables (0 for tables
+    // >= L), and for the unit's first CTA their norms (float64 sums).  The
+    // scoring kernel reads these rows only after this grid has completed.
+    // (aid is complete: its last writes precede the barrier before the
+    // nibble tables; a CTA with nt == 0 writes zeros without reading it.)
+    if (appending) {
+        const int nk = nk_all;
         const int Lr = 32 * nblk, pieces = Lr / 16;
         uint8_t* idu = app.ids + ukv * Ncap * Lr;
-        for (int e = tid; e < nk * kTpb; e += kThreads) aid[e / kTpb][e % kTpb] = 0u;
-        __syncthreads();
-        const int wrows = nt * P;
-        for (int key = 0; key < nk && wrows > 0; ++key) {
-            // The key row once per warp (four channels per lane); the CTA's
-            // hyperplane rows from W (four channels per lane).
-            const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
-            float4 kf;
-            if (app.kv_dtype == 1) {
-                const uint2 kq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.K) + off);
-                const float2 k01 = bf16x2_to_f32x2(kq.x), k23 = bf16x2_to_f32x2(kq.y);
-                kf = make_float4(k01.x, k01.y, k23.x, k23.y);
-            } else {
-                kf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.K) + off);
-            }
-            for (int wr = warp; wr < wrows; wr += kThreads / 32) {
-                const uint2 wq = __ldg(reinterpret_cast<const uint2*>(W + ((int64_t)l0 * P + wr) * kHeadDim + 4 * lane));
-                const float2 w01 = bf16x2_to_f32x2(wq.x), w23 = bf16x2_to_f32x2(wq.y);
-                float y = fmaf(w23.y, kf.w, fmaf(w23.x, kf.z, fmaf(w01.y, kf.y, w01.x * kf.x)));
-                for (int o = 16; o > 0; o >>= 1) y += __shfl_xor_sync(kFullMask, y, o);
-                if (lane == 0 && y > 0.0f) atomicOr(&aid[key][wr / P], 1u << (wr % P));
-            }
-        }
-        __syncthreads();
         // Byte of table l in key n's rotated row: block l / 32, slot (l - n) mod 32.
         auto id_byte = [&](int64_t n, int l) -> uint8_t* {
             const int b = (l & ~31) + (((l & 31) - (int)(n & 31)) & 31);
@@ -290,15 +353,8 @@ __global__ __launch_bounds__(kThreads) void soft_tables_kernel(
         }
         if (blockIdx.y == 0) {
             for (int key = warp; key < nk; key += kThreads / 32) {
-                const int64_t off = (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane;
-                float4 vf;
-                if (app.kv_dtype == 1) {
-                    const uint2 vq = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(app.V) + off);
-                    const float2 v01 = bf16x2_to_f32x2(vq.x), v23 = bf16x2_to_f32x2(vq.y);
-                    vf = make_float4(v01.x, v01.y, v23.x, v23.y);
-                } else {
-                    vf = *reinterpret_cast<const float4*>(static_cast<const float*>(app.V) + off);
-                }
+                const float4 vf =
+                    key == warp ? vpre : load_v4(app, (ukv * Ncap + app.begin + key) * kHeadDim + 4 * lane);
                 double s = (double)vf.x * vf.x + (double)vf.y * vf.y + (double)vf.z * vf.z + (double)vf.w * vf.w;
                 for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
                 if (lane == 0) app.vnorm[ukv * Ncap + app.begin + key] = (float)sqrt(s);
@@ -314,16 +370,16 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                uint32_t* counters, uint32_t* topk_done, uint32_t* unit_hist, uint32_t* cand_cnt,
                                cudaStream_t stream)
 {
-    const int smem = smem_bytes(s.G);
+    const int smem = smem_bytes(s.G, app.end > app.begin ? kKeySlots : 0);
     const dim3 grid((unsigned)s.U, (unsigned)(32 / kTpb * ((s.L + 31) / 32)));
     if (q_dtype == 1) {
-        cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<uint16_t>, smem_bytes(kMaxGroup));
+        cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<uint16_t>, smem_bytes(kMaxGroup, kKeySlots));
         if (e != cudaSuccess) return e;
         return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), (size_t)smem, stream,
                           static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables,
                           err_word, counters, topk_done, unit_hist, cand_cnt);
     }
-    cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<float>, smem_bytes(kMaxGroup));
+    cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<float>, smem_bytes(kMaxGroup, kKeySlots));
     if (e != cudaSuccess) return e;
     return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), (size_t)smem, stream,
                       static_cast<const float*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables, err_word,
