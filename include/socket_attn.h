@@ -65,6 +65,7 @@ extern "C" {
 #define SOCKET_WS_ERROR_OFFSET 0
 #define SOCKET_DEVERR_GATHER_TIMEOUT 0x1u  /* attention: a key/value row gather */
 #define SOCKET_DEVERR_TABLE_TIMEOUT  0x2u  /* scoring: a copy into shared memory (soft tables, ids) */
+#define SOCKET_DEVERR_SELECT_TIMEOUT 0x4u  /* selection + attention: a slice's wait for the unit's threshold */
 
 /*
  * socket_hash_keys -- prefill hashing ([ES] step 1 "Pre-cálculo (Prellenado)";
@@ -373,9 +374,11 @@ int socket_set_step_events(void* const* events, int n);
 
 /*
  * socket_set_wait_limit -- failure-path diagnostic.  Sets how many times a
- * decode kernel (scoring, attention) polls for data it has requested before
- * it gives up, sets its bit in the workspace error word
- * (SOCKET_DEVERR_TABLE_TIMEOUT, SOCKET_DEVERR_GATHER_TIMEOUT), lets the
+ * decode kernel polls before it gives up on a wait: scoring and attention
+ * for data they have requested, the fused selection + attention for the
+ * unit's threshold that another of its CTAs publishes.  On expiry the kernel
+ * sets its bit in the workspace error word (SOCKET_DEVERR_TABLE_TIMEOUT,
+ * SOCKET_DEVERR_GATHER_TIMEOUT, SOCKET_DEVERR_SELECT_TIMEOUT), lets the
  * copies it has already issued land, and returns without its results.
  * Default 4194304 polls (~ a second or more); 0 makes every such wait give
  * up at once, which is how tests drive the give-up path without a fault;

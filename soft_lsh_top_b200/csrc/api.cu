@@ -267,8 +267,11 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
         if (B * Hq > 65535) return fail(SOCKET_EUNSUPPORTED, "B*Hq=%lld above 65535", (long long)(B * Hq));
         select_per_head(s);
     }
-    // Splits never exceed ceil(k / 16), the count the advertised size covers.
-    s.nsplit = attention_splits(kv_dtype, q_dtype, s.G, s.U, k, device_num_sms());
+    // Attention splits (or slices of the fused selection + attention) never
+    // exceed ceil(k / 16), the count the advertised size covers.
+    const int num_sms = device_num_sms();
+    const bool fused = select_attend_supported(kv_dtype, q_dtype, s, num_sms);
+    s.nsplit = fused ? select_attend_slices(s, num_sms) : attention_splits(kv_dtype, q_dtype, s.G, s.U, k, num_sms);
     const size_t need = workspace_size(per_head, B, Hq, Hkv, Ncap, d, L, P, k);
     if (workspace_bytes < need)
         return fail(SOCKET_EWORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
@@ -308,6 +311,15 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
                      "score kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(2, cs), "step event record")) != SOCKET_OK) return st;
+    if (fused) {
+        // One kernel selects and attends; the step's fourth event follows the third at once.
+        st = cuda_status(launch_select_attend(scores, unit_hist, cand_cnt, cand, bitmap, topk_done, counters, q, K, V,
+                                              s, part_o, part_ml, err_word, idx_out, out, cs),
+                         "selection + attention kernel launch");
+        if (st != SOCKET_OK) return st;
+        if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
+        return cuda_status(mark_step(4, cs), "step event record");
+    }
     st = cuda_status(launch_topk(scores, unit_hist, cand_cnt, cand, bitmap, topk_done, s, idx_out, cs),
                      "top-k kernel launch");
     if (st != SOCKET_OK) return st;

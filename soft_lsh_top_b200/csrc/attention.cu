@@ -20,13 +20,14 @@
 #include "common.cuh"
 #include "internal.h"
 #include "socket_attn.h"
+#include "warp_attn.cuh"
 
 namespace socket_attn {
 namespace {
 
 constexpr int kThreads = 128;
 constexpr uint32_t kMaxPolls = 1u << 22;
-constexpr float kScale = 0.088388347648318440550f;  // 1 / sqrt(128)
+constexpr float kScale = kInvSqrtD;
 
 template <typename KT>
 struct Rows;
@@ -332,29 +333,13 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
 
 // ---------------------------------------------------------------------------
 // bfloat16 K/V and q, G <= 8: flash-decode split-K with every warp on its own
-// 16-key chunks and both contractions on the tensor cores (warp-level
-// mma.sync m16n8k16, bf16 in, fp32 accumulate):
-//   logits^T [16 heads x 16 keys] = q [16 x 128] * K_chunk^T [128 x 16]
-//     (A = q held in registers, heads G..15 zero; B from ldmatrix of the key
-//      rows, which are B's columns);
-//   out^T   [128 x 16 heads]     += V_chunk^T [128 x 16] * P^T [16 x 8]
-//     (A from ldmatrix.trans of the value rows; B = the weights).
-// The logits' accumulator fragment (head lane/4, keys 2 (lane%4) + {0,1}
-// and + 8) is exactly the B fragment the second product needs, so weights
-// never leave registers; the online softmax of a head reduces over one lane
-// quad.  Weights enter the second product as a bfloat16 high part plus a
-// bfloat16 remainder (~16 bits).  bf16 x bf16 products are exact in fp32, so
-// the logits carry only fp32 accumulation error.
-// Each warp gathers its chunks itself (one bulk copy per 256-byte key or
-// value row, into rows padded to 272 bytes so an ldmatrix phase's 8 rows hit
-// distinct banks) on its own two-stage ring of mbarriers: the chunk loop has
-// no CTA-wide barrier.  The two warps of a CTA then merge in shared memory
-// and the last CTA of the unit merges the CTAs' partials.
+// 16-key chunks and both contractions on the tensor cores (WarpAttn, in
+// warp_attn.cuh).  Each warp gathers its chunks itself on its own two-stage
+// ring of mbarriers: the chunk loop has no CTA-wide barrier.  The two warps
+// of a CTA then merge in shared memory and the last CTA of the unit merges
+// the CTAs' partials.
 // ---------------------------------------------------------------------------
-constexpr int kWChunk = 16;                                // keys per warp chunk
 constexpr int kWStages = 2;
-constexpr int kWRowStride = 272;
-constexpr int kWStageBytes = 2 * kWChunk * kWRowStride;   // keys + values
 constexpr int kWWarps = 2;
 constexpr int kWThreads = 32 * kWWarps;
 constexpr int kWSmemBytes = kWWarps * kWStages * kWStageBytes;
@@ -362,15 +347,6 @@ constexpr int kWCtasPerSm = 6;
 
 // The tensor-core kernel takes bfloat16 q, K, V and groups of up to 8 heads.
 bool warp_path(int kv_dtype, int q_dtype, int G) { return kv_dtype == 1 && q_dtype == 1 && G <= 8; }
-
-// Two floats -> bfloat16x2 (round to nearest even), first in the low half.
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
-{
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-__device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(pack_bf16(x, 0.0f) << 16); }
 
 // The unit's last CTA merges the splits' partials: head h is merged by warp
 // h % kWWarps with no CTA barrier.  Splits are taken 16 at a time, their
@@ -448,7 +424,6 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     int nsplit, int rpc, float* __restrict__ part_o, float2* __restrict__ part_ml, uint32_t* __restrict__ counters,
     uint32_t* __restrict__ err_word, float* __restrict__ out, float2* __restrict__ ml_out, uint32_t max_polls)
 {
-    static_assert(G <= 8, "heads are the M rows 0..7 of the 16-row tile");
     extern __shared__ __align__(128) char smem[];
     __shared__ __align__(8) uint64_t bar[kWWarps][kWStages];
     __shared__ float xm[kWWarps][8], xl[kWWarps][8];
@@ -463,22 +438,8 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     char* wsm_base = smem + warp * kWStages * kWStageBytes;
     const uint32_t wbase = smem_addr(wsm_base);
 
-    // q as the A operand: row h = lane/4 (< G), channels 16 kk + 2 (lane%4) + {0,1} and + 8.
-    uint32_t qa[8][2];
-    {
-        const int h = lane >> 2, c = (lane & 3) * 2;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t v0 = 0, v1 = 0;
-            if (h < G) {
-                const uint16_t* qh = q + (qrow0 + h) * kHeadDim + kk * 16 + c;
-                v0 = (uint32_t)qh[0] | ((uint32_t)qh[1] << 16);
-                v1 = (uint32_t)qh[8] | ((uint32_t)qh[9] << 16);
-            }
-            qa[kk][0] = v0;
-            qa[kk][1] = v1;
-        }
-    }
+    WarpAttn<G> at;
+    at.init(q, qrow0);
     if (tid == 0) {
         for (int w = 0; w < kWWarps; ++w)
             for (int st = 0; st < kWStages; ++st) mbar_init(&bar[w][st], 1);
@@ -502,43 +463,19 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         const int i = lane & 15;
         return (j < cw && i < r_end - r0) ? __ldcg(idx + u * k + r0 + i) : -1;
     };
-    // Gather this warp's chunk j into stage st: lane i < 16 copies key row i,
-    // lane 16 + i value row i; value rows past the chunk's end are zeroed
-    // (their weights are 0, and 0 * NaN from stale bytes must not happen).
+    // Gather this warp's chunk j into stage st.  Indices come from the top-k
+    // kernel and are < N; they are clamped anyway so a gather can never leave
+    // the unit's cache rows.
     auto issue = [&](int j, int st, int32_t r) {
         const int r0 = r_begin + (warp + kWWarps * j) * kWChunk;
         const int nr = min(kWChunk, r_end - r0);
-        const int i = lane & 15;
-        char* dst = wsm_base + st * kWStageBytes + (lane >> 4) * kWChunk * kWRowStride + i * kWRowStride;
-        if (i < nr) {
-            // Indices come from the top-k kernel and are < N; clamp anyway so a
-            // gather can never leave the unit's cache rows.
-            r = (r >= 0 && r < Ncap) ? r : 0;
-            const uint16_t* src = (lane < 16 ? K : V) + (ukv * Ncap + r) * kHeadDim;
-            bulk_copy_g2s(dst, src, kHeadDim * 2, &bar[warp][st]);
-        } else if (lane >= 16) {
-            uint4* z = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-            for (int e = 0; e < kHeadDim * 2 / 16; ++e) z[e] = make_uint4(0, 0, 0, 0);
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&bar[warp][st], (uint32_t)nr * 2u * kHeadDim * 2u);
+        r = (r >= 0 && r < Ncap) ? r : 0;
+        at.issue(wsm_base + st * kWStageBytes, K, V, ukv * Ncap + r, nr, &bar[warp][st]);
     };
     if (cw > 0) issue(0, 0, row_index(0));
     if (cw > 1) issue(1, 1, row_index(1));
     __syncwarp();  // zeroed value rows visible to the warp
 
-    // out^T accumulators: m-tile mt = channels 16 mt ..; [0], [1]: channel
-    // 16 mt + lane/4, heads 2 (lane%4) + {0,1}; [2], [3]: channel + 8.
-    float acc[8][4];
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
-    float m_run = -INFINITY, l_run = 0.0f;  // of head lane/4
-    const int q4 = lane >> 3;
-    // ldmatrix lane address: key row (q4 >> 1) * 8 + lane % 8, channel half q4 & 1
-    const uint32_t lrow = (uint32_t)(((q4 >> 1) * 8 + (lane & 7)) * kWRowStride + (q4 & 1) * 16);
-    const int t2 = (lane & 3) * 2;
     bool ok = true;
     for (int j = 0; j < cw; ++j) {
         const int st = j & 1;
@@ -552,95 +489,25 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
             break;
         }
         const int nr = min(kWChunk, r_end - (r_begin + (warp + kWWarps * j) * kWChunk));
-        const uint32_t ks = wbase + st * kWStageBytes, vs = ks + kWChunk * kWRowStride;
-        // ---- logits^T: keys 0-7 (c0) and 8-15 (c1) of head lane/4.
-        float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            uint32_t bk[4];
-            ldsm_x4(ks + lrow + kk * 32, bk);
-            const uint32_t a[4] = {qa[kk][0], 0u, qa[kk][1], 0u};
-            mma_bf16(c0, a, bk[0], bk[1]);
-            mma_bf16(c1, a, bk[2], bk[3]);
+        at.consume(wbase + st * kWStageBytes, nr);
+        if (j + 2 < cw) {
+            issue(j + 2, st, next_row);
+            __syncwarp();
         }
-        float sv[4] = {c0[0] * kScale, c0[1] * kScale, c1[0] * kScale, c1[1] * kScale};
-        sv[0] = t2 < nr ? sv[0] : -INFINITY;
-        sv[1] = t2 + 1 < nr ? sv[1] : -INFINITY;
-        sv[2] = t2 + 8 < nr ? sv[2] : -INFINITY;
-        sv[3] = t2 + 9 < nr ? sv[3] : -INFINITY;
-        // ---- online softmax of head lane/4 over the quad's 16 keys.
-        float mc = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-        mc = fmaxf(mc, __shfl_xor_sync(kFullMask, mc, 1));
-        mc = fmaxf(mc, __shfl_xor_sync(kFullMask, mc, 2));
-        const float m_new = fmaxf(m_run, mc);
-        const float sc = expf(m_run - m_new);  // 0 on the first chunk (m_run = -inf)
-        float p[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) p[e] = expf(sv[e] - m_new);
-        float ps = (p[0] + p[1]) + (p[2] + p[3]);
-        ps += __shfl_xor_sync(kFullMask, ps, 1);
-        ps += __shfl_xor_sync(kFullMask, ps, 2);
-        l_run = l_run * sc + ps;
-        m_run = m_new;
-        // ---- rescale: the accumulators hold heads 2 (lane%4) and + 1 (quads 2 (lane%4), + 1).
-        const float sa = __shfl_sync(kFullMask, sc, (lane & 3) * 8);
-        const float sb = __shfl_sync(kFullMask, sc, (lane & 3) * 8 + 4);
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            acc[mt][0] *= sa;
-            acc[mt][1] *= sb;
-            acc[mt][2] *= sa;
-            acc[mt][3] *= sb;
-        }
-        // ---- weights as B: (keys 2 (lane%4) + {0,1}, head lane/4) and keys + 8.
-        const float h0 = bf16_round(p[0]), h1 = bf16_round(p[1]), h2 = bf16_round(p[2]), h3 = bf16_round(p[3]);
-        const uint32_t bh0 = pack_bf16(h0, h1), bh1 = pack_bf16(h2, h3);
-        const uint32_t bl0 = pack_bf16(p[0] - h0, p[1] - h1), bl1 = pack_bf16(p[2] - h2, p[3] - h3);
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            uint32_t av[4];
-            ldsm_x4_t(vs + lrow + mt * 32, av);
-            // .trans of (keys (q4>>1)*8.., channels 16 mt + (q4&1)*8..) gives A = V^T in
-            // the order (ch 0-7, k 0-7), (ch 8-15, k 0-7), (ch 0-7, k 8-15), (ch 8-15, k 8-15).
-            mma_bf16(acc[mt], av, bh0, bh1);
-            mma_bf16(acc[mt], av, bl0, bl1);
-        }
-        // Every lane's reads of this stage precede the next copies into it.
-        fence_proxy_async_shared();
-        __syncwarp();
-        if (j + 2 < cw) issue(j + 2, st, next_row);
     }
-    if (!ok) {
-        m_run = -INFINITY;
-        l_run = 0.0f;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[mt][e] = 0.0f;
-    }
+    if (!ok) at.reset();
 
     // ---- merge the two warps: warp 1 leaves (m, l, o^T) in its own stage memory.
     float* xo = reinterpret_cast<float*>(smem + kWStages * kWStageBytes);  // warp 1's area, [8 heads][128]
-    if (warp == 1) {
-        if ((lane & 3) == 0) {
-            xm[1][lane >> 2] = m_run;
-            xl[1][lane >> 2] = l_run;
-        }
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            const int ch = mt * 16 + (lane >> 2);
-            xo[t2 * kHeadDim + ch] = acc[mt][0];
-            xo[(t2 + 1) * kHeadDim + ch] = acc[mt][1];
-            xo[t2 * kHeadDim + ch + 8] = acc[mt][2];
-            xo[(t2 + 1) * kHeadDim + ch + 8] = acc[mt][3];
-        }
-    } else if ((lane & 3) == 0) {
-        xm[0][lane >> 2] = m_run;
-        xl[0][lane >> 2] = l_run;
+    if (warp == 1) at.store(xo, xm[1], xl[1]);
+    else if ((lane & 3) == 0 && (lane >> 2) < G) {
+        xm[0][lane >> 2] = at.m_run;
+        xl[0][lane >> 2] = at.l_run;
     }
     __syncthreads();
     const int64_t pbase = u * G * (int64_t)nsplit;
     if (warp == 0) {
+        const int t2 = (lane & 3) * 2;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int h = t2 + hh;
@@ -652,8 +519,8 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {
                     const int ch = mt * 16 + (lane >> 2);
-                    po[ch] = w0 * acc[mt][hh] + w1 * xo[h * kHeadDim + ch];
-                    po[ch + 8] = w0 * acc[mt][2 + hh] + w1 * xo[h * kHeadDim + ch + 8];
+                    po[ch] = w0 * at.acc[mt][hh] + w1 * xo[h * kHeadDim + ch];
+                    po[ch + 8] = w0 * at.acc[mt][2 + hh] + w1 * xo[h * kHeadDim + ch + 8];
                 }
                 if ((lane >> 2) == 0) part_ml[pbase + h * nsplit + split] = make_float2(M, w0 * xl[0][h] + w1 * xl[1][h]);
             }

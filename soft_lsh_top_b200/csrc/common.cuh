@@ -143,6 +143,26 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Per-thread asynchronous 16-byte copy global -> shared (cp.async, through
+// L2 only).  Completion is tracked in commit groups: cp_async_wait<N>()
+// returns once at most N of this thread's groups are still pending.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// The same copy of src_bytes (0 or 16) bytes, the rest of the 16 zero-filled
+// (0: nothing is read from src).
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Streaming 16-byte load that does not allocate in L1.
 __device__ __forceinline__ uint4 ldg_stream_u4(const void* p)
 {

@@ -40,7 +40,8 @@ struct DecodeWorkspace {
     size_t unit_hist;  // uint32 [U][kScoreHistBins] score histogram
     size_t cand_cnt;   // uint32 [U] top-k candidate counters
     size_t cand;       // uint2 [U][cap] top-k candidates (index, bit pattern), cap = topk_candidate_capacity
-    size_t bitmap;     // uint32 [U][topk_bitmap_stride(Ncap)] top-k selection bitmap
+    size_t bitmap;     // uint32 [U][topk_bitmap_stride(Ncap)] top-k selection bitmap; in the fused
+                       // selection + attention, each unit's record (t, ti, sure counts, first slots)
     size_t tables;     // float [U][ceil(L/32)][NB][64], column j = table 32c + j mod 32
     size_t scores;     // float [U][Ncap]
     size_t part_o;     // float [U][G][nsplit][d]
@@ -99,6 +100,19 @@ int ids_row_bytes(int L);
 cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
                         uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
                         cudaStream_t stream);
+
+// Top-k fused with the attention over the selected keys (select_attend.cu):
+// bfloat16 q, K and V, d = 128, G <= 8, k <= 4096, at most one unit per SM.
+// s.nsplit must be select_attend_slices(s, num_sms): the slices per unit,
+// whose partials part_o / part_ml hold ([U][G][C]).  info ([U][bitmap
+// stride] words), done and tickets ([U], zero at entry, zero again at exit)
+// are scratch.
+bool select_attend_supported(int kv_dtype, int q_dtype, const DecodeShape& s, int num_sms);
+int select_attend_slices(const DecodeShape& s, int num_sms);
+cudaError_t launch_select_attend(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
+                                 uint32_t* info, uint32_t* done, uint32_t* tickets, const void* q, const void* K,
+                                 const void* V, const DecodeShape& s, float* part_o, float2* part_ml,
+                                 uint32_t* err_word, int32_t* idx_out, float* out, cudaStream_t stream);
 
 // counts (nullable): rows of each unit's selection to use (the first
 // counts[u] of its k slots; all k when null).  ml_out (nullable): per query
