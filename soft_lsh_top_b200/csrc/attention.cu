@@ -69,12 +69,7 @@ __device__ __forceinline__ void merge_unit(int64_t u, int nsplit, int64_t pbase,
     static_assert(kHeadDim % NT == 0 && NT % 32 == 0, "NT threads cover the head dimension evenly");
     constexpr int kCols = kHeadDim / NT;  // output columns per thread: tid, tid + NT, ...
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&counters[u], 1u) == (uint32_t)(nsplit - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+    if (!cta_ticket(&counters[u], (uint32_t)(nsplit - 1), s_last)) return;
     // Per head: M = max_s m_s; w_s = exp(m_s - M); out = sum_s w_s o_s / sum_s w_s l_s,
     // accumulated in split order.  Weights are staged in shared memory, NT
     // splits at a time, and the partial rows are read with many loads in flight.
@@ -362,12 +357,7 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
                                                  float2* __restrict__ ml_out, uint32_t& s_last)
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&counters[u], 1u) == (uint32_t)(nsplit - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
+    if (!cta_ticket(&counters[u], (uint32_t)(nsplit - 1), s_last)) return;
     constexpr int kTile = 16;  // splits whose rows are loaded at once
     for (int h = warp; h < G; h += kWWarps) {
         const int64_t base = pbase + h * nsplit;

@@ -163,6 +163,25 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// CTA-wide ticket on a global counter.  The barrier orders every thread's
+// earlier global writes before thread 0's release fence and atomic add; the
+// CTA whose add makes the count `last` (0-based) takes an acquire fence
+// before the closing barrier, so all its threads then see every writer's
+// data (read it with L2-coherent loads).  Returns, in every thread, whether
+// this CTA took the last ticket.  s_flag: a shared word.
+__device__ __forceinline__ bool cta_ticket(uint32_t* counter, uint32_t last, uint32_t& s_flag)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const bool l = atomicAdd(counter, 1u) == last;
+        if (l) __threadfence();
+        s_flag = l ? 1u : 0u;
+    }
+    __syncthreads();
+    return s_flag != 0u;
+}
+
 // Streaming 16-byte load that does not allocate in L1.
 __device__ __forceinline__ uint4 ldg_stream_u4(const void* p)
 {

@@ -260,18 +260,14 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
         uint2* cu = a.cand + u * a.cap;
         for (uint32_t i = tid; i < nl; i += kThreads)
             if (base + i < (uint32_t)a.cap) cu[base + i] = scand[i];
-        __threadfence();
-        __syncthreads();
     }
-    if (a.C > 1) {
-        if (tid == 0) sh.last = atomicAdd(a.done + u, 1u) == (uint32_t)(a.C - 1);
-    } else if (tid == 0) {
-        sh.last = 1u;  // one slice: this CTA selects
-    }
-    __syncthreads();
-    const bool selector = sh.last != 0u;
+    // One slice: this CTA selects (after a barrier: its own list entries are
+    // written).  Else the last to take a ticket, which then sees the other
+    // slices' lists and counts.
+    bool selector = true;
+    if (a.C > 1) selector = cta_ticket(a.done + u, (uint32_t)(a.C - 1), sh.last);
+    else __syncthreads();
     if (selector) {
-        __threadfence();  // the other slices' lists and counts are visible after their tickets
         uint32_t t, ti = 0xffffffffu;
         if (fits && ncand <= (uint32_t)kUnitCandMax) {
             const int nc = (int)ncand;
@@ -343,8 +339,7 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
             s_ti = ti;
             s_ok = 1u;
         }
-        __threadfence();
-        __syncthreads();
+        __syncthreads();  // the record's words precede the release below
         if (tid == 0 && a.C > 1) {
             __threadfence();
             atomicOr(a.done + u, kPublished);
@@ -497,12 +492,7 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
         a.part_o[p * kHeadDim + ch] = o;
         if (ch == 0) a.part_ml[p] = make_float2(M, l);
     }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sh.last = atomicAdd(a.tickets + u, 1u) == (uint32_t)(a.C - 1);
-    __syncthreads();
-    if (!sh.last) return;
-    __threadfence();
+    if (!cta_ticket(a.tickets + u, (uint32_t)(a.C - 1), sh.last)) return;
     // The unit's output: the C slice partials merged per head in slice order.
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
         const int h = e / kHeadDim, ch = e % kHeadDim;

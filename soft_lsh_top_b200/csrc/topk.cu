@@ -174,12 +174,7 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         for (uint32_t i = tid; i < nl; i += kThreads)
             if (base + i < (uint32_t)a.cap) cu[base + i] = scand[i];
         // ---- the unit's last CTA to get here selects.
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) sh.last = atomicAdd(a.done + u, 1u) == (uint32_t)(a.C - 1);
-        __syncthreads();
-        if (!sh.last) return;
-        __threadfence();
+        if (!cta_ticket(a.done + u, (uint32_t)(a.C - 1), sh.last)) return;
     }
 
     int32_t* out = a.idx_out + u * (int64_t)a.k;
