@@ -387,6 +387,24 @@ int socket_set_step_events(void* const* events, int n);
  */
 uint32_t socket_set_wait_limit(uint32_t polls);
 
+/*
+ * socket_set_selection_path -- diagnostic.  Chooses the kernels of steps a4
+ * and a5 (selection and attention) for later decode calls of this process:
+ *   SOCKET_PATH_AUTO (0): by shape.  bf16 q and K/V, G <= 8 and k <= 4096
+ *     take one fused selection + attention kernel when the separate top-k
+ *     kernel would not fill the SMs (B*Hkv*ceil(N/32768) below the SM count,
+ *     per-head calls counting B*Hq units); every other shape takes the
+ *     top-k kernel and then an attention kernel.
+ *   SOCKET_PATH_SEPARATE (1): always the top-k kernel, then attention.
+ * Both paths write the same indices (bit for bit) and outputs that agree to
+ * float32 rounding; tests use this to compare them on the same inputs.
+ * Returns the previous path, or -1 (and changes nothing) for another value.
+ * No counterpart in the method.
+ */
+#define SOCKET_PATH_AUTO     0
+#define SOCKET_PATH_SEPARATE 1
+int socket_set_selection_path(int path);
+
 /* socket_version -- ABI version of this library (major * 100 + minor). */
 int socket_version(void);
 

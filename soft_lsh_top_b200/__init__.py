@@ -22,7 +22,7 @@ __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
     "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check", "socket_decode_append",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events",
-    "socket_set_wait_limit", "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
+    "socket_set_wait_limit", "socket_set_selection_path", "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
     "socket_shard_attend_workspace_size", "socket_shard_combine", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -98,6 +98,8 @@ def load_library(path: str | None = None):
     lib.socket_shard_combine.restype = _int
     lib.socket_set_wait_limit.argtypes = [ctypes.c_uint32]
     lib.socket_set_wait_limit.restype = ctypes.c_uint32
+    lib.socket_set_selection_path.argtypes = [_int]
+    lib.socket_set_selection_path.restype = _int
     lib.socket_ids_row_bytes.argtypes = [_int]
     lib.socket_ids_row_bytes.restype = _int
     lib.socket_version.argtypes = []
@@ -428,6 +430,19 @@ def socket_set_wait_limit(polls: int) -> int:
     once, for tests of the failure path; 0xffffffff: the default).  Returns
     the previous limit."""
     return int(load_library().socket_set_wait_limit(polls & 0xffffffff))
+
+
+SOCKET_PATH_AUTO, SOCKET_PATH_SEPARATE = 0, 1
+
+
+def socket_set_selection_path(path: int) -> int:
+    """Kernels for selection and attention in later decode calls:
+    SOCKET_PATH_AUTO (by shape) or SOCKET_PATH_SEPARATE (always top-k, then
+    attention).  Returns the previous path; raises on another value."""
+    prev = int(load_library().socket_set_selection_path(int(path)))
+    if prev < 0:
+        raise SocketError(SOCKET_EINVAL, f"unknown selection path {path}")
+    return prev
 
 
 # ----------------------------------------------------------------------------

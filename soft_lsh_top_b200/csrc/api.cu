@@ -195,6 +195,8 @@ std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
 
 uint32_t wait_poll_limit() { return g_wait_polls.load(std::memory_order_relaxed); }
 
+std::atomic<int> g_selection_path{SOCKET_PATH_AUTO};
+
 bool pdl_enabled()
 {
     static const bool on = getenv("SOCKET_NO_PDL") == nullptr;
@@ -270,7 +272,8 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     // Attention splits (or slices of the fused selection + attention) never
     // exceed ceil(k / 16), the count the advertised size covers.
     const int num_sms = device_num_sms();
-    const bool fused = select_attend_supported(kv_dtype, q_dtype, s, num_sms);
+    const bool fused = g_selection_path.load(std::memory_order_relaxed) == SOCKET_PATH_AUTO &&
+                       select_attend_supported(kv_dtype, q_dtype, s, num_sms);
     s.nsplit = fused ? select_attend_slices(s, num_sms) : attention_splits(kv_dtype, q_dtype, s.G, s.U, k, num_sms);
     const size_t need = workspace_size(per_head, B, Hq, Hkv, Ncap, d, L, P, k);
     if (workspace_bytes < need)
@@ -356,6 +359,12 @@ const char* socket_last_error(void) { return g_last_error.c_str(); }
 uint32_t socket_set_wait_limit(uint32_t polls)
 {
     return g_wait_polls.exchange(polls == 0xffffffffu ? kDefaultWaitPolls : polls);
+}
+
+int socket_set_selection_path(int path)
+{
+    if (path != SOCKET_PATH_AUTO && path != SOCKET_PATH_SEPARATE) return -1;
+    return g_selection_path.exchange(path);
 }
 
 int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv, int64_t Ncap,

@@ -61,6 +61,15 @@ def test_wait_limit_diagnostic_round_trips(lib):
     assert lib.socket_set_wait_limit(0xFFFFFFFF) == default
 
 
+def test_selection_path_diagnostic_round_trips(lib):
+    """socket_set_selection_path returns the previous path and refuses other
+    values without changing the current one (host state only)."""
+    assert lib.socket_set_selection_path(1) == 0
+    assert lib.socket_set_selection_path(7) == -1
+    assert lib.socket_set_selection_path(0) == 1
+    assert lib.socket_set_selection_path(0) == 0
+
+
 # Fake, aligned, never-dereferenced device addresses: every call below fails
 # validation before it could touch them.
 P16 = 0x10000
