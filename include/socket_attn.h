@@ -388,18 +388,25 @@ int socket_set_step_events(void* const* events, int n);
 uint32_t socket_set_wait_limit(uint32_t polls);
 
 /*
- * socket_set_selection_path -- diagnostic.  Chooses the kernels of steps a4
- * and a5 (selection and attention) for later decode calls of this process:
- *   SOCKET_PATH_AUTO (0): by shape.  bf16 q and K/V, G <= 8 and k <= 4096
- *     take one fused selection + attention kernel when the separate top-k
- *     kernel would not fill the SMs (B*Hkv*ceil(N/32768) below the SM count,
- *     per-head calls counting B*Hq units); every other shape takes the
- *     top-k kernel and then an attention kernel.
- *   SOCKET_PATH_SEPARATE (1): always the top-k kernel, then attention.
- * Both paths write the same indices (bit for bit) and outputs that agree to
- * float32 rounding; tests use this to compare them on the same inputs.
- * Returns the previous path, or -1 (and changes nothing) for another value.
- * No counterpart in the method.
+ * socket_set_selection_path -- diagnostic.  Chooses the kernels of a decode
+ * step for later decode calls of this process.  U is the number of units
+ * (B*Hkv, or B*Hq for per-head calls), G the query heads per unit.
+ *   SOCKET_PATH_AUTO (0): by shape.
+ *     - Small problems take one kernel for the whole step (soft tables,
+ *       scores, top-k, attention): N <= 8192, k <= 1024, L <= 32, G <= 8,
+ *       G*L <= 64, G*L*P <= 512, U at most the SM count, no keys appended in
+ *       the call.
+ *     - Otherwise bf16 q and K/V with G <= 8 and k <= 4096 take a soft-table
+ *       kernel, a scoring kernel and one fused selection + attention kernel
+ *       when the separate top-k kernel would not fill the SMs
+ *       (U*ceil(N/32768) below the SM count).
+ *     - Every other shape takes the four separate kernels: soft tables,
+ *       scoring, top-k, attention.
+ *   SOCKET_PATH_SEPARATE (1): always the four separate kernels.
+ * All paths write the same scores and indices (bit for bit) and outputs that
+ * agree to float32 rounding; tests use this to compare them on the same
+ * inputs.  Returns the previous path, or -1 (and changes nothing) for
+ * another value.  No counterpart in the method.
  */
 #define SOCKET_PATH_AUTO     0
 #define SOCKET_PATH_SEPARATE 1

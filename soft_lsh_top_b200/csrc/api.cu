@@ -272,8 +272,9 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     // Attention splits (or slices of the fused selection + attention) never
     // exceed ceil(k / 16), the count the advertised size covers.
     const int num_sms = device_num_sms();
-    const bool fused = g_selection_path.load(std::memory_order_relaxed) == SOCKET_PATH_AUTO &&
-                       select_attend_supported(kv_dtype, q_dtype, s, num_sms);
+    const bool by_shape = g_selection_path.load(std::memory_order_relaxed) == SOCKET_PATH_AUTO;
+    const bool small = by_shape && n_new == 0 && small_step_supported(s, num_sms);
+    const bool fused = by_shape && !small && select_attend_supported(kv_dtype, q_dtype, s, num_sms);
     s.nsplit = fused ? select_attend_slices(s, num_sms) : attention_splits(kv_dtype, q_dtype, s.G, s.U, k, num_sms);
     const size_t need = workspace_size(per_head, B, Hq, Hkv, Ncap, d, L, P, k);
     if (workspace_bytes < need)
@@ -294,6 +295,16 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
 
     if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
+    if (small) {
+        // One kernel for the whole step; the step's other events follow at once.
+        st = cuda_status(launch_small_step(q, q_dtype, W, ids, vnorm, K, V, kv_dtype, s, tau, idx_out, out,
+                                           scores_out, err_word, cs),
+                         "small-step kernel launch");
+        if (st != SOCKET_OK) return st;
+        for (int i = 1; i <= 4; ++i)
+            if ((st = cuda_status(mark_step(i, cs), "step event record")) != SOCKET_OK) return st;
+        return SOCKET_OK;
+    }
     AppendHash app;
     if (n_new > 0) {
         app.K = K;

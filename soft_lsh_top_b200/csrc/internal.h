@@ -114,6 +114,16 @@ cudaError_t launch_select_attend(const float* scores, const uint32_t* unit_hist,
                                  const void* V, const DecodeShape& s, float* part_o, float2* part_ml,
                                  uint32_t* err_word, int32_t* idx_out, float* out, cudaStream_t stream);
 
+// The whole step (soft tables, scores, top-k, attention) in one kernel, one
+// CTA per unit (small_step.cu): N <= 8192, k <= 1024, L <= 32, G <= 8,
+// G*L <= 64, G*L*P <= 512, at most one unit per SM.  Writes only idx_out,
+// out, scores_out (nullable) and clears the error word.
+bool small_step_supported(const DecodeShape& s, int num_sms);
+cudaError_t launch_small_step(const void* q, int q_dtype, const uint16_t* W, const uint8_t* ids, const float* vnorm,
+                              const void* K, const void* V, int kv_dtype, const DecodeShape& s, double tau,
+                              int32_t* idx_out, float* out, float* scores_out, uint32_t* err_word,
+                              cudaStream_t stream);
+
 // counts (nullable): rows of each unit's selection to use (the first
 // counts[u] of its k slots; all k when null).  ml_out (nullable): per query
 // row the largest logit and the sum of exp(logit - largest) over those rows

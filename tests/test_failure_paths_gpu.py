@@ -5,12 +5,16 @@ stays usable.
 socket_set_wait_limit(0) makes every bounded wait of the decode kernels give
 up at once: the scoring kernel's and the attention kernel's waits for data
 they have requested, and the fused selection + attention kernel's wait for
-the threshold that the unit's last CTA publishes (that kernel runs for these
-few-unit bf16 shapes; fp32 keys take the separate top-k and attention
-kernels).  The kernels then set their bit in the error word, wait (with the
-normal, long limit) for the copies they have already issued to land, and
-return without results -- the path a real expiry takes.  Nothing here traps,
-faults or hangs: no wait is left on something that never arrives.
+the threshold that the unit's last CTA publishes.  The kernels then set
+their bit in the error word, wait (with the normal, long limit) for the
+copies they have already issued to land, and return without results -- the
+path a real expiry takes.  Nothing here traps, faults or hangs: no wait is
+left on something that never arrives.
+
+The shape (N above the one-kernel step's limit, so that path, which has no
+bounded waits, is not taken) runs, by path: bf16 by shape -> soft tables,
+scoring, fused selection + attention; bf16 forced separate and fp32 ->
+soft tables, scoring, top-k, attention.
 """
 import pytest
 import torch
@@ -29,9 +33,18 @@ def _bits(t):
     return t.view(torch.int32) if t.dtype == torch.float32 else t
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_expired_waits_are_reported_and_the_context_stays_usable(dtype):
-    w = wl.Workload(name="expiry", B=1, Hq=4, Hkv=2, N=5000, L=8, P=8, tau=0.4, k=300, dtype=dtype, seed=7100)
+@pytest.mark.parametrize("dtype,path", [("bf16", "auto"), ("bf16", "separate"), ("f32", "auto")])
+def test_expired_waits_are_reported_and_the_context_stays_usable(dtype, path):
+    w = wl.Workload(name="expiry", B=1, Hq=4, Hkv=2, N=9000, L=8, P=8, tau=0.4, k=300, dtype=dtype, seed=7100)
+    mode = sk.SOCKET_PATH_AUTO if path == "auto" else sk.SOCKET_PATH_SEPARATE
+    before = sk.socket_set_selection_path(mode)
+    try:
+        _expire_and_recover(w, dtype, fused=(dtype == "bf16" and path == "auto"))
+    finally:
+        sk.socket_set_selection_path(before)
+
+
+def _expire_and_recover(w, dtype, fused):
     inp = wl.make_inputs(w, DEV)
     ids, vnorm = gpu_hash(inp, w)
     ws, idx, out = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, DEV)
@@ -52,9 +65,9 @@ def test_expired_waits_are_reported_and_the_context_stays_usable(dtype):
     finally:
         sk.socket_set_wait_limit(previous)
     assert err & TABLE, hex(err)
-    # bf16: the fused kernel's slices wait for the unit's threshold; fp32: the
-    # attention kernel's row gathers wait for their copies.
-    assert err & (SELECT if dtype == "bf16" else GATHER), hex(err)
+    # The fused kernel's slices wait for the unit's threshold; the attention
+    # kernel's row gathers wait for their copies.
+    assert err & (SELECT if fused else GATHER), hex(err)
 
     idx.fill_(-1)
     out.fill_(float("nan"))

@@ -1,14 +1,17 @@
-"""The two kernel paths for selection and attention agree on the same inputs.
+"""The kernel paths of a decode step agree on the same inputs.
 
-For few (batch, kv-head) units with bf16 data, socket_decode runs one fused
-selection + attention kernel; otherwise it runs the top-k kernel and then an
-attention kernel (socket_set_selection_path documents the rule).  Both are
+By shape, socket_decode runs the whole step in one kernel (small problems),
+or a fused selection + attention kernel after the soft-table and scoring
+kernels (few bf16 units), or four separate kernels (socket_set_selection_path
+documents the rule and can force the separate kernels).  Every path is
 parity-tested against the oracle elsewhere; here the same inputs go through
-both, and the selections must be identical bit for bit (the same exact rule:
-the k largest float32 scores, ties to the lower index, ascending) and the
-outputs equal up to float32 summation order.  The cases cover several slices
-per unit, one slice, per-head units, a threshold bin over the candidate
-capacity (all scores tied), and a ragged tail.
+the shape's own path and through the separate kernels.  Scores must be
+identical bit for bit (the same float32 operations in the same order), so
+must the selections (the k largest scores, ties to the lower index,
+ascending), and the outputs must agree up to float32 summation order.  The
+cases cover several slices per unit, one slice, per-head units, a threshold
+bin over the candidate capacity (all scores tied), a ragged tail, and the
+one-kernel step with fp32 and bf16 data, hard LSH (tau = 0) and P < 4.
 """
 import pytest
 import torch
@@ -32,6 +35,16 @@ CASES = {
                  True, False),
     "all_ties_over_capacity": (wl.Workload(name="paths_e", B=1, Hq=4, Hkv=2, N=12000, L=5, P=8, tau=0.3, k=700,
                                            seed=7305), False, True),
+    # The one-kernel step (N <= 8192, L <= 32, small G * L).
+    "one_kernel_tiny_f32": (wl.TINY, False, False),
+    "one_kernel_bf16_group4": (wl.Workload(name="paths_f", B=2, Hq=8, Hkv=2, N=6001, L=12, P=8, tau=0.3, k=500,
+                                           seed=7306), False, False),
+    "one_kernel_per_head": (wl.Workload(name="paths_g", B=1, Hq=8, Hkv=2, N=5000, L=20, P=6, tau=0.6, k=1000,
+                                        seed=7307), True, False),
+    "one_kernel_hard_lsh_p3": (wl.Workload(name="paths_h", B=1, Hq=2, Hkv=1, N=8192, L=32, P=3, tau=0.0, k=64,
+                                           dtype="f32", seed=7308), False, False),
+    "one_kernel_all_ties": (wl.Workload(name="paths_i", B=1, Hq=4, Hkv=2, N=3000, L=5, P=8, tau=0.3, k=333,
+                                        seed=7309), False, True),
 }
 
 
