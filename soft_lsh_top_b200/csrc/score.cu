@@ -111,21 +111,25 @@ struct ScoreArgs {
 };
 
 // NBLK: 32-table blocks scored by this launch (1 or 2); REGIONS: 64 KB table
-// regions in shared memory (REGIONS / NBLK units staged at once); KEYS:
-// 32-key chunks per warp per batch; NS: batches in a warp's copy ring;
+// regions in shared memory (REGIONS / (NBLK HPC) segments staged at once);
+// KEYS: 32-key chunks per warp per batch; NS: batches in a warp's copy ring;
 // FIRST / LAST: whether this launch starts / finishes the sum (launches in
-// between pass partial sums through the score buffer).
-template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST>
+// between pass partial sums through the score buffer); HPC: units (query
+// heads, when every head selects its own keys) scored by one CTA from the
+// same id rows -- each id row's loads and byte permutes serve all of them,
+// and two heads' sums advance in one packed add.
+template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST, int HPC = 1>
 __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
 {
-    static_assert(REGIONS >= NBLK && REGIONS <= kMaxRegions, "a unit's blocks fit the regions");
+    static_assert(REGIONS >= NBLK * HPC && REGIONS <= kMaxRegions, "a segment's blocks fit the regions");
+    static_assert(HPC == 1 || (HPC == 2 && NBLK == 1 && FIRST && LAST), "two units per CTA: one launch, L <= 32");
     constexpr int V = 2 * NBLK;                            // 16-byte id pieces per key
-    constexpr int kSlots = REGIONS / NBLK;                 // units staged at once
+    constexpr int kSlots = REGIONS / (NBLK * HPC);         // segments staged at once
     constexpr uint32_t kChunkIds = 1024u * NBLK;           // id bytes of a chunk in this launch
     constexpr uint32_t kChunkBytes = kChunkIds + (LAST ? 128u : 0u);  // + the chunk's norms
     constexpr uint32_t kStageBytes = KEYS * kChunkBytes;
     constexpr uint32_t kRingBytes = NS * kStageBytes;
-    constexpr uint32_t kHistBytes = LAST ? kHistBins * 4u : 0u;
+    constexpr uint32_t kHistBytes = LAST ? HPC * kHistBins * 4u : 0u;
     extern __shared__ __align__(1024) char smem[];
     __shared__ __align__(8) uint64_t bar[kSlots];
     __shared__ __align__(8) uint64_t ring_bar[kWarps][NS];
@@ -159,8 +163,9 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     uint32_t* shist = reinterpret_cast<uint32_t*>(smem + (hist_s - sbase));
     char* ring = smem + (ring_s - sbase);
 
-    const int h = (int)(blockIdx.x % (unsigned)a.share);  // this CTA's unit within each kv unit
-    const int64_t c0 = (int64_t)(blockIdx.x / (unsigned)a.share) * a.chunks_per_cta;
+    const unsigned cpg = (unsigned)(a.share / HPC);        // CTAs per group
+    const int h = (int)(blockIdx.x % cpg) * HPC;           // this CTA's first unit within each kv unit
+    const int64_t c0 = (int64_t)(blockIdx.x / cpg) * a.chunks_per_cta;
     const int64_t c1 = min64(a.total_chunks, c0 + a.chunks_per_cta);
     if (c0 >= c1) return;
     const int cpu = (int)a.chunks_per_unit;
@@ -173,7 +178,7 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     // Let the next kernel on the stream get its CTAs queued behind this grid.
     pdl_launch_dependents();
     if (LAST)
-        for (int b = tid; b < kHistBins; b += kThreads) shist[b] = 0;
+        for (int b = tid; b < HPC * kHistBins; b += kThreads) shist[b] = 0;
     if (tid == 0) {
         for (int s = 0; s < kSlots; ++s) mbar_init(&bar[s], 1);
         for (int w = 0; w < kWarps; ++w)
@@ -182,17 +187,20 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     }
     __syncthreads();
 
-    // Bulk copy of segment k's table blocks into its slot's regions.
+    // Bulk copy of segment k's table blocks into its slot's regions (unit
+    // h + hh's blocks at regions (s HPC + hh) NBLK + bl).
     auto issue_tables = [&](int k) {
         const int s = k % kSlots;
-        const int64_t u = (u_first + k) * a.share + h;
-        mbar_arrive_expect_tx(&bar[s], NBLK * region_bytes);
-        for (int bl = 0; bl < NBLK; ++bl) {
-            const char* src = reinterpret_cast<const char*>(a.tables) +
-                              ((u * a.nblk + a.blk0 + bl) * (int64_t)region_bytes);
-            char* dst = region0_ptr + (s * NBLK + bl) * kRegionBytes;
-            for (uint32_t off = 0; off < region_bytes; off += 16384u)
-                bulk_copy_g2s(dst + off, src + off, min(16384u, region_bytes - off), &bar[s]);
+        mbar_arrive_expect_tx(&bar[s], HPC * NBLK * region_bytes);
+        for (int hh = 0; hh < HPC; ++hh) {
+            const int64_t u = (u_first + k) * a.share + h + hh;
+            for (int bl = 0; bl < NBLK; ++bl) {
+                const char* src = reinterpret_cast<const char*>(a.tables) +
+                                  ((u * a.nblk + a.blk0 + bl) * (int64_t)region_bytes);
+                char* dst = region0_ptr + ((s * HPC + hh) * NBLK + bl) * kRegionBytes;
+                for (uint32_t off = 0; off < region_bytes; off += 16384u)
+                    bulk_copy_g2s(dst + off, src + off, min(16384u, region_bytes - off), &bar[s]);
+            }
         }
     };
 
@@ -300,13 +308,19 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                 if (lane == 0) issue(b + NS);
                 issued = b + NS + 1;
             }
-            float acc[KEYS];
+            float acc[KEYS][HPC];
 #pragma unroll
             for (int j = 0; j < KEYS; ++j)
-                acc[j] = FIRST ? 0.0f : __ldcg(su + min(min(chunk_at(b * KEYS + j), cend - 1) * 32 + lane, N - 1));
+#pragma unroll
+                for (int hh = 0; hh < HPC; ++hh)
+                    acc[j][hh] = FIRST ? 0.0f
+                                       : __ldcg(su + hh * a.Ncap +
+                                                min(min(chunk_at(b * KEYS + j), cend - 1) * 32 + lane, N - 1));
 #pragma unroll
             for (int bl = 0; bl < NBLK; ++bl) {
-                const uint32_t base = region0 + (uint32_t)(slot * NBLK + bl) * kRegionBytes + ((uint32_t)lane << 2);
+                // Unit h + hh's block bl sits 64 KB x hh (NBLK) above unit h's.
+                const uint32_t base =
+                    region0 + (uint32_t)(slot * HPC * NBLK + bl) * kRegionBytes + ((uint32_t)lane << 2);
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     const int q = bl * 32 + r;  // id byte within this launch's part of the row
@@ -314,14 +328,23 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                     auto row = [&](int j) {
                         return __byte_perm(base, word_of(v[j][q >> 4], (q >> 2) & 3), 0x3240u | ((q & 3) << 4));
                     };
-                    if constexpr (KEYS % 2 == 0) {
+                    if constexpr (HPC == 2) {
+                        // the two units' sums of a key advance in one packed float32x2 add
+#pragma unroll
+                        for (int j = 0; j < KEYS; ++j) {
+                            const uint32_t rw = row(j);
+                            add_f32x2(acc[j][0], acc[j][1], lds_f32(rw + 4u * r),
+                                      lds_f32(rw + (uint32_t)(NBLK * kRegionBytes) + 4u * r));
+                        }
+                    } else if constexpr (KEYS % 2 == 0) {
                         // two keys' sums advance in one packed float32x2 add
 #pragma unroll
                         for (int j = 0; j < KEYS; j += 2)
-                            add_f32x2(acc[j], acc[j + 1], lds_f32(row(j) + 4u * r), lds_f32(row(j + 1) + 4u * r));
+                            add_f32x2(acc[j][0], acc[j + 1][0], lds_f32(row(j) + 4u * r),
+                                      lds_f32(row(j + 1) + 4u * r));
                     } else {
 #pragma unroll
-                        for (int j = 0; j < KEYS; ++j) acc[j] += lds_f32(row(j) + 4u * r);
+                        for (int j = 0; j < KEYS; ++j) acc[j][0] += lds_f32(row(j) + 4u * r);
                     }
                 }
             }
@@ -330,10 +353,15 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
                 const int c = chunk_at(b * KEYS + j);
                 const int n = c * 32 + lane;
                 if (c < cend && n < N) {
-                    const float sc = LAST ? acc[j] * vn[j] : acc[j];
-                    st_global_hint(su + n, sc, pol_keep);
-                    if (LAST)
-                        atomicAdd(shist + min(__float_as_uint(sc) >> kHistShift, (uint32_t)(kHistBins - 1)), 1u);
+#pragma unroll
+                    for (int hh = 0; hh < HPC; ++hh) {
+                        const float sc = LAST ? acc[j][hh] * vn[j] : acc[j][hh];
+                        st_global_hint(su + hh * a.Ncap + n, sc, pol_keep);
+                        if (LAST)
+                            atomicAdd(shist + hh * kHistBins +
+                                          min(__float_as_uint(sc) >> kHistShift, (uint32_t)(kHistBins - 1)),
+                                      1u);
+                    }
                 }
             }
         }
@@ -345,10 +373,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
         seq += nbatch;
 
         if (LAST) {
-            // The unit's score histogram.
+            // The units' score histograms.
             __syncthreads();
-            uint32_t* gh = a.unit_hist + u * kHistBins;
-            for (int bn = tid; bn < kHistBins; bn += kThreads) {
+            uint32_t* gh = a.unit_hist + u * kHistBins;  // units u .. u + HPC - 1 are adjacent
+            for (int bn = tid; bn < HPC * kHistBins; bn += kThreads) {
                 const uint32_t c = shist[bn];
                 if (c) {
                     atomicAdd(gh + bn, c);
@@ -365,10 +393,10 @@ __global__ __launch_bounds__(kThreads, 1) void score_kernel(const ScoreArgs a)
     }
 }
 
-template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST>
+template <int NBLK, int REGIONS, int KEYS, int NS, bool FIRST, bool LAST, int HPC = 1>
 cudaError_t launch_one(const ScoreArgs& args, int grid, cudaStream_t stream)
 {
-    auto kern = score_kernel<NBLK, REGIONS, KEYS, NS, FIRST, LAST>;
+    auto kern = score_kernel<NBLK, REGIONS, KEYS, NS, FIRST, LAST, HPC>;
     cudaError_t e = set_smem_limit_once((const void*)kern, kSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream, args);
@@ -400,11 +428,15 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
     a.max_polls = wait_poll_limit();
     a.chunks_per_unit = (s.N + 31) / 32;
     a.total_chunks = (s.U / s.share) * a.chunks_per_unit;
+    // When every query head selects its own keys and L <= 32, a CTA scores two
+    // heads of a kv unit from one stream of its ids.
+    const int hpc = (s.share % 2 == 0 && a.nblk == 1) ? 2 : 1;
+    const int cpg = s.share / hpc;  // CTAs per group
     // At least one chunk per warp per CTA; at most one CTA per SM; groups of
-    // `share` CTAs.
+    // `cpg` CTAs.
     const int64_t want = (a.total_chunks + kWarps - 1) / kWarps;
-    const int64_t groups = max64(1, min64(device_num_sms() / s.share, want));
-    const int grid = (int)(groups * s.share);
+    const int64_t groups = max64(1, min64(device_num_sms() / cpg, want));
+    const int grid = (int)(groups * cpg);
     a.chunks_per_cta = (a.total_chunks + groups - 1) / groups;
     // Blocks two at a time (two 64 KB regions); partial sums pass through
     // the score buffer between launches when L > 64.
@@ -414,7 +446,9 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
         a.first = b0 == 0;
         a.last = b0 + nb == a.nblk;
         cudaError_t e;
-        if (nb == 1)
+        if (nb == 1 && hpc == 2)
+            e = launch_one<1, 2, 1, 3, true, true, 2>(a, grid, stream);  // one launch: nblk == 1
+        else if (nb == 1)
             e = a.first ? launch_one<1, 2, 2, 2, true, true>(a, grid, stream)
                         : launch_one<1, 2, 2, 2, false, true>(a, grid, stream);
         else if (a.first)
