@@ -81,9 +81,9 @@ __host__ __device__ constexpr int smem_bytes(int G, int slots)
 template <typename QT>
 __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L, int P, double tau,
-    const AppendHash app, int64_t Ncap, int share, float* __restrict__ tables, uint32_t* __restrict__ err_word,
-    uint32_t* __restrict__ counters, uint32_t* __restrict__ topk_done, uint32_t* __restrict__ unit_hist,
-    uint32_t* __restrict__ cand_cnt)
+    const AppendHash app, int64_t Ncap, int share, bool sep, float* __restrict__ tables,
+    uint32_t* __restrict__ err_word, uint32_t* __restrict__ counters, uint32_t* __restrict__ topk_done,
+    uint32_t* __restrict__ unit_hist, uint32_t* __restrict__ cand_cnt)
 {
     __shared__ uint32_t aid[kMaxAppend][kTpb];  // ids of the appended keys (bit p <-> plane p)
     extern __shared__ __align__(16) char st_dyn[];
@@ -300,33 +300,45 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
         __syncthreads();
     }
 
+    // Units whose tables this CTA writes: u itself, or (sep) the G units
+    // u G .. u G + G - 1, one per query head.
+    const int nunits = sep ? G : 1;
+    const int64_t unit0 = sep ? u * G : u;
     if (blockIdx.y == 0) {
-        if (tid == 0) {
-            counters[u] = 0u;
-            topk_done[u] = 0u;
-            cand_cnt[u] = 0u;
-            if (u == 0) *err_word = 0u;
+        if (tid < nunits) {
+            const int64_t uu = unit0 + tid;
+            counters[uu] = 0u;
+            topk_done[uu] = 0u;
+            cand_cnt[uu] = 0u;
+            if (uu == 0) *err_word = 0u;
         }
-        uint4* hz = reinterpret_cast<uint4*>(unit_hist + u * kScoreHistBins);
-        for (int i = tid; i < kScoreHistBins / 4; i += kThreads) hz[i] = make_uint4(0, 0, 0, 0);
+        uint4* hz = reinterpret_cast<uint4*>(unit_hist + unit0 * kScoreHistBins);
+        for (int i = tid; i < nunits * kScoreHistBins / 4; i += kThreads) hz[i] = make_uint4(0, 0, 0, 0);
     }
     const int nblk = (L + 31) / 32;
-    float* tu = tables + u * nblk * (int64_t)NB * 64;
     // Entry `bucket` of the CTA's four tables: four adjacent columns (and
-    // their copies 32 columns on) of one row, as vector stores.
-    for (int bucket = tid; bucket < NB; bucket += kThreads) {
+    // their copies 32 columns on) of one row, as vector stores.  Summed over
+    // the G heads, or (sep) one table per head, T = lo x hi rounded once.
+    for (int e = tid; e < nunits * NB; e += kThreads) {
+        const int bucket = e % NB, hs = e / NB;
         float vals[kTpb];
 #pragma unroll
         for (int t = 0; t < kTpb; ++t) {
             double acc = 0.0;
-            if (t < nt)
-                for (int h0 = 0; h0 < G; h0 += 4)
+            if (t < nt) {
+                if (sep) {
+                    acc = fma(NIB(hs, t, 0, bucket & 15), NIB(hs, t, 1, bucket >> 4), acc);
+                } else {
+                    for (int h0 = 0; h0 < G; h0 += 4)
 #pragma unroll
-                    for (int hh = 0; hh < 4; ++hh)
-                        if (h0 + hh < G)
-                            acc = fma(NIB(h0 + hh, t, 0, bucket & 15), NIB(h0 + hh, t, 1, bucket >> 4), acc);
+                        for (int hh = 0; hh < 4; ++hh)
+                            if (h0 + hh < G)
+                                acc = fma(NIB(h0 + hh, t, 0, bucket & 15), NIB(h0 + hh, t, 1, bucket >> 4), acc);
+                }
+            }
             vals[t] = (float)acc;
         }
+        float* tu = tables + (unit0 + hs) * nblk * (int64_t)NB * 64;
         float* row = tu + ((int64_t)(l0 >> 5) * NB + bucket) * 64 + (l0 & 31);
         const float4 a = make_float4(vals[0], vals[1], vals[2], vals[3]);
         *reinterpret_cast<float4*>(row) = a;
@@ -370,20 +382,28 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
                                uint32_t* counters, uint32_t* topk_done, uint32_t* unit_hist, uint32_t* cand_cnt,
                                cudaStream_t stream)
 {
-    const int smem = smem_bytes(s.G, app.end > app.begin ? kKeySlots : 0);
-    const dim3 grid((unsigned)s.U, (unsigned)(32 / kTpb * ((s.L + 31) / 32)));
+    // When every query head selects its own keys (G = 1, share heads per kv
+    // unit), a CTA builds the tables of all `share` heads of a kv unit: their
+    // dot products share the hyperplane rows' reads, as a group's do, and
+    // each head keeps its own table (the same operations as one head alone).
+    const bool sep = s.G == 1 && s.share > 1;
+    const int G = sep ? s.share : s.G;
+    const int share = sep ? 1 : s.share;
+    const int64_t ctas = sep ? s.U / s.share : s.U;
+    const int smem = smem_bytes(G, app.end > app.begin ? kKeySlots : 0);
+    const dim3 grid((unsigned)ctas, (unsigned)(32 / kTpb * ((s.L + 31) / 32)));
     if (q_dtype == 1) {
         cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<uint16_t>, smem_bytes(kMaxGroup, kKeySlots));
         if (e != cudaSuccess) return e;
         return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), (size_t)smem, stream,
-                          static_cast<const uint16_t*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables,
-                          err_word, counters, topk_done, unit_hist, cand_cnt);
+                          static_cast<const uint16_t*>(q), W, G, s.L, s.P, tau, app, s.Ncap, share, sep,
+                          tables, err_word, counters, topk_done, unit_hist, cand_cnt);
     }
     cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<float>, smem_bytes(kMaxGroup, kKeySlots));
     if (e != cudaSuccess) return e;
     return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), (size_t)smem, stream,
-                      static_cast<const float*>(q), W, s.G, s.L, s.P, tau, app, s.Ncap, s.share, tables, err_word,
-                      counters, topk_done, unit_hist, cand_cnt);
+                      static_cast<const float*>(q), W, G, s.L, s.P, tau, app, s.Ncap, share, sep, tables,
+                      err_word, counters, topk_done, unit_hist, cand_cnt);
 }
 
 }  // namespace socket_attn
