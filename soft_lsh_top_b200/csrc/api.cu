@@ -237,6 +237,8 @@ DecodeWorkspace decode_workspace_layout(const DecodeShape& s)
     off = align256(off + 8 * (size_t)s.U * s.G * s.nsplit);
     w.sel_idx = off;
     off = align256(off + 4 * (size_t)s.U * s.k);
+    w.topk_info = off;
+    off = align256(off + 4 * (size_t)s.U * (size_t)topk_info_stride(s.Ncap));
     w.total = off;
     return w;
 }
@@ -334,7 +336,8 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
         if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
         return cuda_status(mark_step(4, cs), "step event record");
     }
-    st = cuda_status(launch_topk(scores, unit_hist, cand_cnt, cand, bitmap, topk_done, s, idx_out, cs),
+    st = cuda_status(launch_topk(scores, unit_hist, cand_cnt, cand, bitmap, topk_done,
+                                 reinterpret_cast<uint32_t*>(base + w.topk_info), err_word, s, idx_out, cs),
                      "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     if ((st = cuda_status(mark_step(3, cs), "step event record")) != SOCKET_OK) return st;
@@ -501,7 +504,8 @@ int socket_shard_select(const void* q, int q_dtype, const uint16_t* W, const uin
     st = cuda_status(launch_topk(scores, reinterpret_cast<uint32_t*>(base + w.unit_hist),
                                  reinterpret_cast<uint32_t*>(base + w.cand_cnt), reinterpret_cast<uint2*>(base + w.cand),
                                  reinterpret_cast<uint32_t*>(base + w.bitmap),
-                                 reinterpret_cast<uint32_t*>(base + w.topk_done), s, sel, cs),
+                                 reinterpret_cast<uint32_t*>(base + w.topk_done),
+                                 reinterpret_cast<uint32_t*>(base + w.topk_info), err_word, s, sel, cs),
                      "top-k kernel launch");
     if (st != SOCKET_OK) return st;
     return cuda_status(launch_shard_pairs(scores, sel, s, k_eff, k, n_offset, cand_score, cand_index, cs),

@@ -31,6 +31,9 @@ int topk_candidate_capacity(int64_t Ncap);
 // Words per unit row of the top-k selection bitmap (Ncap / 32 rounded up to
 // a multiple of 4, so every row starts on a 16-byte boundary).
 int64_t topk_bitmap_stride(int64_t Ncap);
+// Words per unit of the top-k slices' record (keys in or above d0 per slice,
+// first output slot per slice).
+int64_t topk_info_stride(int64_t Ncap);
 
 // Workspace regions (byte offsets from the workspace base, 256-aligned).
 struct DecodeWorkspace {
@@ -47,6 +50,7 @@ struct DecodeWorkspace {
     size_t part_o;     // float [U][G][nsplit][d]
     size_t part_ml;    // float2 [U][G][nsplit]
     size_t sel_idx;    // int32 [U][k] a shard's own selection (local indices)
+    size_t topk_info;  // uint32 [U][topk_info_stride(Ncap)] top-k slices' counts and first slots
     size_t total;
 };
 
@@ -98,8 +102,8 @@ cudaError_t launch_score(const float* tables, const uint8_t* ids, const float* v
 int ids_row_bytes(int L);
 
 cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
-                        uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
-                        cudaStream_t stream);
+                        uint32_t* bitmap, uint32_t* done, uint32_t* info, uint32_t* err_word, const DecodeShape& s,
+                        int32_t* idx_out, cudaStream_t stream);
 
 // Top-k fused with the attention over the selected keys (select_attend.cu):
 // bfloat16 q, K and V, d = 128, G <= 8, k <= 4096, at most one unit per SM.

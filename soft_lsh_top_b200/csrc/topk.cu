@@ -29,9 +29,21 @@
 // If the threshold bin holds more keys than the candidate list can take, the
 // last CTA instead selects over all of the unit's scores (three radix digits)
 // and writes the selection from a compaction pass over the scores.
+//
+// When a unit has many slices and the whole grid is resident at once
+// (`spread`), the unit's CTAs share
+// the writing instead: the last CTA clears the dropped candidates' bits in
+// the unit's bitmap, works out every slice's first output slot (its keys in
+// or above d0, less its dropped candidates, summed over the slices before
+// it), and publishes them behind a flag in the ticket word; every CTA of the
+// unit then writes its own slice's selection from its slot.  The other CTAs
+// wait for that flag, a bounded wait (SOCKET_DEVERR_SELECT_TIMEOUT on
+// expiry); they can wait safely because the last CTA is the last to take a
+// ticket, so it is running once anyone waits.
 #include "common.cuh"
 #include "internal.h"
 #include "select.cuh"
+#include "socket_attn.h"
 
 namespace socket_attn {
 namespace {
@@ -52,13 +64,59 @@ struct TopkArgs {
     uint32_t* bitmap;          // [U][bm_stride] (Ncap / 32 words used)
     uint32_t* done;            // [U] tickets of finished CTAs (zeroed before the step)
     int32_t* idx_out;          // [U][k]
-    int64_t Ncap, bm_stride;
+    uint32_t* info;            // [U][info_stride]: keys in or above d0 per slice [C], first slot per slice [C]
+    uint32_t* err_word;
+    int64_t Ncap, bm_stride, info_stride;
     int N, k, C, cap;
+    int spread;                // every CTA writes its own slice's selection (grid resident at once)
+    uint32_t max_polls;
 };
+
+constexpr uint32_t kPublished = 0x80000000u;  // set in the unit's ticket word once the slots are out
+constexpr int kSpreadMinSlices = 8;
+constexpr int kSpreadMaxSlices = 256;
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Writes slice r's selected keys (the set bits of its words of the unit's
+// bitmap, final once the slots are published) in index order from output
+// slot `slot` on: two words per thread, one block-wide scan.
+__device__ __forceinline__ void write_slice(const TopkArgs& a, int64_t u, int r, uint32_t slot, Shared& sh)
+{
+    static_assert(kSliceKeys / 32 == 2 * kThreads, "two bitmap words of the slice per thread");
+    const int tid = threadIdx.x;
+    const int words = (a.N + 31) / 32;
+    const int w = r * (kSliceKeys / 32) + 2 * tid;
+    const uint32_t* bm = a.bitmap + u * a.bm_stride;
+    const uint32_t x0 = w < words ? __ldcg(bm + w) : 0u, x1 = w + 1 < words ? __ldcg(bm + w + 1) : 0u;
+    uint32_t total;
+    uint32_t pos = slot + block_exclusive_scan(__popc(x0) + __popc(x1), sh.warp_sums, total);
+    int32_t* out = a.idx_out + u * (int64_t)a.k;
+    const uint32_t xs[2] = {x0, x1};
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        uint32_t x = xs[q];
+        while (x) {
+            const int b = __ffs(x) - 1;
+            x &= x - 1;
+            // pos < k whenever the threshold is exact; the guard keeps every
+            // store inside the unit's k slots regardless.
+            if (pos < (uint32_t)a.k) out[pos] = 32 * (w + q) + b;
+            ++pos;
+        }
+    }
+}
 
 // Grid: U * C CTAs of kThreads; CTA r of unit u reads keys [r S, min(N, (r+1) S)).
 // Dynamic shared memory: the CTA's candidates (then the unit's) and one tile
 // of the selection bitmap.
+// SPREAD: every CTA writes its own slice of the selection (a.spread).
+template <bool SPREAD>
 __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
 {
     __shared__ Shared sh;
@@ -173,8 +231,35 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         uint2* cu = a.cand + u * a.cap;
         for (uint32_t i = tid; i < nl; i += kThreads)
             if (base + i < (uint32_t)a.cap) cu[base + i] = scand[i];
+        if (SPREAD && fits) {
+            // Keys of this slice in or above d0, from its bitmap words (written above).
+            __syncthreads();
+            const int words = (a.N + 31) / 32, w = r * (kSliceKeys / 32) + 2 * tid;
+            const uint32_t my_ge = (w < words ? __popc(__ldcg(bm + w)) : 0) + (w + 1 < words ? __popc(__ldcg(bm + w + 1)) : 0);
+            uint32_t ge_total;
+            block_exclusive_scan(my_ge, sh.warp_sums, ge_total);
+            if (tid == 0) a.info[u * a.info_stride + r] = ge_total;
+        }
         // ---- the unit's last CTA to get here selects.
-        if (!cta_ticket(a.done + u, (uint32_t)(a.C - 1), sh.last)) return;
+        if (!cta_ticket(a.done + u, (uint32_t)(a.C - 1), sh.last)) {
+            if (!(SPREAD && fits)) return;
+            // Wait (bounded) for the last CTA's slots, then write this slice.
+            if (tid == 0) {
+                bool got = false;
+                for (uint32_t polls = 0; polls < a.max_polls; ++polls) {
+                    if (ld_acquire_u32(a.done + u) & kPublished) {
+                        got = true;
+                        break;
+                    }
+                    __nanosleep(128);
+                }
+                sh.base = got ? __ldcg(a.info + u * a.info_stride + a.C + r) : 0xffffffffu;
+                if (!got) atomicOr(a.err_word, SOCKET_DEVERR_SELECT_TIMEOUT);
+            }
+            __syncthreads();
+            if (sh.base != 0xffffffffu) write_slice(a, u, r, sh.base, sh);
+            return;
+        }
     }
 
     int32_t* out = a.idx_out + u * (int64_t)a.k;
@@ -208,7 +293,7 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     };
     const int nc = (int)ncand;
     if (!single) {
-        load_tile(0);
+        if (!SPREAD) load_tile(0);
         // ---- the unit's candidates in shared memory.
         const uint2* cu = a.cand + u * a.cap;
         for (int i = tid; i < nc; i += kThreads) scand[i] = __ldcg(cu + i);
@@ -278,6 +363,36 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         }
     }
 
+    if constexpr (SPREAD) {
+        // The dropped candidates' bits cleared in the unit's bitmap, counted
+        // per slice; each slice's first slot; the flag; then this slice.
+        uint32_t* dropped = sh.hist;  // [C] (the radix bins are free again)
+        __syncthreads();
+        for (int i = tid; i < a.C; i += kThreads) dropped[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < nc; i += kThreads) {
+            const uint2 e = scand[i];
+            if (!e.y) {
+                atomicAnd(bm + (e.x >> 5), ~(1u << (e.x & 31)));
+                atomicAdd(&dropped[e.x / (uint32_t)kSliceKeys], 1u);
+            }
+        }
+        __syncthreads();
+        uint32_t mine = 0;
+        if (tid < a.C) mine = __ldcg(a.info + u * a.info_stride + tid) - dropped[tid];
+        uint32_t total;
+        const uint32_t slot = block_exclusive_scan(mine, sh.warp_sums, total);
+        if (tid < a.C) a.info[u * a.info_stride + a.C + tid] = slot;
+        if (tid == r) sh.base = slot;
+        __syncthreads();  // the bits and the slots precede the release below
+        if (tid == 0) {
+            __threadfence();
+            atomicOr(a.done + u, kPublished);
+        }
+        write_slice(a, u, r, sh.base, sh);
+        return;
+    }
+
     // ---- selected keys in index order, tile by tile of the bitmap: the
     // tile's words in shared memory, the candidates that are not selected
     // cleared there, then each thread's run of consecutive words written out
@@ -330,13 +445,15 @@ int topk_candidate_capacity(int64_t Ncap) { return (int)min64(Ncap, (int64_t)kTo
 
 int64_t topk_bitmap_stride(int64_t Ncap) { return (Ncap / 32 + 3) / 4 * 4; }
 
+int64_t topk_info_stride(int64_t Ncap) { return 2 * ((Ncap + kSliceKeys - 1) / kSliceKeys); }
+
 namespace {
 int topk_smem_bytes(int cap) { return (int)sizeof(uint2) * cap + 4 * kTileWords; }
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t* cand_cnt, uint2* cand,
-                        uint32_t* bitmap, uint32_t* done, const DecodeShape& s, int32_t* idx_out,
-                        cudaStream_t stream)
+                        uint32_t* bitmap, uint32_t* done, uint32_t* info, uint32_t* err_word, const DecodeShape& s,
+                        int32_t* idx_out, cudaStream_t stream)
 {
     TopkArgs a;
     a.scores = scores;
@@ -352,10 +469,19 @@ cudaError_t launch_topk(const float* scores, const uint32_t* unit_hist, uint32_t
     a.k = s.k;
     a.C = (int)((s.N + kSliceKeys - 1) / kSliceKeys);
     a.cap = topk_candidate_capacity(s.Ncap);
-    cudaError_t e = set_smem_limit_once((const void*)topk_kernel, topk_smem_bytes(kTopkCandidates));
+    a.info = info;
+    a.err_word = err_word;
+    a.info_stride = topk_info_stride(s.Ncap);
+    a.max_polls = wait_poll_limit();
+    // Every CTA writes its own slice when a unit has many slices (one CTA
+    // compacting a long bitmap is slow; with a few slices, CTAs that exit
+    // after their ticket free their SMs sooner, which pays more) and the
+    // grid (two CTAs per SM) is resident at once.
+    a.spread = a.C >= kSpreadMinSlices && a.C <= kSpreadMaxSlices && s.U * a.C <= 2 * (int64_t)device_num_sms() ? 1 : 0;
+    auto kern = a.spread ? topk_kernel<true> : topk_kernel<false>;
+    cudaError_t e = set_smem_limit_once((const void*)kern, topk_smem_bytes(kTopkCandidates));
     if (e != cudaSuccess) return e;
-    return launch_pdl(topk_kernel, dim3((unsigned)(s.U * a.C)), dim3(kThreads), (size_t)topk_smem_bytes(a.cap),
-                      stream, a);
+    return launch_pdl(kern, dim3((unsigned)(s.U * a.C)), dim3(kThreads), (size_t)topk_smem_bytes(a.cap), stream, a);
 }
 
 }  // namespace socket_attn

@@ -35,6 +35,13 @@ CASES = {
                  True, False),
     "all_ties_over_capacity": (wl.Workload(name="paths_e", B=1, Hq=4, Hkv=2, N=12000, L=5, P=8, tau=0.3, k=700,
                                            seed=7305), False, True),
+    # Many 32K-key slices per unit: the top-k CTAs of the separate path write
+    # their own slices of the selection (candidates, and a threshold bin over
+    # the candidate capacity).
+    "many_slices_spread": (wl.Workload(name="paths_j", B=1, Hq=4, Hkv=2, N=300001, L=8, P=8, tau=0.3, k=1500,
+                                       seed=7310), False, False),
+    "many_slices_spread_all_ties": (wl.Workload(name="paths_k", B=1, Hq=4, Hkv=2, N=270000, L=5, P=8, tau=0.3,
+                                                k=900, seed=7311), False, True),
     # The one-kernel step (N <= 8192, L <= 32, small G * L).
     "one_kernel_tiny_f32": (wl.TINY, False, False),
     "one_kernel_bf16_group4": (wl.Workload(name="paths_f", B=2, Hq=8, Hkv=2, N=6001, L=12, P=8, tau=0.3, k=500,
