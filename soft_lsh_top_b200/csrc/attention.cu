@@ -589,7 +589,11 @@ int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num
     const int chunk = wp ? kWChunk : attention_chunk_rows(kv_dtype);
     const int per_sm = wp ? kWCtasPerSm : 3;
     const int max_splits = (k + chunk - 1) / chunk;
-    const int64_t want = max64(1, (int64_t)per_sm * num_sms / U);
+    // At most kMaxSplits per unit: the unit's last CTA merges every split's
+    // partial, so with few units (a million-token sequence: 8) more splits
+    // cost more in the merge than they gain in gather parallelism.
+    constexpr int64_t kMaxSplits = 48;
+    const int64_t want = min64(kMaxSplits, max64(1, (int64_t)per_sm * num_sms / U));
     const int splits = (int)max64(1, min64(want, max_splits));
     const int rpc = attention_rows_per_cta(k, splits, chunk);
     return (k + rpc - 1) / rpc;
