@@ -367,7 +367,11 @@ const char* socket_last_error(void);
  * reads with cudaEventElapsedTime; the library only records them.  Inside a
  * stream capture they are recorded as external event nodes.  Returns
  * SOCKET_EINVAL if n < 0, n > SOCKET_DECODE_KERNELS + 1, or a handle is NULL.
- * The kernels, in order: soft tables, scoring, top-k, attention.
+ * The kernels, in order: soft tables, scoring, top-k, attention.  When a
+ * shape runs fewer kernels (socket_set_selection_path), the events after the
+ * last one are recorded right after it: with the fused selection + attention
+ * kernel, events[3] and events[4] follow it; with the whole step in one
+ * kernel, events[1] .. events[4] follow that kernel.
  */
 #define SOCKET_DECODE_KERNELS 4
 int socket_set_step_events(void* const* events, int n);
