@@ -11,8 +11,8 @@ copies they have already issued to land, and return without results -- the
 path a real expiry takes.  Nothing here traps, faults or hangs: no wait is
 left on something that never arrives.
 
-The shape (N above the one-kernel step's limit, so that path, which has no
-bounded waits, is not taken) runs, by path: bf16 by shape -> soft tables,
+The shapes (N above the one-kernel step's limit, so that path, which has no
+bounded waits, is not taken) run, by path: bf16 by shape -> soft tables,
 scoring, fused selection + attention; bf16 forced separate and fp32 ->
 soft tables, scoring, top-k, attention.
 """
@@ -33,18 +33,26 @@ def _bits(t):
     return t.view(torch.int32) if t.dtype == torch.float32 else t
 
 
-@pytest.mark.parametrize("dtype,path", [("bf16", "auto"), ("bf16", "separate"), ("f32", "auto")])
-def test_expired_waits_are_reported_and_the_context_stays_usable(dtype, path):
-    w = wl.Workload(name="expiry", B=1, Hq=4, Hkv=2, N=9000, L=8, P=8, tau=0.4, k=300, dtype=dtype, seed=7100)
+@pytest.mark.parametrize("dtype,path,N", [("bf16", "auto", 9000), ("bf16", "separate", 9000), ("f32", "auto", 9000),
+                                          ("bf16", "separate", 9 * 32768 + 5)])
+def test_expired_waits_are_reported_and_the_context_stays_usable(dtype, path, N):
+    """The last case has nine 32K-key top-k slices per unit: each slice CTA
+    waits for the unit's output slots (SELECT) before writing its part."""
+    w = wl.Workload(name="expiry", B=1, Hq=4, Hkv=2, N=N, L=8, P=8, tau=0.4, k=300, dtype=dtype, seed=7100)
     mode = sk.SOCKET_PATH_AUTO if path == "auto" else sk.SOCKET_PATH_SEPARATE
     before = sk.socket_set_selection_path(mode)
     try:
-        _expire_and_recover(w, dtype, fused=(dtype == "bf16" and path == "auto"))
+        want = [GATHER]
+        if dtype == "bf16" and path == "auto":
+            want = [SELECT]  # the fused kernel's slices wait for the unit's threshold
+        elif N > 8 * 32768:
+            want = [GATHER, SELECT]
+        _expire_and_recover(w, dtype, want)
     finally:
         sk.socket_set_selection_path(before)
 
 
-def _expire_and_recover(w, dtype, fused):
+def _expire_and_recover(w, dtype, want):
     inp = wl.make_inputs(w, DEV)
     ids, vnorm = gpu_hash(inp, w)
     ws, idx, out = sk.alloc_decode_buffers(w.B, w.Hq, w.Hkv, w.ncap, w.L, w.P, w.k, DEV)
@@ -65,9 +73,11 @@ def _expire_and_recover(w, dtype, fused):
     finally:
         sk.socket_set_wait_limit(previous)
     assert err & TABLE, hex(err)
-    # The fused kernel's slices wait for the unit's threshold; the attention
-    # kernel's row gathers wait for their copies.
-    assert err & (SELECT if fused else GATHER), hex(err)
+    # The attention kernel's row gathers wait for their copies; the fused
+    # kernel's slices, and the slices of a unit with many top-k slices, wait
+    # for the unit's last CTA.
+    for bit in want:
+        assert err & bit, hex(err)
 
     idx.fill_(-1)
     out.fill_(float("nan"))
