@@ -493,19 +493,39 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
         if (ch == 0) a.part_ml[p] = make_float2(M, l);
     }
     if (!cta_ticket(a.tickets + u, (uint32_t)(a.C - 1), sh.last)) return;
-    // The unit's output: the C slice partials merged per head in slice order.
+    // The unit's output: the C slice partials merged per head in slice order,
+    // 16 slices at a time with all their loads in flight, and a running
+    // maximum rescaling the tiles already summed.
+    constexpr int kMergeTile = 16;
     for (int e = tid; e < G * kHeadDim; e += kThreads) {
         const int h = e / kHeadDim, ch = e % kHeadDim;
         const float2* pml = a.part_ml + (qrow0 + h) * a.C;
         const float* po = a.part_o + (qrow0 + h) * a.C * kHeadDim + ch;
-        float M = -INFINITY;
-        for (int s2 = 0; s2 < a.C; ++s2) M = fmaxf(M, __ldcg(pml + s2).x);
-        float o = 0.0f, l = 0.0f;
-        for (int s2 = 0; s2 < a.C; ++s2) {
-            const float2 ml = __ldcg(pml + s2);
-            const float wt = ml.x == -INFINITY ? 0.0f : expf(ml.x - M);
-            o += wt * __ldcg(po + (int64_t)s2 * kHeadDim);
-            l += wt * ml.y;
+        float M = -INFINITY, o = 0.0f, l = 0.0f;
+        for (int s0 = 0; s0 < a.C; s0 += kMergeTile) {
+            float2 ml[kMergeTile];
+            float ov[kMergeTile];
+#pragma unroll
+            for (int j = 0; j < kMergeTile; ++j) {
+                const bool in = s0 + j < a.C;
+                ml[j] = in ? __ldcg(pml + s0 + j) : make_float2(-INFINITY, 0.0f);
+                ov[j] = in ? __ldcg(po + (int64_t)(s0 + j) * kHeadDim) : 0.0f;
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kMergeTile; ++j) mt = fmaxf(mt, ml[j].x);
+            const float Mn = fmaxf(M, mt);
+            if (Mn == -INFINITY) continue;
+            const float sc = M == -INFINITY ? 0.0f : expf(M - Mn);
+            o *= sc;
+            l *= sc;
+#pragma unroll
+            for (int j = 0; j < kMergeTile; ++j) {
+                const float wt = ml[j].x == -INFINITY ? 0.0f : expf(ml[j].x - Mn);
+                o += wt * ov[j];
+                l += wt * ml[j].y;
+            }
+            M = Mn;
         }
         a.out[(qrow0 + h) * kHeadDim + ch] = l > 0.0f ? o / l : 0.0f;
     }
