@@ -18,7 +18,6 @@ namespace socket_attn {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTpb = 4;                    // tables per CTA
 constexpr int kMaxGroup = 16;
 constexpr int kMaxP = 8;
 constexpr int kTpr = 8;                    // threads per hyperplane row (16 channels each)
@@ -52,16 +51,19 @@ constexpr int kKeySlots = 16;              // appended keys projected per pass g
 
 // Dynamic shared memory of a CTA for group size G, with `slots` rows for
 // appended keys.
-__host__ __device__ constexpr int smem_bytes(int G, int slots)
+__host__ __device__ constexpr int smem_bytes(int G, int slots, int tpb)
 {
     return (G + slots) * kTpr * kQSeg * 8         // query rows, then key rows (fp64), padded channel slices
            + G * 8                                // per-head factor 2 / (tau ||q_h||)
-           + G * kTpb * kMaxP * 2 * 8             // per-plane sigmoid pairs
-           + G * kTpb * 2 * 16 * 8;               // nibble tables
+           + G * tpb * kMaxP * 2 * 8              // per-plane sigmoid pairs
+           + G * tpb * 2 * 16 * 8;                // nibble tables
 }
 
-// Grid: (U, 8 * ceil(L / 32)); CTA y covers tables 4y .. 4y + 3 (the ones
-// >= L are written as zero columns).  Block: kThreads.  Many small CTAs keep
+// Grid: (U, 32 / TPB * ceil(L / 32)); CTA y covers tables TPB y .. TPB y +
+// TPB - 1 (the ones >= L are written as zero columns).  TPB = 4, or 8 for
+// per-head tables when the grid would need several waves: a thread then takes
+// two hyperplane rows, one after the other, and the CTAs (each a chain of
+// short dependent phases) are half as many.  Block: kThreads.  Many small CTAs keep
 // every step's dependent chain short and enough warps resident to hide it.
 //   1. the unit's G query rows are widened to float64 in shared memory, with
 //      their norms; each thread holds 16 channels of one hyperplane row
@@ -78,13 +80,16 @@ __host__ __device__ constexpr int smem_bytes(int G, int slots)
 //      of row b of the expanded layout the scoring kernel copies into shared
 //      memory: per 32-table block c a [bucket][64] row whose column j holds
 //      table 32c + j mod 32.
-template <typename QT>
+template <typename QT, int TPB>
 __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
     const QT* __restrict__ q, const uint16_t* __restrict__ W, int G, int L, int P, double tau,
     const AppendHash app, int64_t Ncap, int share, bool sep, float* __restrict__ tables,
     uint32_t* __restrict__ err_word, uint32_t* __restrict__ counters, uint32_t* __restrict__ topk_done,
     uint32_t* __restrict__ unit_hist, uint32_t* __restrict__ cand_cnt)
 {
+    static_assert(TPB == 4 || TPB == 8, "four or eight tables per CTA");
+    constexpr int kTpb = TPB;
+    constexpr int kRowPasses = TPB * kMaxP / (kThreads / kTpr);  // hyperplane rows per thread, at most
     __shared__ uint32_t aid[kMaxAppend][kTpb];  // ids of the appended keys (bit p <-> plane p)
     extern __shared__ __align__(16) char st_dyn[];
     // Keys appended in this step are hashed here too (step 1 of the method,
@@ -146,16 +151,21 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
     }
 
     if (nt > 0) {
-        // This thread's slice of its hyperplane row (loaded before the query
-        // is staged, so both loads are in flight together).
-        const int r = tid / kTpr, part = tid % kTpr;
+        // This thread's slices of its hyperplane rows (pass rp: row tid / 8 +
+        // 32 rp), loaded before the query is staged, so all the loads are in
+        // flight together.
+        const int part = tid % kTpr;
         const int wrows = nt * P;
-        const bool live = r < wrows;
-        uint4 w2[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        if (live) {
-            const uint4* wsrc = reinterpret_cast<const uint4*>(W + ((int64_t)l0 * P + r) * kHeadDim + kChan * part);
-            w2[0] = __ldg(wsrc);
-            w2[1] = __ldg(wsrc + 1);
+        uint4 w2[kRowPasses][2];
+#pragma unroll
+        for (int rp = 0; rp < kRowPasses; ++rp) {
+            const int r = tid / kTpr + rp * (kThreads / kTpr);
+            w2[rp][0] = w2[rp][1] = make_uint4(0, 0, 0, 0);
+            if (r < wrows) {
+                const uint4* wsrc = reinterpret_cast<const uint4*>(W + ((int64_t)l0 * P + r) * kHeadDim + kChan * part);
+                w2[rp][0] = __ldg(wsrc);
+                w2[rp][1] = __ldg(wsrc + 1);
+            }
         }
         // The unit's G query rows in 16-byte pieces (8 bf16 or 4 fp32 each).
         constexpr int kPer16 = 16 / (int)sizeof(QT);
@@ -194,86 +204,48 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
             for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(kFullMask, s, o);
             if (lane == 0) qscale[h] = (s > 0.0 && tau > 0.0) ? 2.0 / (tau * sqrt(s)) : 0.0;
         }
-        double wd[kChan];  // this thread's 16 channels of the row, widened once
-        {
-            const uint32_t words[8] = {w2[0].x, w2[0].y, w2[0].z, w2[0].w, w2[1].x, w2[1].y, w2[1].z, w2[1].w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                wd[2 * i] = bf16_bits_to_f64(words[i] & 0xffffu);
-                wd[2 * i + 1] = bf16_bits_to_f64(words[i] >> 16);
+#pragma unroll 1
+        for (int rp = 0; rp < kRowPasses; ++rp) {
+            if (rp * (kThreads / kTpr) >= wrows) break;  // no row of this pass is live (CTA-uniform)
+            const int r = tid / kTpr + rp * (kThreads / kTpr);
+            const bool live = r < wrows;
+            if (rp > 0 && nk_all > kKeySlots) {
+                // The first appended keys again (later ones took their rows).
+                __syncthreads();
+                stage_keys(0, nk0);
             }
-        }
-        __syncthreads();
-
-        // Rows 0 .. G-1 of qd are the queries, rows G .. G + nk0 - 1 the first
-        // appended keys: bit p of a key's id in table l is [<W_{l,p}, k> > 0].
-        const int lt = live ? r / P : 0, p = live ? r - lt * P : 0;
-        const int Ht = G + nk0;
-        for (int h0 = 0; h0 < Ht; h0 += kHeadsPerPass) {
-            double acc[kHeadsPerPass];
+            double wd[kChan];  // this thread's 16 channels of the row, widened once
+            {
+                const uint32_t words[8] = {w2[rp][0].x, w2[rp][0].y, w2[rp][0].z, w2[rp][0].w,
+                                           w2[rp][1].x, w2[rp][1].y, w2[rp][1].z, w2[rp][1].w};
 #pragma unroll
-            for (int hh = 0; hh < kHeadsPerPass; ++hh) {
-                double a0 = 0.0, a1 = 0.0;
-                if (h0 + hh < Ht) {
-                    const double* qh = &QD(h0 + hh, kChan * part);
-#pragma unroll
-                    for (int i = 0; i < kChan; i += 2) {
-                        const double2 qv2 = *reinterpret_cast<const double2*>(qh + i);
-                        a0 = fma(wd[i], qv2.x, a0);
-                        a1 = fma(wd[i + 1], qv2.y, a1);
-                    }
-                }
-                acc[hh] = a0 + a1;
-            }
-            // Sum the row's eight slices; thread hh of the row finishes head h0 + hh.
-#pragma unroll
-            for (int hh = 0; hh < kHeadsPerPass; ++hh) {
-                acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 1);
-                acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 2);
-                acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 4);
-            }
-            const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
-            const int h = h0 + part;
-            if (live && part < kHeadsPerPass && h >= G && h < Ht) {
-                if (y > 0.0) atomicOr(&aid[h - G][lt], 1u << p);
-            } else if (live && part < kHeadsPerPass && h < G) {
-                if (tau == 0.0) {
-                    // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
-                    SIG(h, lt, p, 1) = y > 0.0 ? 1.0 : 0.0;
-                    SIG(h, lt, p, 0) = y > 0.0 ? 0.0 : 1.0;
-                } else {
-                    // sigmoid(+-x) from one exponential: e = exp(-|x|),
-                    // sigmoid(|x|) = 1 / (1 + e), sigmoid(-|x|) = e / (1 + e).
-                    const double x = y * qscale[h];
-                    const double e = exp(-fabs(x));
-                    const double big = 1.0 / (1.0 + e), small = e * big;
-                    SIG(h, lt, p, 1) = x >= 0.0 ? big : small;  // sign +1: bit set
-                    SIG(h, lt, p, 0) = x >= 0.0 ? small : big;  // sign -1: bit clear
+                for (int i = 0; i < 8; ++i) {
+                    wd[2 * i] = bf16_bits_to_f64(words[i] & 0xffffu);
+                    wd[2 * i + 1] = bf16_bits_to_f64(words[i] >> 16);
                 }
             }
-        }
-        // Any further appended keys, kKeySlots at a time, on the same rows.
-        for (int k0 = kKeySlots; k0 < nk_all; k0 += kKeySlots) {
-            const int nk = min(kKeySlots, nk_all - k0);
-            __syncthreads();  // the previous keys' rows have been read
-            stage_keys(k0, nk);
             __syncthreads();
-            for (int h0 = 0; h0 < nk; h0 += kHeadsPerPass) {
+            // Rows 0 .. G-1 of qd are the queries, rows G .. G + nk0 - 1 the first
+            // appended keys: bit p of a key's id in table l is [<W_{l,p}, k> > 0].
+            const int lt = live ? r / P : 0, p = live ? r - lt * P : 0;
+            const int Ht = G + nk0;
+            for (int h0 = 0; h0 < Ht; h0 += kHeadsPerPass) {
                 double acc[kHeadsPerPass];
 #pragma unroll
                 for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                     double a0 = 0.0, a1 = 0.0;
-                    if (h0 + hh < nk) {
-                        const double* kh = &QD(G + h0 + hh, kChan * part);
+                    if (h0 + hh < Ht) {
+                        const double* qh = &QD(h0 + hh, kChan * part);
 #pragma unroll
                         for (int i = 0; i < kChan; i += 2) {
-                            const double2 kv2 = *reinterpret_cast<const double2*>(kh + i);
-                            a0 = fma(wd[i], kv2.x, a0);
-                            a1 = fma(wd[i + 1], kv2.y, a1);
+                            const double2 qv2 = *reinterpret_cast<const double2*>(qh + i);
+                            a0 = fma(wd[i], qv2.x, a0);
+                            a1 = fma(wd[i + 1], qv2.y, a1);
                         }
                     }
                     acc[hh] = a0 + a1;
                 }
+                // Sum the row's eight slices; thread hh of the row finishes head h0 + hh.
 #pragma unroll
                 for (int hh = 0; hh < kHeadsPerPass; ++hh) {
                     acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 1);
@@ -281,8 +253,57 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
                     acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 4);
                 }
                 const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
-                if (live && part < kHeadsPerPass && h0 + part < nk && y > 0.0)
-                    atomicOr(&aid[k0 + h0 + part][lt], 1u << p);
+                const int h = h0 + part;
+                if (live && part < kHeadsPerPass && h >= G && h < Ht) {
+                    if (y > 0.0) atomicOr(&aid[h - G][lt], 1u << p);
+                } else if (live && part < kHeadsPerPass && h < G) {
+                    if (tau == 0.0) {
+                        // Hard LSH: the plane's bit is [<W_{l,p}, q_h> > 0], as for keys.
+                        SIG(h, lt, p, 1) = y > 0.0 ? 1.0 : 0.0;
+                        SIG(h, lt, p, 0) = y > 0.0 ? 0.0 : 1.0;
+                    } else {
+                        // sigmoid(+-x) from one exponential: e = exp(-|x|),
+                        // sigmoid(|x|) = 1 / (1 + e), sigmoid(-|x|) = e / (1 + e).
+                        const double x = y * qscale[h];
+                        const double e = exp(-fabs(x));
+                        const double big = 1.0 / (1.0 + e), small = e * big;
+                        SIG(h, lt, p, 1) = x >= 0.0 ? big : small;  // sign +1: bit set
+                        SIG(h, lt, p, 0) = x >= 0.0 ? small : big;  // sign -1: bit clear
+                    }
+                }
+            }
+            // Any further appended keys, kKeySlots at a time, on the same rows.
+            for (int k0 = kKeySlots; k0 < nk_all; k0 += kKeySlots) {
+                const int nk = min(kKeySlots, nk_all - k0);
+                __syncthreads();  // the previous keys' rows have been read
+                stage_keys(k0, nk);
+                __syncthreads();
+                for (int h0 = 0; h0 < nk; h0 += kHeadsPerPass) {
+                    double acc[kHeadsPerPass];
+#pragma unroll
+                    for (int hh = 0; hh < kHeadsPerPass; ++hh) {
+                        double a0 = 0.0, a1 = 0.0;
+                        if (h0 + hh < nk) {
+                            const double* kh = &QD(G + h0 + hh, kChan * part);
+#pragma unroll
+                            for (int i = 0; i < kChan; i += 2) {
+                                const double2 kv2 = *reinterpret_cast<const double2*>(kh + i);
+                                a0 = fma(wd[i], kv2.x, a0);
+                                a1 = fma(wd[i + 1], kv2.y, a1);
+                            }
+                        }
+                        acc[hh] = a0 + a1;
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < kHeadsPerPass; ++hh) {
+                        acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 1);
+                        acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 2);
+                        acc[hh] += __shfl_xor_sync(kFullMask, acc[hh], 4);
+                    }
+                    const double y = part == 0 ? acc[0] : part == 1 ? acc[1] : part == 2 ? acc[2] : acc[3];
+                    if (live && part < kHeadsPerPass && h0 + part < nk && y > 0.0)
+                        atomicOr(&aid[k0 + h0 + part][lt], 1u << p);
+                }
             }
         }
         __syncthreads();
@@ -290,7 +311,7 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
         // Nibble tables: lo over planes 0..min(P,4)-1, hi over planes 4..P-1.
         const int plo = min(P, 4);
         for (int e = tid; e < G * kTpb * 32; e += kThreads) {
-            const int h = e >> 7, t = (e >> 5) & (kTpb - 1), hi = (e >> 4) & 1, v = e & 15;
+            const int h = e / (kTpb * 32), t = (e >> 5) % kTpb, hi = (e >> 4) & 1, v = e & 15;
             if (t >= nt) continue;
             double prod = 1.0;
             const int p0 = hi ? 4 : 0, p1 = hi ? P : plo;
@@ -340,9 +361,12 @@ __global__ __launch_bounds__(kThreads, 4) void soft_tables_kernel(
         }
         float* tu = tables + (unit0 + hs) * nblk * (int64_t)NB * 64;
         float* row = tu + ((int64_t)(l0 >> 5) * NB + bucket) * 64 + (l0 & 31);
-        const float4 a = make_float4(vals[0], vals[1], vals[2], vals[3]);
-        *reinterpret_cast<float4*>(row) = a;
-        *reinterpret_cast<float4*>(row + 32) = a;
+#pragma unroll
+        for (int t4 = 0; t4 < kTpb; t4 += 4) {
+            const float4 a = make_float4(vals[t4], vals[t4 + 1], vals[t4 + 2], vals[t4 + 3]);
+            *reinterpret_cast<float4*>(row + t4) = a;
+            *reinterpret_cast<float4*>(row + t4 + 32) = a;
+        }
     }
 
     // The appended keys' id slots of this CTA's four tables (0 for tables
@@ -390,20 +414,30 @@ cudaError_t launch_soft_tables(const void* q, int q_dtype, const uint16_t* W, co
     const int G = sep ? s.share : s.G;
     const int share = sep ? 1 : s.share;
     const int64_t ctas = sep ? s.U / s.share : s.U;
-    const int smem = smem_bytes(G, app.end > app.begin ? kKeySlots : 0);
-    const dim3 grid((unsigned)ctas, (unsigned)(32 / kTpb * ((s.L + 31) / 32)));
-    if (q_dtype == 1) {
-        cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<uint16_t>, smem_bytes(kMaxGroup, kKeySlots));
-        if (e != cudaSuccess) return e;
-        return launch_pdl(soft_tables_kernel<uint16_t>, grid, dim3(kThreads), (size_t)smem, stream,
-                          static_cast<const uint16_t*>(q), W, G, s.L, s.P, tau, app, s.Ncap, share, sep,
-                          tables, err_word, counters, topk_done, unit_hist, cand_cnt);
+    // Four tables per CTA; eight for per-head tables when four would need
+    // several waves (there each CTA writes all its heads' tables, and halving
+    // the CTAs pays; for grouped tables it measured slower).
+    const int nblk = (s.L + 31) / 32;
+    const int tpb = sep && ctas * 8 * nblk > 4 * (int64_t)device_num_sms() ? 8 : 4;
+    const int slots = app.end > app.begin ? kKeySlots : 0;
+    const int smem = smem_bytes(G, slots, tpb);
+    const dim3 grid((unsigned)ctas, (unsigned)(32 / tpb * nblk));
+#define SOCKET_ST_CASE(QTT, TPBV)                                                                              \
+    {                                                                                                          \
+        cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<QTT, TPBV>,                        \
+                                            smem_bytes(kMaxGroup, kKeySlots, TPBV));                           \
+        if (e != cudaSuccess) return e;                                                                        \
+        return launch_pdl(soft_tables_kernel<QTT, TPBV>, grid, dim3(kThreads), (size_t)smem, stream,          \
+                          static_cast<const QTT*>(q), W, G, s.L, s.P, tau, app, s.Ncap, share, sep, tables,    \
+                          err_word, counters, topk_done, unit_hist, cand_cnt);                                 \
     }
-    cudaError_t e = set_smem_limit_once((const void*)soft_tables_kernel<float>, smem_bytes(kMaxGroup, kKeySlots));
-    if (e != cudaSuccess) return e;
-    return launch_pdl(soft_tables_kernel<float>, grid, dim3(kThreads), (size_t)smem, stream,
-                      static_cast<const float*>(q), W, G, s.L, s.P, tau, app, s.Ncap, share, sep, tables,
-                      err_word, counters, topk_done, unit_hist, cand_cnt);
+    if (q_dtype == 1) {
+        if (tpb == 8) SOCKET_ST_CASE(uint16_t, 8)
+        SOCKET_ST_CASE(uint16_t, 4)
+    }
+    if (tpb == 8) SOCKET_ST_CASE(float, 8)
+    SOCKET_ST_CASE(float, 4)
+#undef SOCKET_ST_CASE
 }
 
 }  // namespace socket_attn

@@ -91,15 +91,22 @@ def test_hash_in_ranges_matches_oracle(case):
                orc_ids, orc_vn, margin, 0, w.N)
 
 
+# Many units with more appended keys than one projection pass holds.
+APPEND_EXTRA = {
+    "many_units_l32": wl.Workload(name="append_many", B=80, Hq=2, Hkv=1, N=2100, L=32, P=8, tau=0.3, k=64,
+                                  seed=7401),
+}
+
+
 @pytest.mark.parametrize("case", ["bf16_single_head", "odd_group3_p5", "f32_group2_p6", "bf16_l80_p7",
-                                  "bf16_group16"])
+                                  "bf16_group16", "many_units_l32"])
 def test_decode_append_hashes_and_decodes(case):
     """socket_decode_append: the step hashes the keys just appended (1, 5, then
     33 keys, so chunk boundaries are crossed) and decodes over them.  The ids
     and norms of every key match the oracle's hash (within the float32
     exemption band), and each step's scores, selection and output match the
     oracle run on the index the step saw."""
-    w = SMALL[case]
+    w = SMALL[case] if case in SMALL else APPEND_EXTRA[case]
     inp = wl.make_inputs(w, DEV)
     B = inp["K"].shape[0]
     ids, vnorm = sk.alloc_cache_index(B, w.Hkv, w.ncap, w.L, DEV)
@@ -323,6 +330,19 @@ def test_batch8_128k_per_head_sampled_units_and_needles():
     check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, per_head=True)
     del inp
     torch.cuda.empty_cache()
+
+
+def test_per_head_many_kv_units_sampled():
+    """Per-head selection over enough kv units that the soft-table kernel
+    takes eight tables per CTA (each CTA writes its kv unit's four heads'
+    tables, two hyperplane rows per thread): sampled kv units, head by head,
+    against the oracle."""
+    w = wl.Workload(name="ph_many", B=80, Hq=4, Hkv=1, N=2100, L=32, P=8, tau=0.3, k=64, seed=7402)
+    units = [0, 37, 79]
+    inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
+    substitute_units(ids, vnorm, w, units, orc_ids, orc_vn32)
+    idx, out, sc = gpu_decode(inp, w, ids, vnorm, per_head=True)
+    check_decode(inp, w, orc_ids, orc_vn32, units, idx, out, sc, per_head=True)
 
 
 def test_million_token_sampled_units():
