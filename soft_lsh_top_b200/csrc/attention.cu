@@ -329,8 +329,10 @@ __global__ __launch_bounds__(kThreads) void attention_kernel(
 // ---------------------------------------------------------------------------
 // bfloat16 K/V and q, G <= 8: flash-decode split-K with every warp on its own
 // 16-key chunks and both contractions on the tensor cores (WarpAttn, in
-// warp_attn.cuh).  Each warp gathers its chunks itself on its own two-stage
-// ring of mbarriers: the chunk loop has no CTA-wide barrier.  The two warps
+// warp_attn.cuh).  Each warp gathers its chunks itself (16-byte cp.async
+// copies, each lane's completion arriving on the stage's mbarrier) on its own
+// two-stage ring, so the chunk loop has no CTA-wide barrier and every wait is
+// a bounded mbarrier wait.  The two warps
 // of a CTA then merge in shared memory and the last CTA of the unit merges
 // the CTAs' partials.
 // ---------------------------------------------------------------------------
@@ -431,8 +433,9 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     WarpAttn<G> at;
     at.init(q, qrow0);
     if (tid == 0) {
+        // One arrival per lane and chunk (issue_lsu_mbar).
         for (int w = 0; w < kWWarps; ++w)
-            for (int st = 0; st < kWStages; ++st) mbar_init(&bar[w][st], 1);
+            for (int st = 0; st < kWStages; ++st) mbar_init(&bar[w][st], 32);
         fence_mbarrier_init();
     }
     __syncthreads();
@@ -460,7 +463,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
         const int r0 = r_begin + (warp + kWWarps * j) * kWChunk;
         const int nr = min(kWChunk, r_end - r0);
         r = (r >= 0 && r < Ncap) ? r : 0;
-        at.issue(wsm_base + st * kWStageBytes, K, V, ukv * Ncap + r, nr, &bar[warp][st]);
+        at.issue_lsu_mbar(wsm_base + st * kWStageBytes, K, V, ukv * Ncap + r, nr, &bar[warp][st]);
     };
     if (cw > 0) issue(0, 0, row_index(0));
     if (cw > 1) issue(1, 1, row_index(1));

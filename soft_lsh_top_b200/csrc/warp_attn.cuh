@@ -18,9 +18,12 @@
 // "SOCKET: SOft Collision Kernel EsTimator for Sparse Attention", "Auswahl").
 //
 // A chunk's rows are gathered by the warp itself into one stage of shared
-// memory: one bulk copy per 256-byte key or value row, into rows padded to
-// 272 bytes so an ldmatrix phase's 8 rows hit distinct banks, completion
-// counted on the stage's mbarrier.
+// memory, into rows padded to 272 bytes so an ldmatrix phase's 8 rows hit
+// distinct banks: 16-byte cp.async copies, completion counted on the stage's
+// mbarrier (issue_lsu_mbar) or in a commit group (issue_lsu), or one bulk
+// copy per 256-byte key or value row (issue).  The cp.async copies cost the
+// copy engine nothing per row, which pays where an SM gathers thousands of
+// rows.
 #pragma once
 
 #include "common.cuh"
@@ -143,6 +146,27 @@ struct WarpAttn {
             cp_async16_zfill(s0 + (uint32_t)(rr * kWRowStride + (lane & 15) * 16), src, kr < nr ? 16u : 0u);
         }
         cp_async_commit();
+    }
+
+    // The same copies as issue_lsu, with their completion counted on `bar`
+    // instead of in a commit group: each lane's arrival (cp.async.mbarrier.
+    // arrive.noinc) lands once its own copies have, so `bar` must expect 32
+    // arrivals per phase (mbar_init(bar, 32)) and the chunk has landed when the
+    // phase completes; a wait on it can be bounded.
+    __device__ __forceinline__ void issue_lsu_mbar(char* stage, const uint16_t* __restrict__ K,
+                                                   const uint16_t* __restrict__ V, int64_t row, int nr, uint64_t* bar)
+    {
+        const int lane = threadIdx.x & 31;
+        const uint32_t s0 = smem_addr(stage);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int rr = 2 * i + (lane >> 4);  // stage row: 0-15 keys, 16-31 values
+            const int kr = rr & 15;
+            const int64_t rk = __shfl_sync(kFullMask, row, kr);
+            const uint16_t* src = (rr < 16 ? K : V) + rk * kHeadDim + (lane & 15) * 8;
+            cp_async16_zfill(s0 + (uint32_t)(rr * kWRowStride + (lane & 15) * 16), src, kr < nr ? 16u : 0u);
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
     }
 
     // Adds the chunk of nr rows that has landed in the stage at shared address
