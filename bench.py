@@ -175,6 +175,31 @@ def whole_job_rate(world: int, steps: int, ms_max: float) -> float:
     return world * steps / (ms_max * 1e-3)
 
 
+def step_kernel_times(evs, n: int, path: int) -> dict:
+    """Mean ms of each kernel of a decode step from the events the library
+    recorded around its kernels (socket_set_step_events), named after the
+    kernels the step's path launched (socket_last_decode_path)."""
+    import soft_lsh_top_b200 as sk
+
+    def gap(i):
+        return statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(n))
+    if path == sk.SOCKET_STEP_ONE_KERNEL:
+        return {"small_step": gap(0)}
+    if path == sk.SOCKET_STEP_FUSED:
+        return {"soft_tables": gap(0), "score": gap(1), "select_attend": gap(2)}
+    return {name: gap(i) for i, name in enumerate(["soft_tables", "score", "topk", "attention"])}
+
+
+def kernels_per_step(path: int, L: int) -> int:
+    """Library kernels one decode step launches on its path (the scoring stage
+    takes one launch per 64 tables)."""
+    import soft_lsh_top_b200 as sk
+
+    if path == sk.SOCKET_STEP_ONE_KERNEL:
+        return 1
+    return (2 if path == sk.SOCKET_STEP_FUSED else 3) + -(-L // 64)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -431,7 +456,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
     # library between the kernels, on the launching stream.  The events
     # serialise the kernels, so these are each kernel's own time.
     KD = min(K, 200)
-    nk = 4
+    nk = 4  # kernel slots of a step's events (socket_set_step_events)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(KD)]
     for row in evs:  # torch creates the CUDA event on first record
         for e in row:
@@ -442,9 +467,8 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         step(s)
     torch.cuda.synchronize()
     sk.socket_set_step_events([])
-    names = ["soft_tables", "score", "topk", "attention"]
-    kern_ms = {n: statistics.fmean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(KD))
-               for i, n in enumerate(names)}
+    path = sk.socket_last_decode_path()
+    kern_ms = step_kernel_times(evs, KD, path)
     assert sk.read_device_error(ws) == 0
 
     # ---- prefill: hashing a whole layer (socket_hash_keys), for the hash
@@ -495,8 +519,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         step_h(s)
     torch.cuda.synchronize()
     sk.socket_set_step_events([])
-    ph_kern = {n: statistics.fmean(evs_h[s][i].elapsed_time(evs_h[s][i + 1]) for s in range(KHD))
-               for i, n in enumerate(names)}
+    ph_kern = step_kernel_times(evs_h, KHD, sk.socket_last_decode_path())
     assert sk.read_device_error(ws_h) == 0
     del ws_h, idx_h, out_h, evs_h
     torch.cuda.empty_cache()
@@ -554,9 +577,8 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             fn(t)
         torch.cuda.synchronize()
         sk.socket_set_step_events([])
-        append[name]["decode_kernels_us"] = {n: 1e3 * statistics.fmean(ev_a[t][i].elapsed_time(ev_a[t][i + 1])
-                                                                       for t in range(wa.appends))
-                                             for i, n in enumerate(names)}
+        append[name]["decode_kernels_us"] = {
+            n: 1e3 * v for n, v in step_kernel_times(ev_a, wa.appends, sk.socket_last_decode_path()).items()}
     # Prefill of this workload (L * P = 480 hyperplanes: two tensor-core passes).
     h0.record()
     for _ in range(3):
@@ -636,9 +658,16 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         ms_step = ms_total / K
         bytes_step = w.step_bytes()
         peak, peak_src = hbm_peak()
-        score_bytes = w.U * w.N * (w.L + 4)
-        score_gbs = score_bytes / (kern_ms["score"] * 1e-3) / 1e9
+        # The dominant kernel: scoring (its ids and norms), or the one kernel
+        # of a small step (the whole step's bytes).
+        if "score" in kern_ms:
+            dom_kernel, dom_bytes, dom_ms = "score_kernel", w.U * w.N * (w.L + 4), kern_ms["score"]
+        else:
+            dom_kernel, dom_bytes, dom_ms = "small_step_kernel", bytes_step, kern_ms["small_step"]
+        dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
         attn_bytes = w.U * 2 * w.k * w.d * w.elem_bytes
+        # The gather kernel's own rate, where the step runs it on its own.
+        attn_gbs = attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9 if "attention" in kern_ms else None
         keys = w.U * w.N
         hash_bytes = keys * (2 * w.d * w.elem_bytes + sk.socket_ids_row_bytes(w.L) + 4)
         hash_flops = 2.0 * keys * w.d * w.L * w.P
@@ -659,7 +688,8 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         # Per-head scoring reads each kv unit's ids and norms once (its heads'
         # CTAs stream them side by side) and writes a score row per head.
         ph_score_bytes = w.U * w.N * (w.L + 4) + w.U * w.G * w.N * 4
-        ph_score_gbs = ph_score_bytes / (ph_kern["score"] * 1e-3) / 1e9
+        ph_score_ms = ph_kern.get("score", ph_kern.get("small_step"))
+        ph_score_gbs = ph_score_bytes / (ph_score_ms * 1e-3) / 1e9
         # Each (head, key, table) is one 4-byte shared-memory lookup: per head
         # that is the whole lookup stream, bound by the SMs' shared-memory
         # bandwidth (128 B per clock per SM) at the sampled SM clock.
@@ -668,7 +698,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
         smem_peak = n_sm * 128 * mhz * 1e6 / 1e9
         lookup_bytes = w.U * w.G * w.N * w.L * 4
-        lookup_gbs = lookup_bytes / (ph_kern["score"] * 1e-3) / 1e9
+        lookup_gbs = lookup_bytes / (ph_score_ms * 1e-3) / 1e9
         per_head = {
             "what": "socket_decode_per_head: one selection per query head (B*Hq units) on the same layers; "
                     "direct calls",
@@ -678,10 +708,12 @@ def run_socket(args, world: int, rank: int, local_rank: int):
                       "bound": "smem", "lookup_bytes": lookup_bytes, "achieved": lookup_gbs, "peak": smem_peak,
                       "unit": "GB/s", "frac": lookup_gbs / smem_peak,
                       "peak_source": f"derived: {n_sm} SMs x 128 B/clock x {mhz:.0f} MHz (sampled SM clock)"},
-            "attention_gbs": w.U * w.G * 2 * w.k * w.d * w.elem_bytes / (ph_kern["attention"] * 1e-3) / 1e9,
+            "attention_gbs": (w.U * w.G * 2 * w.k * w.d * w.elem_bytes / (ph_kern["attention"] * 1e-3) / 1e9
+                              if "attention" in ph_kern else None),
         }
-        traffic = profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
-                                                            "soft_lsh_top_b200/csrc/common.cuh"])
+        traffic = (profiled_traffic("score_kernel", w.name, ["soft_lsh_top_b200/csrc/score.cu",
+                                                             "soft_lsh_top_b200/csrc/common.cuh"])
+                   if dom_kernel == "score_kernel" else None)
         result = {
             "metric": METRIC, "value": whole_job_rate(world, K, ms_total), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -696,15 +728,16 @@ def run_socket(args, world: int, rank: int, local_rank: int):
             "step_hbm_gbs": bytes_step / (ms_step * 1e-3) / 1e9,
             "step_roofline_frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak,
             "kernels_ms": kern_ms,
-            "roofline": {"bound": "hbm", "kernel": "score_kernel", "achieved": score_gbs, "peak": peak,
-                         "unit": "GB/s", "frac": score_gbs / peak, "traffic": traffic,
-                         "algorithmic_bytes_per_launch": score_bytes, "peak_source": peak_src,
-                         "step": {"what": "the whole decode step (4 kernels): ids + norms + 2 k d 2 bytes per kv "
+            "roofline": {"bound": "hbm", "kernel": dom_kernel, "achieved": dom_gbs, "peak": peak,
+                         "unit": "GB/s", "frac": dom_gbs / peak, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": dom_bytes, "peak_source": peak_src,
+                         "step": {"what": "the whole decode step: ids + norms + 2 k d 2 bytes per kv "
                                           "head, over ms_per_step", "achieved": bytes_step / (ms_step * 1e-3) / 1e9,
                                   "frac": bytes_step / (ms_step * 1e-3) / 1e9 / peak, "bytes": bytes_step,
                                   "target_frac": 0.70},
-                         "attention_gbs": attn_bytes / (kern_ms["attention"] * 1e-3) / 1e9},
-            "gpu_launches": nk * K,
+                         "attention_gbs": attn_gbs},
+            "gpu_launches": kernels_per_step(path, w.L) * K,
+            "step_kernels": list(kern_ms),
             "clocks": clocks.summary(),
             "prefill": prefill,
             "per_head": per_head,

@@ -416,6 +416,22 @@ uint32_t socket_set_wait_limit(uint32_t polls);
 #define SOCKET_PATH_SEPARATE 1
 int socket_set_selection_path(int path);
 
+/*
+ * socket_last_decode_path -- diagnostic.  Which kernels the calling host
+ * thread's most recent successful socket_decode, socket_decode_static,
+ * socket_decode_append or socket_decode_per_head launched:
+ *   SOCKET_STEP_SEPARATE (0): soft tables, scoring, top-k, attention;
+ *   SOCKET_STEP_FUSED (1): soft tables, scoring, fused selection + attention;
+ *   SOCKET_STEP_ONE_KERNEL (2): the whole step in one kernel.
+ * -1 if the thread has made no such call, or its last one failed before it
+ * launched anything.  Timing tools use it to name the intervals between the
+ * events of socket_set_step_events.  No counterpart in the method.
+ */
+#define SOCKET_STEP_SEPARATE   0
+#define SOCKET_STEP_FUSED      1
+#define SOCKET_STEP_ONE_KERNEL 2
+int socket_last_decode_path(void);
+
 /* socket_version -- ABI version of this library (major * 100 + minor). */
 int socket_version(void);
 

@@ -22,7 +22,7 @@ __all__ = [
     "SocketError", "socket_hash_keys", "socket_decode", "socket_decode_static", "socket_decode_workspace_size",
     "socket_decode_per_head", "socket_decode_per_head_workspace_size", "socket_hash_check", "socket_decode_append",
     "socket_last_error", "socket_version", "socket_ids_row_bytes", "ids_shape", "socket_set_step_events",
-    "socket_set_wait_limit", "socket_set_selection_path", "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
+    "socket_set_wait_limit", "socket_set_selection_path", "socket_last_decode_path", "socket_shard_select", "socket_shard_merge", "socket_shard_attend",
     "socket_shard_attend_workspace_size", "socket_shard_combine", "library_path", "load_library",
     "alloc_cache_index", "alloc_decode_buffers",
 ]
@@ -100,6 +100,8 @@ def load_library(path: str | None = None):
     lib.socket_set_wait_limit.restype = ctypes.c_uint32
     lib.socket_set_selection_path.argtypes = [_int]
     lib.socket_set_selection_path.restype = _int
+    lib.socket_last_decode_path.argtypes = []
+    lib.socket_last_decode_path.restype = _int
     lib.socket_ids_row_bytes.argtypes = [_int]
     lib.socket_ids_row_bytes.restype = _int
     lib.socket_version.argtypes = []
@@ -443,6 +445,17 @@ def socket_set_selection_path(path: int) -> int:
     if prev < 0:
         raise SocketError(SOCKET_EINVAL, f"unknown selection path {path}")
     return prev
+
+
+SOCKET_STEP_SEPARATE, SOCKET_STEP_FUSED, SOCKET_STEP_ONE_KERNEL = 0, 1, 2
+
+
+def socket_last_decode_path() -> int:
+    """Kernels of this thread's last decode call: SOCKET_STEP_SEPARATE (soft
+    tables, scoring, top-k, attention), SOCKET_STEP_FUSED (soft tables,
+    scoring, fused selection + attention) or SOCKET_STEP_ONE_KERNEL; -1 if
+    there was none, or it failed before launching."""
+    return int(load_library().socket_last_decode_path())
 
 
 # ----------------------------------------------------------------------------

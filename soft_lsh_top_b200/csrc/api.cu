@@ -196,6 +196,9 @@ std::atomic<uint32_t> g_wait_polls{kDefaultWaitPolls};
 uint32_t wait_poll_limit() { return g_wait_polls.load(std::memory_order_relaxed); }
 
 std::atomic<int> g_selection_path{SOCKET_PATH_AUTO};
+thread_local int g_last_path = -1;  // SOCKET_STEP_* of this thread's last decode, or -1
+
+void clear_last_decode_path() { g_last_path = -1; }
 
 bool pdl_enabled()
 {
@@ -253,6 +256,7 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
            float* app_vnorm = nullptr)
 {
     g_last_error.clear();
+    g_last_path = -1;
     DecodeShape s;
     int st = fill_shape(s, B, Hq, Hkv, Ncap, N, d, L, P, k);
     if (st != SOCKET_OK) return st;
@@ -297,6 +301,7 @@ int decode(bool per_head, const void* q, int q_dtype, const uint16_t* W, const u
     float2* part_ml = reinterpret_cast<float2*>(base + w.part_ml);
 
     if ((st = cuda_status(mark_step(0, cs), "step event record")) != SOCKET_OK) return st;
+    g_last_path = small ? SOCKET_STEP_ONE_KERNEL : fused ? SOCKET_STEP_FUSED : SOCKET_STEP_SEPARATE;
     if (small) {
         // One kernel for the whole step; the step's other events follow at once.
         st = cuda_status(launch_small_step(q, q_dtype, W, ids, vnorm, K, V, kv_dtype, s, tau, idx_out, out,
@@ -380,6 +385,8 @@ int socket_set_selection_path(int path)
     if (path != SOCKET_PATH_AUTO && path != SOCKET_PATH_SEPARATE) return -1;
     return g_selection_path.exchange(path);
 }
+
+int socket_last_decode_path(void) { return g_last_path; }
 
 int socket_hash_keys(const void* K, const void* V, int kv_dtype, int64_t B, int64_t Hkv, int64_t Ncap,
                      int64_t n_begin, int64_t n_end, int64_t d, const uint16_t* W, int L, int P, uint8_t* ids,

@@ -63,6 +63,9 @@ int attention_splits(int kv_dtype, int q_dtype, int G, int64_t U, int k, int num
 int attention_rows_per_cta(int k, int nsplit, int chunk);
 // Multiprocessors of the current device (looked up once per device).
 int device_num_sms();
+// Forgets the calling thread's last decode path (socket_last_decode_path
+// then returns -1 until a decode launches its kernels).
+void clear_last_decode_path();
 // Raises `func`'s dynamic shared-memory limit to `bytes` unless an earlier
 // call already did so on the current device (one runtime call per kernel and
 // device, not per launch).

@@ -57,6 +57,7 @@ extern "C" int socket_decode_static(const void* q, int q_dtype, const uint16_t* 
                                     void* stream)
 {
     using namespace socket_attn;
+    clear_last_decode_path();
     const size_t need = socket_decode_workspace_size(B, Hq, Hkv, Ncap, d, L, P, k);
     if (need > SOCKET_STATIC_WORKSPACE_BYTES) {
         char msg[320];

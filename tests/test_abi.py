@@ -115,6 +115,7 @@ def decode(lib, entry="socket_decode", **kw):
 def test_decode_rejects(lib, entry, kw, status):
     assert decode(lib, entry, **kw) == status
     assert lib.socket_last_error().decode() != ""
+    assert lib.socket_last_decode_path() == -1  # nothing launched
 
 
 @pytest.mark.parametrize("n_new", [0, -1, 65, 9])

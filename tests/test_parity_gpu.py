@@ -293,6 +293,7 @@ def test_batch8_128k_sampled_units_and_needles():
     units = [0, 11, 27, 63]
     inp, ids, vnorm, orc_ids, orc_vn32 = _full_size(w, units)
     idx, _, _ = gpu_decode(inp, w, ids, vnorm)
+    assert sk.socket_last_decode_path() == sk.SOCKET_STEP_SEPARATE  # 64 units: the four kernels
     needles = inp["needles"]
     found = sum(int(torch.isin(needles[b, h].to(torch.int32), idx[b, h]).sum())
                 for b in range(w.B) for h in range(w.Hkv))

@@ -54,6 +54,10 @@ CASES = {
                                         seed=7309), False, True),
 }
 
+# The kernels each case takes by shape (socket_last_decode_path reports them).
+ONE, FUSED = sk.SOCKET_STEP_ONE_KERNEL, sk.SOCKET_STEP_FUSED
+EXPECTED_PATH = {name: (ONE if name.startswith("one_kernel") else FUSED) for name in CASES}
+
 
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_fused_and_separate_paths_agree(case):
@@ -66,8 +70,10 @@ def test_fused_and_separate_paths_agree(case):
     assert sk.socket_set_selection_path(sk.SOCKET_PATH_AUTO) == sk.SOCKET_PATH_AUTO
     try:
         idx_a, out_a, sc_a = gpu_decode(inp, w, ids, vnorm, per_head=per_head)
+        assert sk.socket_last_decode_path() == EXPECTED_PATH[case]
         sk.socket_set_selection_path(sk.SOCKET_PATH_SEPARATE)
         idx_s, out_s, sc_s = gpu_decode(inp, w, ids, vnorm, per_head=per_head)
+        assert sk.socket_last_decode_path() == sk.SOCKET_STEP_SEPARATE
     finally:
         sk.socket_set_selection_path(sk.SOCKET_PATH_AUTO)
     assert torch.equal(sc_a.view(torch.int32), sc_s.view(torch.int32))  # the same scoring kernels
