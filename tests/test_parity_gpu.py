@@ -124,6 +124,9 @@ def test_decode_append_hashes_and_decodes(case):
                                 out, scores_out=scores)
         torch.cuda.synchronize()
         assert sk.read_device_error(ws) == 0
+        # Keys appended in the call are hashed by the soft-table kernel, so such
+        # a step never runs as the one-kernel step.
+        assert sk.socket_last_decode_path() in (sk.SOCKET_STEP_SEPARATE, sk.SOCKET_STEP_FUSED)
         g_ids = rows_to_ids(ids.reshape(w.U, w.ncap // 32, -1, 32, 16).cpu().numpy(), w.L)
         g_vn = vnorm.reshape(w.U, w.ncap).cpu().numpy()
         check_decode(inp, w, g_ids, g_vn, units, idx, out, scores, N=n)
