@@ -80,3 +80,20 @@ def test_fused_and_separate_paths_agree(case):
     assert torch.equal(idx_a, idx_s)
     assert torch.all(idx_a[..., 1:] > idx_a[..., :-1])
     torch.testing.assert_close(out_a, out_s, rtol=1e-5, atol=1e-5)
+
+
+def test_last_decode_path_is_per_thread():
+    """socket_last_decode_path reports the calling host thread's own last
+    decode: another thread that made none sees -1."""
+    import threading
+
+    w = CASES["one_kernel_bf16_group4"][0]
+    inp = wl.make_inputs(w, DEV)
+    ids, vnorm = gpu_hash(inp, w)
+    gpu_decode(inp, w, ids, vnorm)
+    assert sk.socket_last_decode_path() == sk.SOCKET_STEP_ONE_KERNEL
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(sk.socket_last_decode_path()))
+    t.start()
+    t.join()
+    assert seen == [-1]
