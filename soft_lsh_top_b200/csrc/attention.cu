@@ -346,13 +346,14 @@ constexpr int kWCtasPerSm = 6;
 bool warp_path(int kv_dtype, int q_dtype, int G) { return kv_dtype == 1 && q_dtype == 1 && G <= 8; }
 
 // The unit's last CTA merges the splits' partials: head h is merged by warp
-// h % kWWarps with no CTA barrier.  Splits are taken 16 at a time, their
-// (m, l) pairs (split s in lane s) and 16-byte loads of their rows issued
+// h % kWWarps with no CTA barrier.  Splits are taken TILE at a time (16, or 32
+// when a unit has more than 16 splits: fewer round trips, more registers),
+// their (m, l) pairs (split s in lane s) and 16-byte loads of their rows issued
 // together; the weights w_s = exp(m_s - M) reach the other lanes by shuffle,
 // and each lane accumulates four output columns in split order, rescaling
 // when a later tile raises the running max M:
 // out = sum_s w_s o_s / sum_s w_s l_s with M = max_s m_s.
-template <int G>
+template <int G, int TILE>
 __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t pbase, int64_t qrow0,
                                                  const float* __restrict__ part_o, const float2* __restrict__ part_ml,
                                                  uint32_t* __restrict__ counters, float* __restrict__ out,
@@ -360,7 +361,7 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
 {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (!cta_ticket(&counters[u], (uint32_t)(nsplit - 1), s_last)) return;
-    constexpr int kTile = 16;  // splits whose rows are loaded at once
+    constexpr int kTile = TILE;  // splits whose rows are loaded at once
     for (int h = warp; h < G; h += kWWarps) {
         const int64_t base = pbase + h * nsplit;
         float M = -INFINITY, lsum = 0.0f;  // lsum: this lane's splits, at the running max M
@@ -409,7 +410,7 @@ __device__ __forceinline__ void merge_unit_warps(int64_t u, int nsplit, int64_t 
     if (tid == 0) counters[u] = 0u;
 }
 
-template <int G>
+template <int G, int TILE>
 __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ counts, int share, int64_t Ncap, int k,
@@ -519,7 +520,7 @@ __global__ __launch_bounds__(kWThreads) void attention_warp_kernel(
             }
         }
     }
-    merge_unit_warps<G>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, ml_out, s_last);
+    merge_unit_warps<G, TILE>(u, nsplit, pbase, qrow0, part_o, part_ml, counters, out, ml_out, s_last);
 }
 
 template <int G>
@@ -528,7 +529,10 @@ cudaError_t launch_warp(const void* q, const void* K, const void* V, const int32
                         float* out, float2* ml_out, cudaStream_t stream)
 {
     const int rpc = attention_rows_per_cta(s.k, s.nsplit, kWChunk);
-    auto kern = attention_warp_kernel<G>;
+    // The wide merge tile only where a unit has more than 16 splits: its
+    // registers would otherwise cost every shape (the kernel's CTAs share SMs
+    // with the top-k grid while they wait for it).
+    auto kern = s.nsplit > 16 ? attention_warp_kernel<G, 32> : attention_warp_kernel<G, 16>;
     cudaError_t e = set_smem_limit_once((const void*)kern, kWSmemBytes);
     if (e != cudaSuccess) return e;
     e = launch_pdl(kern, dim3((unsigned)(s.U * s.nsplit)), dim3(kWThreads), kWSmemBytes, stream,
