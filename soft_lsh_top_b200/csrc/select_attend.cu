@@ -281,7 +281,9 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
             uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
             auto bits_of = [&](int i) { return selc[i].y; };
             radix_digit(sh, nc, bits_of, 8, 0x7ffu, true, prefix, mask, need);
-            radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
+            // A bin holding exactly the keys still needed is kept whole: its
+            // lowest pattern is the threshold, with no ties to resolve.
+            if (sh.count != need) radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
             t = prefix;
             // Ties at t beyond `need`: the need lowest indices are kept, i.e. those
             // at or below the need-th smallest tie index ti (digits 30-20, 19-9,

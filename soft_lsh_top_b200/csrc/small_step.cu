@@ -264,9 +264,13 @@ __global__ __launch_bounds__(kThreads, 1) void small_step_kernel(const SmallArgs
     {
         uint32_t prefix = 0, mask = 0, krem = (uint32_t)k;
         auto get = [&](int i) { return scb[i]; };
+        // A digit's bin holding exactly the keys still needed is taken whole:
+        // its lowest pattern is the threshold and the later digits are skipped.
         radix_digit(sh, N, get, 20, 0x7ffu, true, prefix, mask, krem);
-        radix_digit(sh, N, get, 9, 0x7ffu, true, prefix, mask, krem);
-        radix_digit(sh, N, get, 0, 0x1ffu, true, prefix, mask, krem);
+        if (sh.count != krem) {
+            radix_digit(sh, N, get, 9, 0x7ffu, true, prefix, mask, krem);
+            if (sh.count != krem) radix_digit(sh, N, get, 0, 0x1ffu, true, prefix, mask, krem);
+        }
         const uint32_t t = prefix;
         // Keys above t, and the first krem keys equal to t, in index order
         // (tiles of 16 consecutive keys per thread, block-wide scans).

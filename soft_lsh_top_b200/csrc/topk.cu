@@ -340,8 +340,12 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
         uint32_t prefix = d0 << kScoreHistShift, mask = 0xffffffffu << kScoreHistShift, need = krem0;
         auto bits_of = [&](int i) { return scand[i].y; };
         radix_digit(sh, nc, bits_of, 8, 0x7ffu, true, prefix, mask, need);
-        radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
-        const uint32_t t = prefix, ties_total = sh.count;  // keys equal to t
+        // When the bin found holds exactly the keys still needed, all of them
+        // are kept: the threshold is the bin's lowest pattern, with no ties to
+        // resolve, and the last digit is skipped (the common case: a few
+        // hundred candidates spread over 2048 bins).
+        if (sh.count != need) radix_digit(sh, nc, bits_of, 0, 0xffu, true, prefix, mask, need);
+        const uint32_t t = prefix, ties_total = sh.count;  // keys equal to t (or the bin's keys, all kept)
         // Ties at t beyond `need`: keep the `need` lowest indices, i.e. those at
         // or below the need-th smallest tie index ti (digits 30-20, 19-9, 8-0 of
         // the ties' indices, ascending; non-ties map to 2^32 - 1 and never match).
