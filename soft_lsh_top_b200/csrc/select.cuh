@@ -17,6 +17,7 @@ struct Shared {
     uint32_t digit, krem, last;
     uint32_t count;  // keys in the bin found by the last digit; candidates of this CTA during the read
     uint32_t base;   // offset of this CTA's candidates in the unit list
+    uint32_t bin_count;  // keys in the bin find_bin found
     __align__(16) uint32_t hist[kBins];
 };
 
@@ -51,9 +52,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* w
 
 // Over bins given in descending order as per-thread runs c[0..NB) (thread
 // t's run precedes thread t+1's), finds the bin holding the krem-th key from
-// the top: writes its id (bin_of(q)) to sh.digit and the keys still needed
-// inside it to sh.krem.  Every thread must call it; sh is valid after the
-// next barrier.
+// the top: writes its id (bin_of(q)) to sh.digit, the keys still needed
+// inside it to sh.krem and the keys it holds to sh.bin_count.  Every thread
+// must call it; sh is valid after the next barrier.
 template <int NB, typename BinOf>
 __device__ __forceinline__ void find_bin(const uint32_t (&c)[NB], uint32_t krem, Shared& sh, BinOf bin_of)
 {
@@ -67,6 +68,7 @@ __device__ __forceinline__ void find_bin(const uint32_t (&c)[NB], uint32_t krem,
         if (run < krem && krem <= run + c[q]) {
             sh.digit = bin_of(q);
             sh.krem = krem - run;
+            sh.bin_count = c[q];
         }
         run += c[q];
     }

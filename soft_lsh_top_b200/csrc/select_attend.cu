@@ -134,6 +134,7 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
         sh.count = 0u;
         sh.digit = 0u;
         sh.krem = (uint32_t)a.k;
+        sh.bin_count = 0u;
     }
     for (int i = tid; i < Sw; i += kThreads) sure_w[i] = 0u;
     if (tid < kMaxSlices) kept_cnt[tid] = 0u;
@@ -149,8 +150,8 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
     // (lanes 8m .. 8m + 7 of a warp: the 32 keys of one bitmap word).  The
     // thread copies its 16 bytes of round g into ring stage g mod kRing (one
     // commit group per round, empty past the slice) and reads them back
-    // itself; the first kRing - 1 rounds are issued before the histogram is
-    // read.
+    // itself; the first kRing - 1 rounds are issued right after the
+    // histogram's loads, so they stream while d0 is found.
     const int rounds = (hi - lo + kRoundKeys - 1) / kRoundKeys;
     auto key_of = [&](int g) { return lo + g * kRoundKeys + 4 * tid; };
     const uint32_t my_slot = smem_addr(stages) + 16u * (uint32_t)tid;
@@ -159,26 +160,28 @@ __global__ __launch_bounds__(kThreads, 1) void select_attend_kernel(const FusedA
         if (g < rounds && n0 < hi) cp_async16(my_slot + (uint32_t)(g % kRing) * kRingStageBytes, su + n0);
         cp_async_commit();
     };
-#pragma unroll
-    for (int g = 0; g < kRing - 1; ++g) issue_round(g);
     {
         constexpr int kPer = kScoreHistBins / kThreads;  // 8 bins per thread, descending
         const int b0 = kScoreHistBins - 1 - kPer * tid;
         const uint4* hp = reinterpret_cast<const uint4*>(a.unit_hist + u * kScoreHistBins + (b0 - (kPer - 1)));
+        uint4 hw[kPer / 4];
+#pragma unroll
+        for (int qq = 0; qq < kPer / 4; ++qq) hw[qq] = __ldcg(hp + (kPer / 4 - 1 - qq));
+#pragma unroll
+        for (int g = 0; g < kRing - 1; ++g) issue_round(g);
         uint32_t c[kPer];
 #pragma unroll
         for (int qq = 0; qq < kPer / 4; ++qq) {
-            const uint4 w = __ldcg(hp + (kPer / 4 - 1 - qq));
-            c[4 * qq] = w.w;
-            c[4 * qq + 1] = w.z;
-            c[4 * qq + 2] = w.y;
-            c[4 * qq + 3] = w.x;
+            c[4 * qq] = hw[qq].w;
+            c[4 * qq + 1] = hw[qq].z;
+            c[4 * qq + 2] = hw[qq].y;
+            c[4 * qq + 3] = hw[qq].x;
         }
         find_bin<kPer>(c, (uint32_t)a.k, sh, [&](int qq) { return (uint32_t)(b0 - qq); });
         __syncthreads();
     }
     const uint32_t d0 = sh.digit, krem0 = sh.krem;
-    const uint32_t ncand = __ldcg(a.unit_hist + u * kScoreHistBins + d0);  // keys of the unit in bin d0
+    const uint32_t ncand = sh.bin_count;  // keys of the unit in bin d0
     const bool fits = ncand <= (uint32_t)a.cap;
 
     // ---- B. one read of the slice.

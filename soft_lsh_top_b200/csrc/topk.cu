@@ -138,41 +138,45 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
 
     // Load g of this thread covers keys lo + 2048 g + 4 tid .. + 3 (lanes
     // 8m .. 8m + 7 of a warp: the 32 keys of one bitmap word).  The first
-    // kInFlight loads are issued before the histogram is read.
+    // kInFlight loads are issued right after the histogram's, so they stream
+    // while d0 is found, without delaying the histogram behind them.
     auto key_of = [&](int g) { return lo + g * 4 * kThreads + 4 * tid; };
     auto load = [&](int g) {
         const int n0 = key_of(g);
         return n0 < hi ? __ldcg(reinterpret_cast<const uint4*>(su + n0)) : make_uint4(0, 0, 0, 0);
     };
     uint4 v[kInFlight];
-#pragma unroll
-    for (int g = 0; g < kInFlight; ++g) v[g] = load(g);
 
     // ---- the unit histogram: bin d0 of the k-th largest score.
     {
         constexpr int kPer = kScoreHistBins / kThreads;  // 8 bins per thread, descending
         const int b0 = kScoreHistBins - 1 - kPer * tid;
         const uint4* hp = reinterpret_cast<const uint4*>(a.unit_hist + u * kScoreHistBins + (b0 - (kPer - 1)));
+        uint4 hw[kPer / 4];
+#pragma unroll
+        for (int q = 0; q < kPer / 4; ++q) hw[q] = __ldcg(hp + (kPer / 4 - 1 - q));
+#pragma unroll
+        for (int g = 0; g < kInFlight; ++g) v[g] = load(g);
         uint32_t c[kPer];
 #pragma unroll
         for (int q = 0; q < kPer / 4; ++q) {
-            const uint4 w = __ldcg(hp + (kPer / 4 - 1 - q));
-            c[4 * q] = w.w;
-            c[4 * q + 1] = w.z;
-            c[4 * q + 2] = w.y;
-            c[4 * q + 3] = w.x;
+            c[4 * q] = hw[q].w;
+            c[4 * q + 1] = hw[q].z;
+            c[4 * q + 2] = hw[q].y;
+            c[4 * q + 3] = hw[q].x;
         }
         if (tid == 0) {
             sh.digit = 0;
             sh.krem = (uint32_t)a.k;
             sh.count = 0;
+            sh.bin_count = 0;
         }
         __syncthreads();
         find_bin<kPer>(c, (uint32_t)a.k, sh, [&](int q) { return (uint32_t)(b0 - q); });
         __syncthreads();
     }
     const uint32_t d0 = sh.digit, krem0 = sh.krem;
-    const uint32_t ncand = __ldcg(a.unit_hist + u * kScoreHistBins + d0);  // keys of the unit in bin d0
+    const uint32_t ncand = sh.bin_count;  // keys of the unit in bin d0
     const bool fits = ncand <= (uint32_t)a.cap;
 
     // ---- one read of the slice: bitmap words, and the candidates into
