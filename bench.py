@@ -95,6 +95,7 @@ class ClockSampler:
         self.samples = []
         self.reasons = 0
         self.error = None
+        self.errors = 0
         self._stop = threading.Event()
         self._thread = None
         try:
@@ -126,13 +127,24 @@ class ClockSampler:
         self.samples.append(mhz)
         self.reasons |= int(r) & ~0x1
 
+    def sample_now(self):
+        """One sample from the calling thread (while queued GPU work runs)."""
+        if self.error is None or self.samples:
+            try:
+                self._sample()
+            except Exception as e:
+                self.errors += 1
+                self.error = f"{type(e).__name__}: {e}"
+
     def _run(self):
+        # A failed query is recorded and sampling goes on (one NVML error must
+        # not end the clock record of the timed region).
         while not self._stop.is_set():
             try:
                 self._sample()
             except Exception as e:
+                self.errors += 1
                 self.error = f"{type(e).__name__}: {e}"
-                return
             time.sleep(self.period)
 
     def __enter__(self):
@@ -153,9 +165,13 @@ class ClockSampler:
     def summary(self):
         if self.error is not None and not self.samples:
             return {"error": self.error}
-        return {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
-                "sm_max_mhz": float(self.max_mhz), "samples": len(self.samples),
-                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+        out = {"sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+               "sm_max_mhz": float(self.max_mhz), "samples": len(self.samples),
+               "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+        if self.errors:
+            out["query_errors"] = self.errors
+            out["last_error"] = self.error
+        return out
 
 
 def max_over_ranks(x: float, world: int) -> float:
@@ -445,6 +461,7 @@ def run_socket(args, world: int, rank: int, local_rank: int):
         else:
             for s in range(K):
                 step(s)
+        clocks.sample_now()  # the queue still holds most of the steps
         end.record()
         torch.cuda.synchronize()
     graph = None
