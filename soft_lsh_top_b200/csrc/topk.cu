@@ -125,7 +125,13 @@ __global__ __launch_bounds__(kThreads, 2) void topk_kernel(const TopkArgs a)
     uint32_t* sbits = reinterpret_cast<uint32_t*>(topk_dyn + sizeof(uint2) * a.cap);  // [kTileWords]
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t u = blockIdx.x / a.C;
-    const int r = blockIdx.x % a.C;
+    // With many slices per unit, consecutive CTAs (which tend to share an SM:
+    // the grid is placed two per SM as the scoring grid's CTAs leave) take
+    // slices from opposite ends of the unit, so that where keys drift along a
+    // long sequence the crowded late slices share SMs with sparse early ones.
+    // With few slices the plain order measured faster.
+    const int b = blockIdx.x % a.C;
+    const int r = !SPREAD ? b : (b & 1) ? a.C - 1 - (b >> 1) : (b >> 1);
     const bool single = a.C == 1;  // one CTA holds the whole unit: bitmap and candidates stay in shared memory
     const uint32_t* su = reinterpret_cast<const uint32_t*>(a.scores + u * a.Ncap);
     uint32_t* bm = a.bitmap + u * a.bm_stride;  // 16-byte aligned rows
