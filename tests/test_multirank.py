@@ -67,3 +67,20 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_launch_count_follows_the_step_path():
+    """gpu_launches in the bench line counts the kernels of the path the step
+    took: four on the separate path (one more scoring launch per further 64
+    tables), three with the fused selection + attention kernel, one for the
+    one-kernel step."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import soft_lsh_top_b200 as sk
+
+    assert bench.kernels_per_step(sk.SOCKET_STEP_SEPARATE, 32) == 4
+    assert bench.kernels_per_step(sk.SOCKET_STEP_SEPARATE, 64) == 4
+    assert bench.kernels_per_step(sk.SOCKET_STEP_SEPARATE, 80) == 5
+    assert bench.kernels_per_step(sk.SOCKET_STEP_SEPARATE, 128) == 5
+    assert bench.kernels_per_step(sk.SOCKET_STEP_FUSED, 60) == 3
+    assert bench.kernels_per_step(sk.SOCKET_STEP_ONE_KERNEL, 16) == 1
