@@ -265,3 +265,22 @@ def test_sharded_calls_reject_bad_arguments_on_the_host(lib):
     assert lib.socket_shard_attend(f, 1, f, f, 1, 1, 4, 1, 64, 128, 8, f, f, f, 16, f, f, None) == EWS
     assert lib.socket_shard_combine(f, f, 2, 1, 4, 64, f, None) == EUNSUP
     assert lib.socket_shard_combine(f, f, 0, 1, 4, 128, f, None) == EINVAL
+
+
+@pytest.mark.parametrize("L, expect", [(16, 36 / 512), (32, 36 / 512), (60, 68 / 512), (80, 100 / 512)])
+def test_index_memory_overhead(L, expect):
+    """The cached index (id rows of socket_ids_row_bytes(L) bytes plus a
+    float32 value norm per key) against the bf16 key and value rows it sits
+    beside: (Lr + 4) / (2 d 2).  The pages report about 15 % over the KV
+    cache ([ES] "Resultados Experimentales", "Sobrecarga de Memoria"; [DE]
+    "Experimentelle Ergebnisse", "Speicher-Overhead") without naming L; the
+    workloads here (L = 32 and 60) come to 7.0 % and 13.3 %."""
+    import soft_lsh_top_b200 as sk
+
+    B, Hkv, Ncap = 2, 3, 4096
+    ids, vnorm = sk.alloc_cache_index(B, Hkv, Ncap, L, "cpu")
+    index_bytes = ids.numel() * ids.element_size() + vnorm.numel() * vnorm.element_size()
+    kv_bytes = 2 * B * Hkv * Ncap * sk.HEAD_DIM * 2
+    assert index_bytes / kv_bytes == pytest.approx(expect, rel=1e-12)
+    if L in (32, 60):
+        assert index_bytes / kv_bytes < 0.15
