@@ -84,3 +84,27 @@ def test_launch_count_follows_the_step_path():
     assert bench.kernels_per_step(sk.SOCKET_STEP_SEPARATE, 128) == 5
     assert bench.kernels_per_step(sk.SOCKET_STEP_FUSED, 60) == 3
     assert bench.kernels_per_step(sk.SOCKET_STEP_ONE_KERNEL, 16) == 1
+
+
+def test_step_kernel_times_are_named_by_path():
+    """The bench names the intervals between a step's events after the kernels
+    its path launched (the library records events 1..4 right after the last
+    kernel when a path has fewer than four)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import soft_lsh_top_b200 as sk
+
+    class Ev:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    stamps = [0.0, 1.0, 3.0, 6.0, 10.0]  # intervals 1, 2, 3, 4 ms
+    evs = [[Ev(t) for t in stamps] for _ in range(3)]
+    assert bench.step_kernel_times(evs, 3, sk.SOCKET_STEP_SEPARATE) == {
+        "soft_tables": 1.0, "score": 2.0, "topk": 3.0, "attention": 4.0}
+    assert bench.step_kernel_times(evs, 3, sk.SOCKET_STEP_FUSED) == {
+        "soft_tables": 1.0, "score": 2.0, "select_attend": 3.0}
+    assert bench.step_kernel_times(evs, 3, sk.SOCKET_STEP_ONE_KERNEL) == {"small_step": 1.0}
