@@ -20,7 +20,9 @@
 // candidates (index, bit pattern) to the unit's candidate list.  The last CTA
 // of the unit to finish (an atomic ticket; nobody waits) then
 //   * radix-selects the exact k-th bit pattern t among the candidates (two
-//     more digits) and the number of keys equal to t still to take,
+//     more digits; one when the first digit's bin holds exactly the keys
+//     still needed, which are then all kept) and the number of keys equal to
+//     t still to take,
 //   * clears the bitmap bits of the candidates below t, and of the ties at t
 //     beyond that number (the lowest indices are kept: a radix select over
 //     the ties' indices when they do not all fit),
